@@ -1,0 +1,316 @@
+"""Pins of the float64 oracle against facts fixed outside the oracle itself.
+
+Each pin_* function raises AssertionError when the oracle disagrees with a
+hand-worked example (tests/golden/hand_examples.json), a closed form, an
+invariant of the definitions, or a brute-force restatement on tiny inputs.
+test_oracle_pins.py runs them against the oracle; test_oracle_mutants.py runs
+them against deliberately broken copies of the oracle and requires every copy
+to fail at least one pin.
+
+Definitions pinned (TokenSelect GitHub README, "Key Takeaways"; GrooveSquid
+summary of the TokenSelect paper): per-head Q.K criticality, per-head softmax
+over tokens summed over heads (soft vote), top-k selection with sink and local
+windows (ties to the lower id), Selection Cache by cosine of consecutive
+queries, attention over the selected tokens.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_examples.json")
+SCALES = {"ln2/2": math.log(2.0) / 2.0, "ln3/2": math.log(3.0) / 2.0}
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _bits(x) -> np.ndarray:
+    """Exact bf16 bits of small integers / floats given as nested lists."""
+    t = torch.tensor(x, dtype=torch.float64).to(torch.bfloat16)
+    assert torch.equal(t.to(torch.float64), torch.tensor(x, dtype=torch.float64)), "not exact in bf16"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _frac(lst):
+    return np.array([float(Fraction(s)) for s in lst])
+
+
+def _rand_case(seed, n, h_q, h_kv, d, dist="normal"):
+    k, v = W.random_kv(n, h_kv, d, seed, dist=dist)
+    g = torch.Generator().manual_seed(seed + 7)
+    q = torch.randn((h_q, d), generator=g).to(torch.bfloat16)
+    return W.bf16_bits(k), W.bf16_bits(v), W.bf16_bits(q)
+
+
+# ---------------------------------------------------------------- scoring
+
+
+def pin_logits_default_scale():
+    c = _golden()["logits_default_scale"]
+    k, q = _bits(c["k"]), _bits(c["q"])
+    s = oracle.head_logits(k, q, 0)
+    assert np.array_equal(s, _frac(c["logits"])), s
+
+
+def pin_softmax_powers_of_two():
+    c = _golden()["softmax_powers_of_two"]
+    k, q = _bits(c["k"]), _bits(c["q"])
+    s = oracle.head_logits(k, q, 0, SCALES[c["scale"]])
+    p, L = oracle.softmax_row(s)
+    assert np.allclose(p, _frac(c["p"]), rtol=0, atol=1e-14), p
+    assert abs(L - math.log(15.0)) < 1e-13, L          # L = ln(1+2+4+8)
+
+
+def pin_soft_vote_two_heads():
+    c = _golden()["soft_vote_two_heads"]
+    v, L = oracle.votes(_bits(c["k"]), _bits(c["q"]), SCALES[c["scale"]])
+    assert np.allclose(v, _frac(c["v"]), rtol=0, atol=1e-14), v
+
+
+def pin_gqa_contiguous_groups():
+    c = _golden()["gqa_contiguous_groups"]
+    v, L = oracle.votes(_bits(c["k"]), _bits(c["q"]), SCALES[c["scale"]])
+    assert np.allclose(v, _frac(c["v"]), rtol=0, atol=1e-14), v
+
+
+def pin_votes_sum_to_heads():
+    """Each head's softmax sums to 1, so the votes sum to h_q."""
+    for seed, (n, hq, hk, d) in enumerate([(97, 4, 2, 64), (300, 28, 4, 128), (1, 8, 8, 64),
+                                           (513, 6, 3, 64), (64, 32, 8, 128)]):
+        k, _, q = _rand_case(seed, n, hq, hk, d)
+        v, L = oracle.votes(k, q)
+        assert abs(v.sum() - hq) < 1e-12 * hq, (v.sum(), hq)
+        assert (v >= 0).all()
+        for h in range(hq):
+            p, _ = oracle.softmax_row(oracle.head_logits(k, q, h))
+            assert abs(p.sum() - 1.0) < 1e-13
+
+
+def pin_identical_keys_uniform():
+    """Identical keys: every head is uniform, v = h_q / n exactly (up to rounding)."""
+    k, _ = W.random_kv(50, 2, 64, 3, dist="const")
+    q = torch.randn((6, 64), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    v, _ = oracle.votes(W.bf16_bits(k), W.bf16_bits(q))
+    assert np.allclose(v, 6.0 / 50.0, rtol=1e-14, atol=0), v
+
+
+def pin_single_token():
+    k, _, q = _rand_case(11, 1, 4, 2, 64)
+    v, _ = oracle.votes(k, q)
+    assert v.shape == (1,) and abs(v[0] - 4.0) < 1e-14
+
+
+def pin_large_logits_stable():
+    """Logits in the thousands: the max shift keeps the softmax finite."""
+    k = _bits([[[60.0] * 64], [[59.0] * 64], [[-60.0] * 64]])
+    q = _bits([[60.0] * 64])
+    v, L = oracle.votes(k, q)
+    assert np.isfinite(v).all() and abs(v.sum() - 1.0) < 1e-12
+    # logits are 60*60*64/8 = 28800, 28320 and -28800: the last is e^-57600 below -> 0
+    assert abs(v[0] - 1.0) < 1e-12 and v[2] == 0.0
+    assert abs(L[0] - 28800.0) < 1e-9
+
+
+def pin_strided_layout():
+    """A padded layout (junk 1e4 in the gaps) gives the same results as the dense one."""
+    n, hk, d, hq = 77, 2, 64, 4
+    kd, vd = W.random_kv(n, hk, d, 21)
+    kp, vp = W.random_kv(n, hk, d, 21, stride_tok=3 * hk * d + 8, stride_head=d + 40)
+    assert torch.equal(kd.float(), kp.float()) and torch.equal(vd.float(), vp.float())
+    q = torch.randn((hq, d), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    qb = W.bf16_bits(q)
+    a, La = oracle.votes(W.bf16_bits(kd), qb)
+    b, Lb = oracle.votes(W.bf16_bits(kp), qb)
+    assert np.array_equal(a, b) and np.array_equal(La, Lb)
+    ids = np.array([0, 5, 9, 40, 76], np.int32)
+    oa = oracle.sparse_attn(W.bf16_bits(kd), W.bf16_bits(vd), qb, ids)
+    ob = oracle.sparse_attn(W.bf16_bits(kp), W.bf16_bits(vp), qb, ids)
+    assert np.array_equal(oa, ob)
+
+
+# ---------------------------------------------------------------- selection
+
+
+def _brute_select(v, k, s, l):
+    """Rank counting: candidate i is in T iff fewer than k candidates precede it
+    in (vote desc, id asc) order.  O(n^2), no sorting."""
+    n = v.size
+    s_end = min(s, n)
+    l0 = max(n - l, s_end)
+    chosen = np.zeros(n, bool)
+    chosen[:s_end] = True
+    chosen[l0:] = True
+    c = np.arange(s_end, l0)
+    if c.size and k > 0:
+        vc = v[c]
+        before = (vc[None, :] > vc[:, None]) | ((vc[None, :] == vc[:, None]) & (c[None, :] < c[:, None]))
+        rank = before.sum(axis=1)
+        chosen[c[rank < k]] = True
+    return np.nonzero(chosen)[0].astype(np.int32)
+
+
+def pin_select_hand_example():
+    c = _golden()["select_with_ties"]
+    ids, m = oracle.select(np.array(c["votes"], np.float64), c["k"], c["n_sink"], c["n_local"])
+    assert m == c["count"] and ids.tolist() == c["ids"], (ids, m)
+
+
+def pin_windows():
+    for n, s, l, se, lb in _golden()["windows"]["cases"]:
+        assert oracle.windows(n, s, l) == (se, lb), (n, s, l, oracle.windows(n, s, l))
+
+
+def pin_select_brute_force(seeds=1000):
+    rng = np.random.default_rng(12345)
+    for _ in range(seeds):
+        n = int(rng.integers(0, 65))
+        k = int(rng.integers(0, 24))
+        s = int(rng.integers(0, 6))
+        l = int(rng.integers(0, 10))
+        v = np.round(rng.random(n) * rng.choice([4, 16, 1 << 20])) / 8.0   # many ties
+        ids, m = oracle.select(v, k, s, l)
+        want = _brute_select(v, k, s, l)
+        assert m == want.size and np.array_equal(ids[:m], want), (n, k, s, l)
+        assert (ids[m:] == -1).all()
+
+
+def pin_select_all_equal():
+    """All-equal votes: the tie-break takes the lowest candidate ids."""
+    n, k, s, l = 40, 7, 3, 5
+    ids, m = oracle.select(np.full(n, 0.25), k, s, l)
+    want = list(range(0, s)) + list(range(s, s + k)) + list(range(n - l, n))
+    assert m == len(want) and ids[:m].tolist() == want
+
+
+def pin_select_counts():
+    for n, k, s, l in [(100, 10, 4, 20), (20, 10, 4, 20), (24, 10, 4, 20), (30, 10, 4, 20),
+                       (0, 5, 1, 1), (5, 0, 0, 0), (50, 100, 0, 0)]:
+        ids, m = oracle.select(np.linspace(0, 1, n), k, s, l)
+        assert m == min(n, k + s + l), (n, k, s, l, m)
+        assert np.all(np.diff(ids[:m]) > 0)
+
+
+def pin_planted_keys_selected():
+    """Planted query-aligned keys carry the top votes and are always selected."""
+    cfg = W.CONFIGS["tiny"]
+    li = W.layer_inputs(cfg)
+    k, q = W.bf16_bits(li.k), W.bf16_bits(li.q[0, 0])
+    v, _ = oracle.votes(k, q)
+    ids, m = oracle.select(v, cfg.k, cfg.n_sink, cfg.n_local)
+    assert set(li.planted[0].tolist()) <= set(ids[:m].tolist())
+    top = np.argsort(-v, kind="stable")[:len(li.planted[0])]
+    assert set(top.tolist()) == set(li.planted[0].tolist())
+
+
+# ---------------------------------------------------------------- attention
+
+
+def pin_attention_two_tokens():
+    c = _golden()["attention_two_tokens"]
+    out = oracle.sparse_attn(_bits(c["k"]), _bits(c["v"]), _bits(c["q"]),
+                             np.array([0, 1], np.int32), scale=SCALES[c["scale"]])
+    want = np.array([[float(Fraction(x)) for x in row] for row in c["out"]])
+    assert np.allclose(out, want, rtol=0, atol=1e-13), out
+    dense = oracle.dense_attn(_bits(c["k"]), _bits(c["v"]), _bits(c["q"]), scale=SCALES[c["scale"]])
+    assert np.allclose(dense, want, rtol=0, atol=1e-13), dense
+
+
+def pin_attention_single_row():
+    """One selected row: every head's output is that row of its kv head's V."""
+    k, v, q = _rand_case(31, 20, 6, 3, 64)
+    for j in (0, 7, 19):
+        out = oracle.sparse_attn(k, v, q, np.array([j], np.int32))
+        vf = torch.from_numpy(v.astype(np.int16)).view(torch.bfloat16).double().numpy()
+        for h in range(6):
+            assert np.array_equal(out[h], vf[j, h // 2]), (j, h)
+
+
+def pin_full_selection_is_dense():
+    """k >= |candidates| selects every token: sparse attention = dense attention."""
+    for seed, (n, hq, hk, d) in enumerate([(90, 4, 2, 64), (33, 28, 4, 128), (5, 2, 2, 64)]):
+        k, v, q = _rand_case(40 + seed, n, hq, hk, d)
+        vv, _ = oracle.votes(k, q)
+        ids, m = oracle.select(vv, n, 4, 8)
+        assert m == n
+        sp = oracle.sparse_attn(k, v, q, ids, m)
+        de = oracle.dense_attn(k, v, q)
+        assert np.allclose(sp, de, rtol=0, atol=1e-12)
+
+
+def pin_mha_is_per_head():
+    """h_q == h_kv: each head attends with its own K/V head only."""
+    k, v, q = _rand_case(51, 30, 3, 3, 64)
+    ids = np.arange(0, 30, 3, dtype=np.int32)
+    full = oracle.sparse_attn(k, v, q, ids)
+    for h in range(3):
+        one = oracle.sparse_attn(np.ascontiguousarray(k[:, h:h + 1]), np.ascontiguousarray(v[:, h:h + 1]),
+                                 np.ascontiguousarray(q[h:h + 1]), ids)
+        assert np.array_equal(full[h], one[0])
+
+
+# ---------------------------------------------------------------- selection cache
+
+
+def pin_selcache_cases():
+    a = _bits([1.0, 0.0, 0.0, 0.0])
+    b = _bits([1.0, 1.0, 0.0, 0.0])
+    o = _bits([0.0, 1.0, 0.0, 0.0])
+    assert abs(oracle.cosine(a, b) - 1.0 / math.sqrt(2.0)) < 1e-15
+    assert oracle.cosine(a, o) == 0.0
+    q = W.bf16_bits(torch.randn(3, 64, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16))
+    neg = (q ^ np.uint16(0x8000))                      # bf16 sign flip: -q exactly
+    assert abs(oracle.cosine(q, q) - 1.0) < 1e-15
+    assert abs(oracle.cosine(q, neg) + 1.0) < 1e-15
+
+    prev = q.copy().reshape(-1)
+    r, c = oracle.selcache(q, prev, first_step=False, theta=0.9)
+    assert r and abs(c - 1.0) < 1e-15
+    prev = neg.copy().reshape(-1)
+    r, c = oracle.selcache(q, prev, first_step=False, theta=0.9)
+    assert (not r) and abs(c + 1.0) < 1e-15
+    assert np.array_equal(prev, q.reshape(-1)), "q_prev must hold the current query afterwards"
+    prev = q.copy().reshape(-1)
+    r, c = oracle.selcache(q, prev, first_step=True, theta=-2.0)
+    assert not r, "the first step never reuses"
+    # "at or above": cosine exactly equal to theta reuses
+    prev = o.copy()
+    r, c = oracle.selcache(a, prev, first_step=False, theta=0.0)
+    assert r and c == 0.0
+    prev = o.copy()
+    r, c = oracle.selcache(a, prev, first_step=False, theta=1e-9)
+    assert not r
+
+
+def pin_ar1_reuse_rate():
+    """AR(1) queries q_t = rho q_{t-1} + e_t: the flattened cosine of consecutive
+    queries tends to rho*sqrt(V_{t-1}/V_t) with V_t = sum_{j<=t} rho^(2j)."""
+    cfg = W.CONFIGS["llama8b_b4"]
+    qs = W.queries(cfg)
+    T = qs.shape[0]
+    rho = cfg.ar_rho
+    prev = W.bf16_bits(qs[0]).copy()
+    got = np.zeros((T, cfg.batch))
+    for t in range(1, T):
+        cur = W.bf16_bits(qs[t])
+        for b in range(cfg.batch):
+            _, got[t, b] = oracle.selcache(cur[b], prev[b], False, cfg.theta)
+    Vt = np.cumsum(rho ** (2 * np.arange(T)))
+    want = rho * np.sqrt(Vt[:-1] / Vt[1:])
+    err = np.abs(got[1:].mean(axis=1) - want)
+    assert err.max() < 0.04, err.max()            # per-decision noise ~ 1/sqrt(h_q d) = 0.016
+    reuse = (got[1:] >= cfg.theta).mean()
+    assert 0.80 < reuse < 0.95, reuse
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
