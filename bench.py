@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""Decode layer-steps/s of the TokenSelect hot path on B200 (sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole decode hot path over one batch of synthetic
+input, for every layer of the workload: selection-cache decision (ts_selcache),
+soft vote (ts_score), top-k + sink/local selection (ts_select) and attention
+over the selected tokens (ts_sparse_attn), all through the C ABI.  The default
+workload is the Qwen2-7B-shaped single layer (B=1, h_q=28, h_kv=4, d=128,
+n=32768, k=2048 + 4 sink + 512 local).  Every step is replayed from CUDA graphs;
+inputs rotate over enough copies of the KV cache that each step reads data
+that is not in L2.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(the path has no cross-sequence exchange); the timed region is bracketed by
+barriers and the elapsed time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on the same workload (rank 0
+only): the pages ship no runnable implementation, so the oracle is the
+reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+LAUNCHES_PER_LAYER_STEP = 5     # selcache, score pass A, score pass B, select, attention
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="qwen7b_32k", choices=W.ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    big = a.workload in ("llama8b_b4", "ragged_b32", "qwen7b_1m")
+    if a.steps is None:
+        a.steps = {"reference": 10}.get(a.impl, 200 if big else 3000)
+    if a.warmup is None:
+        a.warmup = 3 if a.impl == "reference" else (10 if big else 50)
+    if a.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps are required")
+    return a
+
+
+# ---------------------------------------------------------------------------
+# process group
+# ---------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            if torch.cuda.is_available() and self.pg.get_backend() == "nccl":
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        dev = "cuda" if self.pg.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def aggregate(per_rank_units: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return per_rank_units * world / max_seconds
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML, sampled in a thread during the timed region)
+# ---------------------------------------------------------------------------
+
+_REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+REJECT_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id, props.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # NVML missing: clocks are reported as unavailable
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in _REASON_BITS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+        return False
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+    def rejected(self):
+        s = self.summary()
+        if self.reasons & REJECT_REASONS:
+            return True
+        return bool(s["sm_mhz"] and s["sm_max_mhz"] and s["sm_mhz"] < 0.6 * s["sm_max_mhz"] and not self.reasons)
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel_src: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "score_pass_a_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(kernel_src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("source_sha256") != digest:
+            return None
+        return rec.get("per_launch_bytes", {}).get(workload)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# workload set-up
+# ---------------------------------------------------------------------------
+
+class Workload:
+    def __init__(self, name: str, device):
+        import query_aware_kv_ts_b200 as ts
+        self.ts = ts
+        self.cfg = cfg = W.CONFIGS[name]
+        self.name = name
+        self.device = device
+        self.layers = []
+        for layer in range(cfg.layers):
+            li = W.layer_inputs(cfg, layer, device)
+            self.layers.append(li)
+        self.lengths = np.diff(self.layers[0].seq_offsets)
+        self.k_bytes = int(self.lengths.sum()) * cfg.h_kv * cfg.head_dim * 2            # per layer
+        per_step = self.k_bytes * cfg.layers
+        self.rotate = max(1, math.ceil(4 * L2_BYTES / per_step)) if per_step < 4 * L2_BYTES else 1
+        self.T = cfg.steps
+        # rotating copies of each layer's cache (identical contents)
+        self.kvs = []
+        for li in self.layers:
+            copies = []
+            for r in range(self.rotate):
+                k = li.k if r == 0 else li.k.clone()
+                v = li.v if r == 0 else li.v.clone()
+                copies.append(ts.KVCache(k, v, li.seq_offsets, cfg.h_q))
+            self.kvs.append(copies)
+        self.q = [li.q.to(device).contiguous() for li in self.layers]          # [T, B, h_q, d] per layer
+        self.bufs = [ts.StepBuffers(c[0], cfg.k, cfg.n_sink, cfg.n_local) for c in self.kvs]
+        self.theta = cfg.theta if cfg.theta is not None else 2.0   # 2.0: cosine never reaches it
+        self.period = self.rotate * self.T // math.gcd(self.rotate, self.T)
+
+    def k_rows_bytes(self):
+        """Algorithmic bytes of one full (non-reused) layer-step, all sequences."""
+        c = self.cfg
+        m = np.minimum(self.lengths, c.k + c.n_sink + c.n_local)
+        return self.k_bytes + int(m.sum()) * c.h_kv * c.head_dim * 2 * 2
+
+    # one layer-step through the public C ABI
+    def layer_step(self, layer: int, i: int):
+        ts, b = self.ts, self.bufs[layer]
+        kv = self.kvs[layer][i % self.rotate]
+        q = self.q[layer][i % self.T]
+        ts.ts_selcache(q, b.q_prev, b.reuse, False, self.theta, b.cos)
+        ts.ts_score(kv, q, b.reuse, b.votes, b.ws)
+        ts.ts_select(kv, b.votes, b.k, b.n_sink, b.n_local, b.reuse, b.ids, b.count, b.ws)
+        ts.ts_sparse_attn(kv, q, b.ids, b.count, b.out, b.ws)
+
+    def step(self, i: int):
+        for layer in range(self.cfg.layers):
+            self.layer_step(layer, i)
+
+    def capture(self, fn_per_index, count):
+        graphs = []
+        for i in range(count):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn_per_index(i)
+            graphs.append(g)
+        return graphs
+
+
+def time_graphs(graphs, K, W_):
+    for i in range(W_):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(K):
+        graphs[i % len(graphs)].replay()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / 1000.0
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_layer_step_fn(wl_cfg, li, max_tokens=None):
+    import oracle
+    off = li.seq_offsets
+    kb, vb = W.bf16_bits(li.k), W.bf16_bits(li.v)
+    qb = W.bf16_bits(li.q[0])
+    if max_tokens is not None and off[1] > max_tokens:
+        off = np.array([0, max_tokens], np.int64)
+        qb = qb[:1]
+    tokens = int(off[-1])
+
+    def run():
+        oracle.decode_step(kb, vb, off, qb, wl_cfg.k, wl_cfg.n_sink, wl_cfg.n_local)
+    return run, tokens
+
+
+def cpu_baseline(wl: Workload, budget_s: float):
+    """Oracle layer-steps/s on this host, one core, on whole layer-steps of the
+    workload when one fits the budget, else on a token sample of sequence 0."""
+    cfg = wl.cfg
+    li = wl.layers[0]
+    total = int(li.seq_offsets[-1])
+    run, tokens = oracle_layer_step_fn(cfg, li)
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    sample_desc = "whole %s layer-steps (%d tokens)" % (cfg.name, tokens)
+    scale = 1.0
+    if one > budget_s / 2:
+        run, tokens = oracle_layer_step_fn(cfg, li, max_tokens=32768)
+        scale = tokens / total
+        sample_desc = "%d-token sample of sequence 0 of a %s layer-step, scaled by tokens" % (tokens, cfg.name)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    value = n * scale / el
+    return {"value": value, "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
+            "sample": "%d x %s, float64 C oracle, 1 thread, %.1f s" % (n, sample_desc, el)}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_ours(a, d: Dist):
+    torch.cuda.set_device(d.local)
+    dev = torch.device("cuda", d.local)
+    d.init("nccl")
+    wl = Workload(a.workload, dev)
+    cfg = wl.cfg
+    ts = wl.ts
+
+    # eager warm-up (also configures kernel attributes before capture)
+    for i in range(2):
+        wl.step(i)
+    torch.cuda.synchronize()
+    graphs = wl.capture(wl.step, wl.period)
+
+    # ---- main timed region: whole steps ----
+    d.barrier()
+    torch.cuda.synchronize()
+    for attempt in range(2):
+        with ClockSampler(d.local) as clk:
+            el = time_graphs(graphs, a.steps, a.warmup)
+        if not clk.rejected():
+            break
+    d.barrier()
+    el_max = d.max(el)
+    layer_steps = a.steps * cfg.layers
+    value = aggregate(layer_steps, d.world, el_max)
+    ms_per_step = el_max / a.steps * 1000.0
+
+    # ---- dominant kernel alone: score pass A (all sequences scored) ----
+    def pass_a(i):
+        for layer in range(cfg.layers):
+            ts.ts_score_logits(wl.kvs[layer][i % wl.rotate], wl.q[layer][i % wl.T], None, wl.bufs[layer].ws)
+    ga = wl.capture(pass_a, wl.rotate)
+    Ka = max(a.steps, 20)
+    el_a = time_graphs(ga, Ka, a.warmup)
+    per_launch_s = el_a / (Ka * cfg.layers)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = wl.k_bytes / per_launch_s / 1e9
+    traffic = profile_traffic(os.path.join(ROOT, "query_aware_kv_ts_b200", "csrc", "score.cu"), a.workload)
+
+    # per-kernel breakdown (each kernel alone, same rotation)
+    def one(fn):
+        g = wl.capture(fn, wl.rotate)
+        return time_graphs(g, Ka, a.warmup) / (Ka * cfg.layers) * 1e6
+    kernels = {"score_pass_a_us": per_launch_s * 1e6}
+    kernels["score_pass_b_us"] = one(lambda i: [ts.ts_score_vote(wl.kvs[l][i % wl.rotate], None, wl.bufs[l].votes,
+                                                                 wl.bufs[l].ws) for l in range(cfg.layers)])
+    kernels["select_us"] = one(lambda i: [ts.ts_select(wl.kvs[l][i % wl.rotate], wl.bufs[l].votes, cfg.k, cfg.n_sink,
+                                                       cfg.n_local, None, wl.bufs[l].ids, wl.bufs[l].count,
+                                                       wl.bufs[l].ws) for l in range(cfg.layers)])
+    kernels["sparse_attn_us"] = one(lambda i: [ts.ts_sparse_attn(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T],
+                                                                 wl.bufs[l].ids, wl.bufs[l].count, wl.bufs[l].out,
+                                                                 wl.bufs[l].ws) for l in range(cfg.layers)])
+
+    # ---- end to end: pinned host query in, result out, every step ----
+    q_host = [q.cpu().pin_memory() for q in wl.q]
+    out_host = [torch.empty_like(b.out, device="cpu").pin_memory() for b in wl.bufs]
+    h2d = sum(q[0].numel() * q.element_size() for q in q_host)
+    d2h = sum(o.numel() * o.element_size() for o in out_host)
+    K_e2e = min(a.steps, 2000)
+
+    def e2e_step(i):
+        for layer in range(cfg.layers):
+            wl.q[layer][i % wl.T].copy_(q_host[layer][i % wl.T], non_blocking=True)
+        graphs[i % len(graphs)].replay()
+        for layer in range(cfg.layers):
+            out_host[layer].copy_(wl.bufs[layer].out, non_blocking=True)
+        torch.cuda.synchronize()
+    for i in range(a.warmup):
+        e2e_step(i)
+    d.barrier()
+    t0 = time.perf_counter()
+    for i in range(K_e2e):
+        e2e_step(i)
+    e2e_el = d.max(time.perf_counter() - t0)
+    e2e_value = aggregate(K_e2e * cfg.layers, d.world, e2e_el)
+
+    # reuse rate over one pass of the query sequence (selection-cache workloads)
+    reuse_rate = None
+    if cfg.theta is not None:
+        flags = []
+        for b in wl.bufs:
+            b.q_prev.zero_()
+        for i in range(wl.T):
+            for layer in range(cfg.layers):
+                wl.layer_step(layer, i)
+                flags.append(wl.bufs[layer].reuse.clone())
+        reuse_rate = float(torch.stack(flags).float().mean().item())
+
+    alg_bytes = wl.k_rows_bytes() * cfg.layers
+    result = {
+        "metric": "decode layer-steps/s (score+select+sparse-attn); HBM GB/s vs roofline",
+        "value": value,
+        "unit": "layer-steps/s",
+        "n_gpus": d.world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": a.workload, "batch": cfg.batch, "h_q": cfg.h_q, "h_kv": cfg.h_kv,
+                   "head_dim": cfg.head_dim, "n": int(wl.lengths.max()), "tokens_total": int(wl.lengths.sum()),
+                   "layers": cfg.layers, "k": cfg.k, "n_sink": cfg.n_sink, "n_local": cfg.n_local,
+                   "selection_cache_theta": cfg.theta, "parallelism": "replicas" if d.world > 1 else "single",
+                   "l2": "inputs larger than L2: %d rotating KV copies, %.0f MiB of K read per rotation"
+                         % (wl.rotate, wl.rotate * wl.k_bytes * cfg.layers / 2**20),
+                   "graphs": "every step replayed from a CUDA graph of the C-ABI calls"},
+        "step_hbm_gbs": alg_bytes / (el_max / a.steps) / 1e9 if cfg.theta is None else None,
+        "step_alg_bytes": alg_bytes,
+        "roofline": {"bound": "hbm", "kernel": "score pass A (ts_score_logits)", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "alg_bytes_per_launch": wl.k_bytes,
+                     "launch_us": per_launch_s * 1e6},
+        "kernels": kernels,
+        "e2e": {"value": e2e_value, "unit": "layer-steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "pinned host query copied in, graph of the C-ABI calls replayed, fp32 output copied "
+                       "out and synchronised, every step; host wall clock"},
+        "gpu_launches": a.steps * cfg.layers * LAUNCHES_PER_LAYER_STEP,
+        "clocks": clk.summary(),
+    }
+    if reuse_rate is not None:
+        result["reuse_rate"] = reuse_rate
+    if d.world == 1 and not a.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
+    del graphs, ga
+    d.close()
+    if d.rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(a, d: Dist):
+    """The float64 oracle as the reference arm: rank 0 times it on the host."""
+    if d.rank != 0:
+        return
+    cfg = W.CONFIGS[a.workload]
+    li = W.layer_inputs(cfg, 0, "cpu")
+    total = int(li.seq_offsets[-1])
+    run, tokens = oracle_layer_step_fn(cfg, li)
+    scale = 1.0
+    sample = "one whole %s layer-step (%d tokens) per step" % (cfg.name, tokens)
+    t0 = time.perf_counter()
+    run()
+    if time.perf_counter() - t0 > 2.0:
+        run, tokens = oracle_layer_step_fn(cfg, li, max_tokens=32768)
+        scale = tokens / total
+        sample = "%d-token sample of sequence 0 of a %s layer-step per step, scaled by tokens" % (tokens, cfg.name)
+    for _ in range(a.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        run()
+    el = time.perf_counter() - t0
+    value = a.steps * scale / el
+    res = {"impl": "reference", "metric": "decode layer-steps/s (score+select+sparse-attn); HBM GB/s vs roofline",
+           "value": value, "unit": "layer-steps/s", "n_gpus": d.world, "steps": a.steps, "warmup": a.warmup,
+           "ms_per_step": el / a.steps * 1000.0, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": a.workload, "batch": cfg.batch, "h_q": cfg.h_q, "h_kv": cfg.h_kv,
+                      "head_dim": cfg.head_dim, "n": cfg.n, "k": cfg.k, "n_sink": cfg.n_sink,
+                      "n_local": cfg.n_local},
+           "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    d = Dist()
+    if a.impl == "reference":
+        run_reference(a, d)
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    run_ours(a, d)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,206 @@
+/*
+ * ts.h -- C ABI of libts, the B200 (sm_100a) TokenSelect decode-step library.
+ *
+ * TokenSelect picks, at every decode step and for every sequence, a small set
+ * of critical cached tokens and runs attention over those tokens only.  The
+ * method (TokenSelect GitHub README, section "Key Takeaways"; GrooveSquid
+ * summary of the TokenSelect paper, medium-difficulty summary):
+ *   1. criticality of each cached token, per query head, is the Query-Key dot
+ *      product                                             -> ts_score
+ *   2. per-head soft voting: each head's criticality is normalised by a
+ *      softmax over the tokens and the heads' results are summed -> ts_score
+ *   3. the highest-voted tokens, plus fixed sink and local windows, are
+ *      selected                                             -> ts_select
+ *   4. Selection Cache: when consecutive queries are similar the previous
+ *      selection is reused                                  -> ts_selcache
+ *   5. attention over the selected tokens                   -> ts_sparse_attn
+ *
+ * Conventions (every call):
+ *   - All pointers named *_dev or documented as "device" are CUDA device
+ *     memory owned by the caller.  libts never allocates device memory, keeps
+ *     no device state between calls except inside the caller's workspace, and
+ *     never synchronises the stream except in ts_get_device_status.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and target the current CUDA device.  Argument errors are
+ *     detected on the host and returned before anything is launched; launch
+ *     failures return TS_ERR_CUDA.  ts_last_error() describes the last error
+ *     of the calling thread.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns.  There is no CPU fallback:
+ *     every result is computed by sm_100a kernels.
+ *   - A workspace must not be used by two calls that can run concurrently.
+ */
+#ifndef TS_H_
+#define TS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TS_API __attribute__((visibility("default")))
+#else
+#define TS_API
+#endif
+
+typedef enum {
+    TS_OK = 0,
+    TS_ERR_INVALID_ARG = 1,     /* bad shape, pointer, alignment or value      */
+    TS_ERR_UNSUPPORTED = 2,     /* valid but outside what the kernels support  */
+    TS_ERR_WORKSPACE = 3,       /* workspace missing or smaller than required  */
+    TS_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed           */
+    TS_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait gave up          */
+} ts_status_t;
+
+/*
+ * One layer's KV cache for a (possibly ragged) batch, in token-major "NHD"
+ * layout: element (token t, kv head g, channel c) of K is at
+ *   k + t*stride_tok + g*stride_head + c        (in bf16 elements)
+ * where t runs over the concatenated tokens of all sequences; sequence b owns
+ * tokens [seq_offsets[b], seq_offsets[b+1]).  V has the same layout and
+ * strides.  Query head h reads kv head h / (h_q / h_kv) (contiguous GQA
+ * groups).
+ *
+ *   batch              >= 1 sequences
+ *   h_q, h_kv          query / kv heads; h_q % h_kv == 0;
+ *                      supported: h_kv in {1,2,4,8}, h_q/h_kv <= 16
+ *   head_dim           64 or 128
+ *   seq_offsets_dev    device int64 [batch+1], non-decreasing, [0] == 0
+ *   seq_offsets_host   host copy of the same (used for sizing and checks;
+ *                      must match seq_offsets_dev)
+ *   k, v               device bf16, 16-byte aligned
+ *   stride_tok,        in elements; multiples of 8; stride_head >= head_dim,
+ *   stride_head        stride_tok >= (h_kv-1)*stride_head + head_dim
+ *   scale              softmax scale; 0 selects 1/sqrt(head_dim)
+ */
+typedef struct ts_kv {
+    int32_t batch, h_q, h_kv, head_dim;
+    const int64_t *seq_offsets_dev;
+    const int64_t *seq_offsets_host;
+    const void *k;
+    const void *v;
+    int64_t stride_tok, stride_head;
+    float scale;
+} ts_kv_t;
+
+/*
+ * Workspace bytes needed by ts_score, ts_select and ts_sparse_attn for this
+ * cache shape and a selection of k top tokens plus n_sink + n_local window
+ * tokens (capacity k + n_sink + n_local).  The size depends on the current
+ * device's SM count.  Returns 0 when the arguments are invalid.
+ */
+TS_API size_t ts_workspace_bytes(const ts_kv_t *kv, int32_t k, int32_t n_sink, int32_t n_local);
+
+/*
+ * Zero the workspace's control block (device counters and the status word).
+ * Call once after allocating a workspace, before its first use, on the stream
+ * that will use it.  The library returns every counter to zero itself, so a
+ * workspace needs no re-initialisation between calls.
+ */
+TS_API ts_status_t ts_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Selection Cache decision (TokenSelect README, "Key Takeaways", Selection
+ * Cache: consecutive similar queries share one token selection).
+ * For each sequence b, over the flattened h_q*head_dim query vector:
+ *   cos_b    = <q_b, q_prev_b> / (|q_b| |q_prev_b|)     (float64 accumulation)
+ *   reuse[b] = !first_step && |q_b| > 0 && |q_prev_b| > 0 && cos_b >= threshold
+ * then q_prev_b <- q_b.
+ *   q          device bf16 [batch, h_q, head_dim] contiguous
+ *   q_prev     device bf16, same shape; caller-owned state, overwritten
+ *   reuse      device int32 [batch], written (0/1)
+ *   cos_out    device float64 [batch] or NULL; receives cos_b (0 on the first step)
+ */
+TS_API ts_status_t ts_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out,
+                        int32_t first_step, int32_t batch, int32_t h_q, int32_t head_dim,
+                        double threshold, void *stream);
+
+/*
+ * Soft vote (TokenSelect README, "Key Takeaways": per-head Q.K criticality,
+ * per-head softmax over tokens, summed over heads).  For every sequence b with
+ * reuse[b] == 0 and every token i in [0, n_b):
+ *   s[h,i] = scale * q[b,h,:] . K[b,i,h/G,:]
+ *   L[b,h] = log sum_i exp(s[h,i])
+ *   votes[seq_offsets[b] + i] = sum_h exp(s[h,i] - L[b,h])
+ * so the votes of a sequence sum to h_q.  Sequences with reuse[b] != 0 are
+ * skipped (their votes are left as they were).
+ *   q          device bf16 [batch, h_q, head_dim] contiguous
+ *   reuse      device int32 [batch] or NULL (NULL: score every sequence)
+ *   votes      device float32 [seq_offsets[batch]], written
+ * The float32 votes carry a relative error of a few 1e-7.
+ */
+TS_API ts_status_t ts_score(const ts_kv_t *kv, const void *q, const int32_t *reuse, float *votes,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The two phases of ts_score, callable separately (ts_score == ts_score_logits
+ * followed by ts_score_vote on the same stream and workspace):
+ *   ts_score_logits  per-head logits s[h,i] and log-normalisers L[b,h] into
+ *                    the workspace (one streaming pass over K)
+ *   ts_score_vote    votes from the workspace's logits and L
+ * Arguments as for ts_score.  The workspace carries the intermediate results
+ * from the first call to the second.
+ */
+TS_API ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reuse,
+                                   void *ws, size_t ws_bytes, void *stream);
+TS_API ts_status_t ts_score_vote(const ts_kv_t *kv, const int32_t *reuse, float *votes,
+                                 void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Token selection (TokenSelect README summary: a small number of critical KV
+ * tokens take part in attention).  For every sequence b with reuse[b] == 0:
+ *   sink  = [0, s')         s' = min(n_sink, n_b)
+ *   local = [l0, n_b)       l0 = max(n_b - n_local, s')
+ *   T     = the min(k, l0 - s') tokens of [s', l0) with the largest votes,
+ *           equal votes going to the lower token id
+ *   ids[b, 0:count[b]] = sink U T U local in ascending order (sequence-local
+ *   0-based ids), ids[b, count[b]:] = -1.
+ * Sequences with reuse[b] != 0 keep their previous ids and count.
+ *   votes      device float32 [seq_offsets[batch]] (non-negative, finite)
+ *   ids        device int32 [batch, k + n_sink + n_local]
+ *   count      device int32 [batch]
+ */
+TS_API ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink,
+                      int32_t n_local, const int32_t *reuse, int32_t *ids, int32_t *count,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Attention over the selected tokens:
+ *   out[b,h,:] = sum_j softmax_j(scale * q[b,h,:] . K[b,ids_j,h/G,:]) * V[b,ids_j,h/G,:]
+ * over j < count[b] (count[b] == 0 gives zeros).
+ *   ids        device int32 [batch, ids_capacity], ids in [0, n_b)
+ *   count      device int32 [batch], 0 <= count[b] <= ids_capacity
+ *   out        device float32 [batch, h_q, head_dim], written
+ */
+TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_t *ids,
+                           const int32_t *count, int32_t ids_capacity, float *out,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Read and clear the device status word of a workspace (synchronises the
+ * stream).  Returns TS_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave
+ * up since the last read, TS_OK otherwise.  *site_out (may be NULL) receives
+ * a code naming the wait that gave up.
+ */
+TS_API ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on a
+ * shared-memory barrier nobody arrives at, giving up after spin_limit polls;
+ * the give-up is recorded in the workspace status word (read it with
+ * ts_get_device_status).  Nothing else is touched.
+ */
+TS_API ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_limit, void *stream);
+
+TS_API const char *ts_status_string(ts_status_t status);
+
+/* Human-readable description of the calling thread's last error ("" if none). */
+TS_API const char *ts_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TS_H_ */

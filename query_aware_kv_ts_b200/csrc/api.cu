@@ -1,0 +1,460 @@
+// libts C ABI: argument validation, workspace layout, TMA descriptor set-up
+// and kernel launches.  No CPU fallback: every result comes from a kernel.
+#include <cudaTypedefs.h>
+
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "ts_device.cuh"
+#include "ts_internal.h"
+
+namespace ts {
+
+namespace {
+thread_local std::string g_last_error;
+
+int device_sms()
+{
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 0;
+        cached[dev] = sms;
+    }
+    return cached[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+ts_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return TS_ERR_CUDA;
+}
+}  // namespace
+
+void set_error(const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+}
+
+ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
+{
+    if (kv == nullptr) {
+        set_error("kv is NULL");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (kv->batch < 1 || kv->h_q < 1 || kv->h_kv < 1) {
+        set_error("batch, h_q and h_kv must be >= 1 (got %d, %d, %d)", kv->batch, kv->h_q, kv->h_kv);
+        return TS_ERR_INVALID_ARG;
+    }
+    if (kv->h_q % kv->h_kv != 0) {
+        set_error("h_q (%d) must be a multiple of h_kv (%d)", kv->h_q, kv->h_kv);
+        return TS_ERR_INVALID_ARG;
+    }
+    if (kv->head_dim != 64 && kv->head_dim != 128) {
+        set_error("head_dim must be 64 or 128 (got %d)", kv->head_dim);
+        return TS_ERR_UNSUPPORTED;
+    }
+    const int G = kv->h_q / kv->h_kv;
+    if (!(kv->h_kv == 1 || kv->h_kv == 2 || kv->h_kv == 4 || kv->h_kv == 8) || G > 16) {
+        set_error("supported: h_kv in {1,2,4,8} and h_q/h_kv <= 16 (got h_kv %d, group %d)", kv->h_kv, G);
+        return TS_ERR_UNSUPPORTED;
+    }
+    if (kv->batch > kMaxBatch) {
+        set_error("batch %d exceeds the supported maximum %d", kv->batch, kMaxBatch);
+        return TS_ERR_UNSUPPORTED;
+    }
+    if (kv->seq_offsets_dev == nullptr || kv->seq_offsets_host == nullptr) {
+        set_error("seq_offsets_dev and seq_offsets_host are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (kv->k == nullptr || kv->v == nullptr) {
+        set_error("k and v are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(kv->k) | reinterpret_cast<uintptr_t>(kv->v)) & 15u) {
+        set_error("k and v must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    const int D = kv->head_dim;
+    if (kv->stride_tok % 8 != 0 || kv->stride_head % 8 != 0 || kv->stride_head < D ||
+        kv->stride_tok < (int64_t)(kv->h_kv - 1) * kv->stride_head + D) {
+        set_error("strides (tok %lld, head %lld) must be multiples of 8 with stride_head >= head_dim and "
+                  "stride_tok >= (h_kv-1)*stride_head + head_dim",
+                  (long long)kv->stride_tok, (long long)kv->stride_head);
+        return TS_ERR_INVALID_ARG;
+    }
+    if (!isfinite(kv->scale)) {
+        set_error("scale must be finite");
+        return TS_ERR_INVALID_ARG;
+    }
+    const int64_t *off = kv->seq_offsets_host;
+    if (off[0] != 0) {
+        set_error("seq_offsets[0] must be 0");
+        return TS_ERR_INVALID_ARG;
+    }
+    int64_t n_max = 0;
+    for (int b = 0; b < kv->batch; ++b) {
+        const int64_t n = off[b + 1] - off[b];
+        if (n < 0) {
+            set_error("seq_offsets must be non-decreasing (sequence %d)", b);
+            return TS_ERR_INVALID_ARG;
+        }
+        n_max = n > n_max ? n : n_max;
+    }
+    const int64_t n_total = off[kv->batch];
+    if (n_total >= (int64_t(1) << 31)) {
+        set_error("total tokens %lld must be below 2^31", (long long)n_total);
+        return TS_ERR_UNSUPPORTED;
+    }
+    const int sms = device_sms();
+    if (sms <= 0) {
+        set_error("no CUDA device");
+        return TS_ERR_CUDA;
+    }
+
+    p->B = kv->batch;
+    p->Hq = kv->h_q;
+    p->Hkv = kv->h_kv;
+    p->G = G;
+    p->D = D;
+    p->n_total = n_total;
+    p->n_max = n_max;
+    p->scale = kv->scale != 0.0f ? kv->scale : (float)(1.0 / sqrt((double)D));
+    p->sms = sms;
+    p->tile_tokens = (kStageBytesTarget / 2) / (kv->h_kv * D);
+    p->stage_bytes = p->tile_tokens * kv->h_kv * D * 2;
+    p->chunk_tokens = p->tile_tokens;
+    int64_t chunks = 0, vblocks = 0;
+    for (int b = 0; b < kv->batch; ++b) {
+        const int64_t n = off[b + 1] - off[b];
+        chunks += (n + p->chunk_tokens - 1) / p->chunk_tokens;
+        vblocks += (n + kVoteTokensPerBlock - 1) / kVoteTokensPerBlock;
+    }
+    p->max_chunks = chunks;
+    p->score_grid = (int)(chunks < sms ? chunks : sms);
+    p->max_vote_blocks = vblocks;
+    p->capacity = capacity;
+    if (capacity > 0) {
+        int64_t want = (2 * (int64_t)sms + (int64_t)p->B * p->Hkv - 1) / ((int64_t)p->B * p->Hkv);
+        int64_t cap_splits = (capacity + 31) / 32;
+        p->attn_splits = (int)(want < 1 ? 1 : (want > cap_splits ? cap_splits : want));
+        if (p->attn_splits < 1)
+            p->attn_splits = 1;
+    } else {
+        p->attn_splits = 0;
+    }
+
+    size_t o = 0;
+    p->off_ctrl = o;
+    o += 256;
+    p->off_score_tickets = o;
+    o = align_up(o + sizeof(uint32_t) * p->B, 256);
+    p->off_attn_tickets = o;
+    o = align_up(o + sizeof(uint32_t) * p->B * p->Hkv, 256);
+    // everything above is the control block that ts_workspace_init zeroes
+    p->off_L = o;
+    o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
+    p->off_partials = o;
+    o = align_up(o + sizeof(float) * 2 * (size_t)(chunks > 0 ? chunks : 1) * p->Hq, 256);
+    p->off_logits = o;
+    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(n_total > 0 ? n_total : 1), 256);
+    p->off_attn_part = o;
+    if (capacity > 0)
+        o = align_up(o + sizeof(float) * (size_t)p->B * p->Hkv * p->attn_splits * p->G * (D + 2), 256);
+    p->total_bytes = o;
+    return TS_OK;
+}
+
+static ts_status_t check_ws(const Plan &p, void *ws, size_t ws_bytes)
+{
+    if (ws == nullptr) {
+        set_error("workspace is NULL");
+        return TS_ERR_WORKSPACE;
+    }
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) {
+        set_error("workspace must be 256-byte aligned");
+        return TS_ERR_WORKSPACE;
+    }
+    if (ws_bytes < p.total_bytes) {
+        set_error("workspace too small: %zu bytes given, %zu needed", ws_bytes, p.total_bytes);
+        return TS_ERR_WORKSPACE;
+    }
+    return TS_OK;
+}
+
+static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *map)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return TS_ERR_CUDA;
+    }
+    // dims (innermost first): channels, tokens, kv heads
+    cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.n_total, (cuuint64_t)p.Hkv};
+    cuuint64_t strides[2] = {(cuuint64_t)kv->stride_tok * 2, (cuuint64_t)kv->stride_head * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)p.tile_tokens, (cuuint32_t)p.Hkv};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(kv->k), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return TS_ERR_CUDA;
+    }
+    return TS_OK;
+}
+
+}  // namespace ts
+
+using namespace ts;
+
+extern "C" {
+
+size_t ts_workspace_bytes(const ts_kv_t *kv, int32_t k, int32_t n_sink, int32_t n_local)
+{
+    if (k < 0 || n_sink < 0 || n_local < 0)
+        return 0;
+    Plan p;
+    if (make_plan(kv, k + n_sink + n_local, &p) != TS_OK)
+        return 0;
+    return p.total_bytes;
+}
+
+ts_status_t ts_workspace_init(void *ws, size_t ws_bytes, void *stream)
+{
+    if (ws == nullptr || ws_bytes < 256) {
+        set_error("workspace is NULL or smaller than its control block");
+        return TS_ERR_WORKSPACE;
+    }
+    // The control block is a prefix of every layout; zero at most 1 MiB of it
+    // (it holds the status word and per-sequence / per-head counters).
+    size_t n = ws_bytes < (size_t(1) << 20) ? ws_bytes : (size_t(1) << 20);
+    cudaError_t e = cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_workspace_init");
+}
+
+ts_status_t ts_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int32_t first_step,
+                        int32_t batch, int32_t h_q, int32_t head_dim, double threshold, void *stream)
+{
+    if (q == nullptr || q_prev == nullptr || reuse == nullptr) {
+        set_error("q, q_prev and reuse are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (batch < 1 || h_q < 1 || (head_dim != 64 && head_dim != 128)) {
+        set_error("bad shape (batch %d, h_q %d, head_dim %d)", batch, h_q, head_dim);
+        return TS_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(q_prev)) & 3u) {
+        set_error("q and q_prev must be 4-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (isnan(threshold)) {
+        set_error("threshold is NaN");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_selcache(q, q_prev, reuse, cos_out, first_step != 0, batch, h_q * head_dim, threshold,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_selcache launch");
+}
+
+static ts_status_t score_prologue(const ts_kv_t *kv, void *ws, size_t ws_bytes, Plan *p)
+{
+    ts_status_t s = make_plan(kv, -1, p);
+    if (s != TS_OK)
+        return s;
+    // the score phases need everything up to the attention partials
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < p->off_attn_part) {
+        set_error("workspace missing, misaligned or too small (%zu < %zu)", ws_bytes, p->off_attn_part);
+        return TS_ERR_WORKSPACE;
+    }
+    return TS_OK;
+}
+
+ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reuse, void *ws, size_t ws_bytes,
+                            void *stream)
+{
+    Plan p;
+    ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || (reinterpret_cast<uintptr_t>(q) & 3u)) {
+        set_error("q is required and must be 4-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (p.n_total == 0)
+        return TS_OK;
+    CUtensorMap kmap;
+    s = encode_kmap(p, kv, &kmap);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_score(p, kmap, q, kv->seq_offsets_dev, reuse, static_cast<uint8_t *>(ws),
+                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass A launch");
+}
+
+ts_status_t ts_score_vote(const ts_kv_t *kv, const int32_t *reuse, float *votes, void *ws, size_t ws_bytes,
+                          void *stream)
+{
+    Plan p;
+    ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
+    if (s != TS_OK)
+        return s;
+    if (votes == nullptr) {
+        set_error("votes is required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (p.n_total == 0)
+        return TS_OK;
+    cudaError_t e = launch_vote(p, kv->seq_offsets_dev, reuse, votes, static_cast<uint8_t *>(ws),
+                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass B launch");
+}
+
+ts_status_t ts_score(const ts_kv_t *kv, const void *q, const int32_t *reuse, float *votes, void *ws,
+                     size_t ws_bytes, void *stream)
+{
+    if (votes == nullptr) {
+        set_error("votes is required");
+        return TS_ERR_INVALID_ARG;
+    }
+    ts_status_t s = ts_score_logits(kv, q, reuse, ws, ws_bytes, stream);
+    if (s != TS_OK)
+        return s;
+    return ts_score_vote(kv, reuse, votes, ws, ws_bytes, stream);
+}
+
+ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink, int32_t n_local,
+                      const int32_t *reuse, int32_t *ids, int32_t *count, void *ws, size_t ws_bytes, void *stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    if (k < 0 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > (int64_t(1) << 30)) {
+        set_error("k, n_sink, n_local must be non-negative with a sum below 2^30");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = make_plan(kv, k + n_sink + n_local, &p);
+    if (s != TS_OK)
+        return s;
+    if (votes == nullptr || ids == nullptr || count == nullptr) {
+        set_error("votes, ids and count are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_select(p, kv->seq_offsets_dev, votes, k, n_sink, n_local, reuse, ids, count,
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "select launch");
+}
+
+ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
+                           int32_t ids_capacity, float *out, void *ws, size_t ws_bytes, void *stream)
+{
+    if (ids_capacity < 1) {
+        set_error("ids_capacity must be >= 1");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = make_plan(kv, ids_capacity, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || ids == nullptr || count == nullptr || out == nullptr) {
+        set_error("q, ids, count and out are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(q) & 15u) {
+        set_error("q must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    s = check_ws(p, ws, ws_bytes);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_attn(p, kv, q, ids, count, out, static_cast<uint8_t *>(ws),
+                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "sparse attention launch");
+}
+
+ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream)
+{
+    if (ws == nullptr || ws_bytes < 256) {
+        set_error("workspace is NULL or too small");
+        return TS_ERR_WORKSPACE;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t h[2] = {0u, 0u};
+    cudaError_t e = cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ws, 0, sizeof h, st);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_get_device_status");
+    if (site_out)
+        *site_out = h[1];
+    if (h[0] != 0u) {
+        set_error("a device-side wait gave up (site %u)", h[1]);
+        return TS_ERR_DEVICE_TIMEOUT;
+    }
+    return TS_OK;
+}
+
+ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_limit, void *stream)
+{
+    if (ws == nullptr || ws_bytes < 256) {
+        set_error("workspace is NULL or too small");
+        return TS_ERR_WORKSPACE;
+    }
+    if (spin_limit == 0 || spin_limit > (1u << 20)) {
+        set_error("spin_limit must be in [1, 2^20]");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_selftest_wait(static_cast<uint32_t *>(ws), spin_limit, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "selftest launch");
+}
+
+const char *ts_status_string(ts_status_t status)
+{
+    switch (status) {
+    case TS_OK: return "TS_OK";
+    case TS_ERR_INVALID_ARG: return "TS_ERR_INVALID_ARG";
+    case TS_ERR_UNSUPPORTED: return "TS_ERR_UNSUPPORTED";
+    case TS_ERR_WORKSPACE: return "TS_ERR_WORKSPACE";
+    case TS_ERR_CUDA: return "TS_ERR_CUDA";
+    case TS_ERR_DEVICE_TIMEOUT: return "TS_ERR_DEVICE_TIMEOUT";
+    }
+    return "TS_ERR_UNKNOWN";
+}
+
+const char *ts_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+// Device-side building blocks for the sm_100a kernels of libts: shared-memory
+// barriers with bounded waits, TMA tile loads, ldmatrix / mma.sync wrappers,
+// and the workspace status word.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ts {
+
+// ---------------------------------------------------------------------------
+// Status word (first 256 bytes of every workspace)
+// ---------------------------------------------------------------------------
+// ctrl[0] : 0 = ok, 1 = a bounded wait gave up
+// ctrl[1] : site code of the first wait that gave up
+enum : uint32_t {
+    kSiteScoreFull = 1,       // score consumer waiting for a K tile
+    kSiteScoreEmpty = 2,      // score producer waiting for a free stage
+    kSiteSelftest = 99,
+};
+
+// Polls of a shared-memory barrier before a wait gives up.  With the back-off
+// below this is well over a second of wall time, orders of magnitude above
+// any legitimate wait (a TMA tile lands in microseconds).
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ void report_timeout(uint32_t *ctrl, uint32_t site)
+{
+    if (atomicCAS(&ctrl[0], 0u, 1u) == 0u)
+        atomicExch(&ctrl[1], site);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the other threads and the async proxy.
+__device__ __forceinline__ void mbar_fence_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete, polling at most
+// `limit` times.  Returns false when the wait gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit)
+{
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (i >= 64)
+            __nanosleep(128);
+    }
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), no multicast
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 3-D tile load into this CTA's shared memory; completion is signalled on
+// `bar` as transaction bytes.  x (innermost) must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
+                                            int32_t y, int32_t z, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level tensor-core tiles (bf16 x bf16 -> fp32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                            uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A * B + D for one m16n8k16 tile; A row-major (16 x 16), B column-major (16 x 8).
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Named barrier over a subset of the block's warps.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Small numeric helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Merge two (max, sum of exp(x - max)) pairs in fp32.  -inf max = empty.
+__device__ __forceinline__ void lse_merge(float &m, float &z, float m2, float z2)
+{
+    float mn = fmaxf(m, m2);
+    if (mn == -INFINITY)
+        return;
+    z = z * exp2f((m - mn) * 1.4426950408889634f) + z2 * exp2f((m2 - mn) * 1.4426950408889634f);
+    m = mn;
+}
+
+// Sequence lookup: largest b with start[b] <= v, over start[0..nb] ascending.
+__device__ __forceinline__ int upper_seq(const int32_t *start, int nb, int32_t v)
+{
+    int lo = 0, hi = nb;   // invariant: start[lo] <= v < start[hi]
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (start[mid] <= v)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+}  // namespace ts

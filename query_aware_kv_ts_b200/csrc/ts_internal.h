@@ -1,0 +1,75 @@
+// Host-side internals of libts: workspace layout, per-launch plans and the
+// launchers each kernel file provides to api.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/ts.h"
+
+namespace ts {
+
+constexpr int kMaxBatch = 1024;        // sequences per call (shared-memory tables)
+constexpr int kScoreConsumerWarps = 8;
+constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
+constexpr int kScoreStages = 6;
+constexpr int kStageBytesTarget = 32768;
+constexpr int kVoteThreads = 256;
+constexpr int kVoteTokensPerBlock = 1024;
+constexpr int kSelectClusterSize = 8;
+constexpr int kSelectThreads = 1024;
+constexpr int kAttnThreads = 128;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Everything derived from the cache shape that the kernels and the workspace
+// layout need.  Built identically by every entry point.
+struct Plan {
+    int B, Hq, Hkv, G, D;
+    int64_t n_total;         // seq_offsets[B]
+    int64_t n_max;           // longest sequence
+    float scale;
+    int sms;
+    // score pass A
+    int tile_tokens;         // T: tokens per pipeline stage
+    int stage_bytes;
+    int64_t chunk_tokens;    // tokens per work chunk (multiple of T)
+    int64_t max_chunks;      // sum_b ceil(n_b / chunk_tokens)
+    int score_grid;
+    // vote pass B
+    int64_t max_vote_blocks; // sum_b ceil(n_b / kVoteTokensPerBlock)
+    // attention
+    int capacity;            // ids row length (k + sink + local)
+    int attn_splits;
+    // workspace layout (byte offsets)
+    size_t off_ctrl, off_score_tickets, off_attn_tickets, off_L, off_partials, off_logits,
+        off_attn_part, total_bytes;
+};
+
+// Fill `p` from the cache description (capacity < 0: attention part not
+// needed).  Returns TS_OK or an error with ts_last_error set.
+ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p);
+
+void set_error(const char *fmt, ...);
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step,
+                            int B, int len, double theta, cudaStream_t st);
+
+cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
+                         const int32_t *reuse, uint8_t *ws, cudaStream_t st);
+
+cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
+                        cudaStream_t st);
+
+cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,
+                          int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, cudaStream_t st);
+
+cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
+                        const int32_t *count, float *out, uint8_t *ws, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(uint32_t *ctrl, uint32_t spin_limit, cudaStream_t st);
+
+}  // namespace ts

@@ -1,0 +1,74 @@
+"""The C-ABI library loads and exports every function include/ts.h declares.
+
+Runs without a GPU: only symbol lookup and argument checks that fail on the
+host before any CUDA call are exercised here (no compute)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ts.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"TS_API\s+[\w\s\*]+?\b(ts_\w+)\s*\(", src)))
+
+
+def load_build_module():
+    import importlib.util
+    path = os.path.join(ROOT, "query_aware_kv_ts_b200", "csrc", "build.py")
+    spec = importlib.util.spec_from_file_location("ts_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(load_build_module().build())
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("ts_selcache", "ts_score", "ts_select", "ts_sparse_attn", "ts_workspace_bytes",
+                 "ts_get_device_status", "ts_status_string"):
+        assert want in names, names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_only_declared_symbols_are_exported(lib):
+    out = os.popen("nm -D --defined-only %s" % lib._name).read()
+    exported = sorted(set(re.findall(r"\b[TW] (ts_\w+)", out)))
+    assert exported == _declared(), (exported, _declared())
+
+
+def test_status_strings(lib):
+    lib.ts_status_string.restype = ctypes.c_char_p
+    for code, name in enumerate(["TS_OK", "TS_ERR_INVALID_ARG", "TS_ERR_UNSUPPORTED", "TS_ERR_WORKSPACE",
+                                 "TS_ERR_CUDA", "TS_ERR_DEVICE_TIMEOUT"]):
+        assert lib.ts_status_string(code).decode() == name
+
+
+def test_host_side_argument_errors(lib):
+    """Invalid arguments are rejected on the host before anything is launched."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    lib.ts_score.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_size_t, ctypes.c_void_p]
+    assert lib.ts_score(None, None, None, None, None, 0, None) == 1          # votes NULL
+    assert lib.ts_last_error() != b""
+    lib.ts_score_logits.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_size_t, ctypes.c_void_p]
+    assert lib.ts_score_logits(None, None, None, None, 0, None) == 1       # kv NULL
+    assert b"kv" in lib.ts_last_error()
+    lib.ts_selcache.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int32] * 4 + [ctypes.c_double, ctypes.c_void_p]
+    assert lib.ts_selcache(None, None, None, None, 0, 1, 4, 64, 0.9, None) == 1
+    lib.ts_workspace_init.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert lib.ts_workspace_init(None, 0, None) == 3
+    lib.ts_selftest_expire_wait.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]
+    assert lib.ts_selftest_expire_wait(None, 0, 10, None) == 3

@@ -1,0 +1,94 @@
+"""GPU parity: the C-ABI decode step against the float64 oracle.
+
+Small synthetic cases cover every kernel specialisation (head_dim 64/128,
+group sizes 1..16, h_kv 1..8), ragged batches with empty and one-token
+sequences, tails that are not a multiple of the tile, windows larger than the
+sequence, k = 0 and k >= candidates, tied votes, padded strides and very peaked
+scores.  Each case spans several 16-token tiles and a ragged tail."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_helpers as H
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(lengths, h_q, h_kv, d, seed, dist="normal", strides=None, scale=0.0, planted=0):
+    off = W.seq_offsets(lengths)
+    n = int(off[-1])
+    st, sh = strides if strides else (None, None)
+    k, v = W.random_kv(n, h_kv, d, seed, device="cuda", dist=dist, stride_tok=st, stride_head=sh)
+    g = torch.Generator().manual_seed(seed + 1)
+    q = torch.randn((len(lengths), h_q, d), generator=g).to(torch.bfloat16)
+    if planted:
+        G = h_q // h_kv
+        for b in range(len(lengths)):
+            nb = int(lengths[b])
+            if nb == 0:
+                continue
+            pos = np.random.default_rng(seed + b).choice(nb, size=min(planted, nb), replace=False)
+            qm = q[b].double().reshape(h_kv, G, d).mean(1)
+            key = (3 * d ** 0.5 * qm / qm.norm(dim=1, keepdim=True)).to(torch.bfloat16).cuda()
+            for p_ in pos:
+                k[int(off[b]) + int(p_)] = key
+    return H.Case(k, v, off, q.cuda(), scale=scale)
+
+
+CASES = {
+    # name: (lengths, h_q, h_kv, d, k, sink, local, extra)
+    "d64_g2": ([4096], 4, 2, 64, 256, 4, 64, {"planted": 16}),
+    "d128_g7_ragged_tail": ([1000, 37, 3333], 28, 4, 128, 100, 4, 50, {"planted": 8}),
+    "g8_hkv8": ([777], 64, 8, 128, 64, 2, 16, {}),
+    "g16_two_ntiles": ([2048, 513], 32, 2, 128, 128, 4, 32, {}),
+    "g16_d64": ([999], 16, 1, 64, 90, 3, 7, {}),
+    "mha_g1": ([500], 4, 4, 64, 50, 1, 10, {}),
+    "hkv1_d128": ([1500], 8, 1, 128, 100, 4, 100, {}),
+    "short_sequences": ([3, 10, 70, 1], 28, 4, 128, 16, 4, 64, {}),
+    "k_above_candidates": ([300], 4, 2, 64, 1000, 4, 64, {}),
+    "k_zero": ([300], 4, 2, 64, 0, 4, 64, {}),
+    "empty_sequences": ([0, 500, 0, 1], 4, 2, 64, 32, 4, 8, {}),
+    "no_windows": ([1234], 8, 2, 128, 77, 0, 0, {}),
+    "constant_keys_all_tied": ([1000], 4, 2, 64, 100, 4, 16, {"dist": "const"}),
+    "integer_keys_many_ties": ([2000], 28, 4, 128, 200, 4, 64, {"dist": "int"}),
+    "padded_strides": ([3000], 28, 4, 128, 256, 4, 64, {"strides": (4 * 128 * 2 + 64, 256)}),
+    "peaked_scores": ([2500], 8, 2, 128, 64, 4, 32, {"scale": 1.0}),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_case(name):
+    lengths, h_q, h_kv, d, k, s, l, extra = CASES[name]
+    case = _case(lengths, h_q, h_kv, d, seed=zlib.crc32(name.encode()) % 10000, **extra)
+    buf = H.run_step(case, k, s, l)
+    H.check_step(case, buf, k, s, l)
+
+
+def test_all_tied_picks_lowest_ids():
+    case = _case([1000], 4, 2, 64, 3, dist="const")
+    buf = H.run_step(case, 100, 4, 16)
+    ids = buf.ids.cpu().numpy()[0]
+    want = list(range(0, 4)) + list(range(4, 104)) + list(range(984, 1000))
+    assert ids[:buf.count.item()].tolist() == want
+
+
+def test_deterministic():
+    case = _case([5000, 777], 28, 4, 128, 11, planted=5)
+    a = H.run_step(case, 300, 4, 64)
+    va, ia, oa = a.votes.clone(), a.ids.clone(), a.out.clone()
+    for _ in range(3):
+        b = H.run_step(case, 300, 4, 64, buf=a)
+        assert torch.equal(va, b.votes) and torch.equal(ia, b.ids) and torch.equal(oa, b.out)
+
+
+def test_planted_keys_selected():
+    case = _case([8192], 28, 4, 128, 5, planted=40)
+    buf = H.run_step(case, 64, 4, 64)
+    ids = set(buf.ids.cpu().numpy()[0].tolist())
+    # the 40 planted keys carry the top votes
+    votes = buf.votes.cpu().numpy()
+    top = np.argsort(-votes)[:40]
+    assert set(top.tolist()) <= ids
