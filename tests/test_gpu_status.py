@@ -47,5 +47,9 @@ def test_host_errors():
     k3, v3 = W.random_kv(100, 3, 64, 2, device="cuda")      # h_kv = 3 unsupported
     kv3 = m.KVCache(k3, v3, [0, 100], 6)
     with pytest.raises(m.TsError) as e:
-        m.ts_workspace_bytes(kv3, 8, 1, 1)
+        m.ts_workspace_bytes(kv3, 8, 1, 1)                   # sizing reports failure as 0 bytes
+    big = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    q6 = torch.randn((1, 6, 64)).to(torch.bfloat16).cuda()
+    with pytest.raises(m.TsError) as e:
+        m.ts_score_logits(kv3, q6, None, big)
     assert e.value.status == m.TS_ERR_UNSUPPORTED
