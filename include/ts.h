@@ -179,6 +179,30 @@ TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_
                            void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * ts_sparse_attn for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a deployment variant of the same attention.
+ * Some hosts own every byte of device memory through their own pool and let
+ * no library call cudaMalloc or take a workspace after start-up, or run under
+ * a memory budget fixed when the process initialises.  This call therefore
+ * takes no workspace and allocates nothing: its scratch (split-K partials and
+ * counters) is a 4 MiB array built into the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   - Arguments, results and errors as for ts_sparse_attn.  Shapes whose
+ *     scratch would exceed 4 MiB (B * h_kv * splits * (h_q/h_kv) * (d+2) * 4
+ *     bytes plus the counters) are rejected with TS_ERR_UNSUPPORTED before
+ *     anything is launched.
+ *   - The first call on each device looks the array up (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array: calls that can overlap on the GPU (on
+ *     different streams, or from different threads) race with each other.
+ *     Each call clears the counters it needs on its stream before launching.
+ */
+TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32_t *ids,
+                                          const int32_t *count, int32_t ids_capacity, float *out,
+                                          void *stream);
+
+/*
  * Read and clear the device status word of a workspace (synchronises the
  * stream).  Returns TS_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave
  * up since the last read, TS_OK otherwise.  *site_out (may be NULL) receives

@@ -64,6 +64,7 @@ _SIGS = {
     "ts_score_vote": (ctypes.c_int, [_KV, _P, _P, _P, _SZ, _P]),
     "ts_select": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "ts_sparse_attn": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
+    "ts_sparse_attn_noalloc": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -177,6 +178,13 @@ def ts_select(kv: KVCache, votes, k: int, n_sink: int, n_local: int, reuse, ids,
 def ts_sparse_attn(kv: KVCache, q, ids, count, out, ws, stream=None):
     _check(_lib.ts_sparse_attn(kv.ref(), _ptr(q), _ptr(ids), _ptr(count), ids.shape[-1], _ptr(out),
                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ts_sparse_attn_noalloc(kv: KVCache, q, ids, count, out, stream=None):
+    """ts_sparse_attn without a workspace: for hosts that own all device memory
+    and let no library allocate; the scratch is a fixed array inside libts."""
+    _check(_lib.ts_sparse_attn_noalloc(kv.ref(), _ptr(q), _ptr(ids), _ptr(count), ids.shape[-1], _ptr(out),
+                                       _stream(stream)))
 
 
 def ts_get_device_status(ws, stream=None):

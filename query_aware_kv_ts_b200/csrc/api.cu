@@ -402,6 +402,28 @@ ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_t *ids,
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "sparse attention launch");
 }
 
+ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
+                                   int32_t ids_capacity, float *out, void *stream)
+{
+    if (ids_capacity < 1) {
+        set_error("ids_capacity must be >= 1");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = make_plan(kv, ids_capacity, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || ids == nullptr || count == nullptr || out == nullptr) {
+        set_error("q, ids, count and out are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(q) & 15u) {
+        set_error("q must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    return launch_attn_noalloc(p, kv, q, ids, count, out, static_cast<cudaStream_t>(stream));
+}
+
 ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream)
 {
     if (ws == nullptr || ws_bytes < 256) {

@@ -10,6 +10,8 @@
 // an online softmax (max, sum, weighted V) per head.  The CTA merges its warps
 // and writes one partial per (split, head); the CTA that completes the last
 // split of (b, g) (atomic ticket, no waiting) merges the splits into out.
+#include <mutex>
+
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -218,7 +220,100 @@ cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant (ts_sparse_attn_noalloc)
+// ---------------------------------------------------------------------------
+// Some callers cannot hand this library any device memory: runtimes that own
+// every byte of device memory through their own pool and let no library call
+// cudaMalloc or take a workspace after start-up, and deployments whose memory
+// budget is fixed when the process initialises.  For them the split-K
+// partials and the per-(sequence, kv head) tickets live in this file-scope
+// array instead of a caller workspace.  Every GPU that loads the library holds
+// it until the process exits; all calls share it (and it keeps the last call's
+// contents), so calls that can overlap on the GPU race with each other.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) uint8_t g_attn_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array for the current device, looked up once per
+// device (with that device current) and cached.
+static uint8_t *noalloc_scratch_ptr(ts_status_t *status)
+{
+    static std::mutex mu;
+    static uint8_t *ptrs[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        set_error("ts_sparse_attn_noalloc: no usable current device");
+        *status = TS_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_attn_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) {
+            set_error("ts_sparse_attn_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+            *status = TS_ERR_CUDA;
+            return nullptr;
+        }
+        ptrs[dev] = static_cast<uint8_t *>(ptr);
+    }
+    *status = TS_OK;
+    return ptrs[dev];
+}
+
 }  // namespace
+
+ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
+                                const int32_t *count, float *out, cudaStream_t st)
+{
+    const size_t ticket_bytes = align_up(sizeof(uint32_t) * (size_t)p.B * p.Hkv, 256);
+    const size_t part_bytes = sizeof(float) * (size_t)p.B * p.Hkv * p.attn_splits * p.G * (p.D + 2);
+    if (ticket_bytes + part_bytes > kNoAllocScratchBytes) {
+        set_error("ts_sparse_attn_noalloc: this shape needs %zu bytes of scratch, more than the fixed %zu; "
+                  "use ts_sparse_attn with a workspace",
+                  ticket_bytes + part_bytes, kNoAllocScratchBytes);
+        return TS_ERR_UNSUPPORTED;
+    }
+    ts_status_t status;
+    uint8_t *scratch = noalloc_scratch_ptr(&status);
+    if (scratch == nullptr)
+        return status;
+    // the tickets must start at zero whatever an earlier call left behind
+    cudaError_t e = cudaMemsetAsync(scratch, 0, ticket_bytes, st);
+    if (e != cudaSuccess) {
+        set_error("ts_sparse_attn_noalloc: clearing the tickets failed: %s", cudaGetErrorString(e));
+        return TS_ERR_CUDA;
+    }
+    AttnArgs a;
+    a.k = static_cast<const __nv_bfloat16 *>(kv->k);
+    a.v = static_cast<const __nv_bfloat16 *>(kv->v);
+    a.st = kv->stride_tok;
+    a.sh = kv->stride_head;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.seq_off = kv->seq_offsets_dev;
+    a.ids = ids;
+    a.count = count;
+    a.cap = p.capacity;
+    a.out = out;
+    a.tickets = reinterpret_cast<uint32_t *>(scratch);
+    a.part = reinterpret_cast<float *>(scratch + ticket_bytes);
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.splits = p.attn_splits;
+    a.scale_log2 = p.scale * kLog2e;
+    if (p.D == 128)
+        e = p.G <= 8 ? launch_attn_t<128, 8>(p, a, st) : launch_attn_t<128, 16>(p, a, st);
+    else
+        e = p.G <= 8 ? launch_attn_t<64, 8>(p, a, st) : launch_attn_t<64, 16>(p, a, st);
+    if (e != cudaSuccess) {
+        set_error("ts_sparse_attn_noalloc launch: %s", cudaGetErrorString(e));
+        return TS_ERR_CUDA;
+    }
+    return TS_OK;
+}
 
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
                         float *out, uint8_t *ws, cudaStream_t st)

@@ -70,6 +70,11 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
                         const int32_t *count, float *out, uint8_t *ws, cudaStream_t st);
 
+// Attention with its scratch in a fixed device array instead of a workspace
+// (sets the error message itself).
+ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
+                                const int32_t *count, float *out, cudaStream_t st);
+
 cudaError_t launch_selftest_wait(uint32_t *ctrl, uint32_t spin_limit, cudaStream_t st);
 
 }  // namespace ts
