@@ -94,10 +94,11 @@ typedef struct ts_kv {
 TS_API size_t ts_workspace_bytes(const ts_kv_t *kv, int32_t k, int32_t n_sink, int32_t n_local);
 
 /*
- * Zero the workspace's control block (device counters and the status word).
- * Call once after allocating a workspace, before its first use, on the stream
- * that will use it.  The library returns every counter to zero itself, so a
- * workspace needs no re-initialisation between calls.
+ * Zero a workspace (the status word and the selection counters and
+ * histogram).  Call once after allocating a workspace, before its first use,
+ * on the stream that will use it.  The library returns every counter to zero
+ * itself at the end of each call, so a workspace needs no re-initialisation
+ * between calls (only after a call that reported an error).
  */
 TS_API ts_status_t ts_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
@@ -161,6 +162,8 @@ TS_API ts_status_t ts_score_vote(const ts_kv_t *kv, const int32_t *reuse, float 
  *   votes      device float32 [seq_offsets[batch]] (non-negative, finite)
  *   ids        device int32 [batch, k + n_sink + n_local]
  *   count      device int32 [batch]
+ *   ws         workspace (ts_workspace_bytes), shared with ts_score
+ * Sequences may hold at most 4194304 tokens.
  */
 TS_API ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink,
                       int32_t n_local, const int32_t *reuse, int32_t *ids, int32_t *count,
@@ -172,7 +175,9 @@ TS_API ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, i
  * over j < count[b] (count[b] == 0 gives zeros).
  *   ids        device int32 [batch, ids_capacity], ids in [0, n_b)
  *   count      device int32 [batch], 0 <= count[b] <= ids_capacity
- *   out        device float32 [batch, h_q, head_dim], written
+ *   out        device float32 [batch, h_q, head_dim], 16-byte aligned, written
+ * ids_capacity (= k + n_sink + n_local) is at most 16384.  Ids outside
+ * [0, n_b) are skipped.
  */
 TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_t *ids,
                            const int32_t *count, int32_t ids_capacity, float *out,
@@ -184,19 +189,20 @@ TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_
  * Some hosts own every byte of device memory through their own pool and let
  * no library call cudaMalloc or take a workspace after start-up, or run under
  * a memory budget fixed when the process initialises.  This call therefore
- * takes no workspace and allocates nothing: its scratch (split-K partials and
- * counters) is a 4 MiB array built into the library, which every GPU that
+ * takes no workspace and allocates nothing: its scratch (the split-K
+ * partials) is a 4 MiB array built into the library, which every GPU that
  * loads the library holds until the process exits.
  *   - Arguments, results and errors as for ts_sparse_attn.  Shapes whose
- *     scratch would exceed 4 MiB (B * h_kv * splits * (h_q/h_kv) * (d+2) * 4
- *     bytes plus the counters) are rejected with TS_ERR_UNSUPPORTED before
- *     anything is launched.
+ *     scratch would exceed 4 MiB (B * h_kv * splits * (h_q/h_kv) * (d+4) * 4
+ *     bytes, splits = ceil(ids_capacity / 128)) are rejected with
+ *     TS_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on each device looks the array up (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream
  *     capture.
- *   - Every call shares the one array: calls that can overlap on the GPU (on
- *     different streams, or from different threads) race with each other.
- *     Each call clears the counters it needs on its stream before launching.
+ *   - Every call shares the one array, which keeps the last call's
+ *     contents: calls that can overlap on the GPU (on different streams, or
+ *     from different threads) race with each other.  Nothing in it has to
+ *     start at zero: a call writes every partial it reads before reading it.
  */
 TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32_t *ids,
                                           const int32_t *count, int32_t ids_capacity, float *out,

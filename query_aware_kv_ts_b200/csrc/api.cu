@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -55,6 +56,15 @@ ts_status_t cuda_fail(cudaError_t e, const char *what)
     return TS_ERR_CUDA;
 }
 }  // namespace
+
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char *e = getenv("TS_NO_PDL");
+        return !(e != nullptr && e[0] == '1');
+    }();
+    return on;
+}
 
 void set_error(const char *fmt, ...)
 {
@@ -136,6 +146,11 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
         set_error("total tokens %lld must be below 2^31", (long long)n_total);
         return TS_ERR_UNSUPPORTED;
     }
+    if (n_max > (int64_t)kMaxSelectRanges * kSelectTokensPerCta) {
+        set_error("sequence length %lld exceeds the supported maximum %lld", (long long)n_max,
+                  (long long)kMaxSelectRanges * kSelectTokensPerCta);
+        return TS_ERR_UNSUPPORTED;
+    }
     const int sms = device_sms();
     if (sms <= 0) {
         set_error("no CUDA device");
@@ -153,44 +168,54 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->sms = sms;
     p->tile_tokens = (kStageBytesTarget / 2) / (kv->h_kv * D);
     p->stage_bytes = p->tile_tokens * kv->h_kv * D * 2;
-    p->chunk_tokens = p->tile_tokens;
-    int64_t chunks = 0, vblocks = 0;
+    int64_t chunks = 0;
     for (int b = 0; b < kv->batch; ++b) {
         const int64_t n = off[b + 1] - off[b];
-        chunks += (n + p->chunk_tokens - 1) / p->chunk_tokens;
-        vblocks += (n + kVoteTokensPerBlock - 1) / kVoteTokensPerBlock;
+        chunks += (n + p->tile_tokens - 1) / p->tile_tokens;
     }
     p->max_chunks = chunks;
-    p->score_grid = (int)(chunks < sms ? chunks : sms);
-    p->max_vote_blocks = vblocks;
+    const int grid_cap = sms < 256 ? sms : 256;
+    p->score_grid = (int)(chunks < grid_cap ? chunks : grid_cap);
+    p->ld_logits = (n_total + 3) / 4 * 4;
+    p->sel_ranges = (int)((n_max + kSelectTokensPerCta - 1) / kSelectTokensPerCta) + 1;
     p->capacity = capacity;
-    if (capacity > 0) {
-        int64_t want = (2 * (int64_t)sms + (int64_t)p->B * p->Hkv - 1) / ((int64_t)p->B * p->Hkv);
-        int64_t cap_splits = (capacity + 31) / 32;
-        p->attn_splits = (int)(want < 1 ? 1 : (want > cap_splits ? cap_splits : want));
-        if (p->attn_splits < 1)
-            p->attn_splits = 1;
-    } else {
-        p->attn_splits = 0;
+    if (capacity > kMaxCapacity) {
+        set_error("k + n_sink + n_local = %d exceeds the supported maximum %d", capacity, kMaxCapacity);
+        return TS_ERR_UNSUPPORTED;
     }
+    // every attention CTA takes at most kAttnRows selected rows
+    p->attn_splits = capacity > 0 ? (capacity + kAttnRows - 1) / kAttnRows : 0;
 
     size_t o = 0;
     p->off_ctrl = o;
     o += 256;
-    p->off_score_tickets = o;
-    o = align_up(o + sizeof(uint32_t) * p->B, 256);
-    p->off_attn_tickets = o;
-    o = align_up(o + sizeof(uint32_t) * p->B * p->Hkv, 256);
     // everything above is the control block that ts_workspace_init zeroes
+    p->off_chunk_table = o;
+    o = align_up(o + sizeof(int32_t) * (p->B + 1), 256);
     p->off_L = o;
     o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
     p->off_partials = o;
     o = align_up(o + sizeof(float) * 2 * (size_t)(chunks > 0 ? chunks : 1) * p->Hq, 256);
     p->off_logits = o;
-    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(n_total > 0 ? n_total : 1), 256);
+    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(p->ld_logits > 0 ? p->ld_logits : 4), 256);
+    const size_t nt1 = (size_t)(n_total > 0 ? n_total : 1);
+    p->off_sel_hist = o;
+    o = align_up(o + sizeof(uint32_t) * 4096 * (size_t)p->B, 256);
+    p->off_sel_cand = o;
+    o = align_up(o + 8 * nt1, 256);
+    p->off_sel_cand_n = o;
+    o = align_up(o + sizeof(uint32_t) * (size_t)p->B, 256);
+    p->off_sel_above = o;
+    o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
+    p->off_sel_range_off = o;
+    o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
+    p->off_sel_thr = o;
+    o = align_up(o + sizeof(uint64_t) * (size_t)p->B, 256);
+    p->off_sel_mode = o;
+    o = align_up(o + sizeof(int32_t) * (size_t)p->B, 256);
     p->off_attn_part = o;
     if (capacity > 0)
-        o = align_up(o + sizeof(float) * (size_t)p->B * p->Hkv * p->attn_splits * p->G * (D + 2), 256);
+        o = align_up(o + sizeof(float) * (size_t)p->B * p->Hkv * p->attn_splits * p->G * (D + 4), 256);
     p->total_bytes = o;
     return TS_OK;
 }
@@ -256,10 +281,10 @@ ts_status_t ts_workspace_init(void *ws, size_t ws_bytes, void *stream)
         set_error("workspace is NULL or smaller than its control block");
         return TS_ERR_WORKSPACE;
     }
-    // The control block is a prefix of every layout; zero at most 1 MiB of it
-    // (it holds the status word and per-sequence / per-head counters).
-    size_t n = ws_bytes < (size_t(1) << 20) ? ws_bytes : (size_t(1) << 20);
-    cudaError_t e = cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream));
+    // The whole workspace starts at zero: the status word, and the selection
+    // histogram and list counters, which the library returns to zero itself
+    // after every use.
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_workspace_init");
 }
 
@@ -356,8 +381,6 @@ ts_status_t ts_score(const ts_kv_t *kv, const void *q, const int32_t *reuse, flo
 ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink, int32_t n_local,
                       const int32_t *reuse, int32_t *ids, int32_t *count, void *ws, size_t ws_bytes, void *stream)
 {
-    (void)ws;
-    (void)ws_bytes;
     if (k < 0 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > (int64_t(1) << 30)) {
         set_error("k, n_sink, n_local must be non-negative with a sum below 2^30");
         return TS_ERR_INVALID_ARG;
@@ -370,8 +393,12 @@ ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t 
         set_error("votes, ids and count are required");
         return TS_ERR_INVALID_ARG;
     }
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < p.off_attn_part) {
+        set_error("workspace missing, misaligned or too small (%zu < %zu)", ws_bytes, p.off_attn_part);
+        return TS_ERR_WORKSPACE;
+    }
     cudaError_t e = launch_select(p, kv->seq_offsets_dev, votes, k, n_sink, n_local, reuse, ids, count,
-                                  static_cast<cudaStream_t>(stream));
+                                  static_cast<uint8_t *>(ws), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "select launch");
 }
 
@@ -390,8 +417,8 @@ ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_t *ids,
         set_error("q, ids, count and out are required");
         return TS_ERR_INVALID_ARG;
     }
-    if (reinterpret_cast<uintptr_t>(q) & 15u) {
-        set_error("q must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u) {
+        set_error("q and out must be 16-byte aligned");
         return TS_ERR_INVALID_ARG;
     }
     s = check_ws(p, ws, ws_bytes);
@@ -417,8 +444,8 @@ ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32
         set_error("q, ids, count and out are required");
         return TS_ERR_INVALID_ARG;
     }
-    if (reinterpret_cast<uintptr_t>(q) & 15u) {
-        set_error("q must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u) {
+        set_error("q and out must be 16-byte aligned");
         return TS_ERR_INVALID_ARG;
     }
     return launch_attn_noalloc(p, kv, q, ids, count, out, static_cast<cudaStream_t>(stream));

@@ -2,14 +2,23 @@
 // number of critical KV cache tokens take part in the attention calculation).
 //   out[b, h, :] = sum_j softmax_j(scale * q_h . K[ids_j, g]) * V[ids_j, g]
 //
-// Split-K decode attention: grid (splits, h_kv, B).  Each CTA takes a slice of
-// one sequence's selected ids for one KV head g and serves all G query heads
-// of g from the same gathered K/V rows, so each selected row is read from HBM
-// once.  Warps take rows round-robin; a lane holds d/32 channels of the row,
-// the G dot products are finished with warp butterflies, and every warp keeps
-// an online softmax (max, sum, weighted V) per head.  The CTA merges its warps
-// and writes one partial per (split, head); the CTA that completes the last
-// split of (b, g) (atomic ticket, no waiting) merges the splits into out.
+// Split-K decode attention: grid (splits, h_kv, B), 256 threads, at most 128
+// selected rows per CTA.  Each CTA:
+//  1. gathers its K and V rows into shared memory with coalesced 16-byte
+//     asynchronous copies (every row of the CTA in flight at once);
+//  2. computes the logits of the G query heads of kv head g on tensor cores
+//     (m16n8k16 bf16 -> fp32: rows as M, heads as N, channels as K; the Q
+//     fragments stay in registers);
+//  3. takes the softmax of each head over its rows (warp reductions);
+//  4. computes O^T = V^T P^T on tensor cores: V^T fragments come from the
+//     row-major V tile with transposed ldmatrix, and P is split into a bf16
+//     high part and a bf16 remainder (two products) so that the weights keep
+//     ~16 significant bits instead of bf16's 8;
+//  5. writes (max, sum, weighted V) per head as its partial.
+// attn_merge (one block per (b, g), launched right after) folds the splits:
+// a thread owns 4 output channels of one head and reads those channels and
+// the (max, sum) of every split, 16 splits at a time, with an online rescale.
+// Each selected K/V row is read from HBM once for all G heads of its group.
 #include <mutex>
 
 #include "ts_device.cuh"
@@ -20,6 +29,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAttnWarps = kAttnThreads / 32;
+constexpr int R = kAttnRows;
 
 struct AttnArgs {
     const __nv_bfloat16 *k, *v;
@@ -30,194 +40,336 @@ struct AttnArgs {
     const int32_t *count;
     int cap;
     float *out;
-    float *part;        // [B][Hkv][splits][G][D + 2]
-    uint32_t *tickets;  // [B][Hkv]
+    float *part;        // [B][Hkv][splits][G][D + 4]: D weighted-V sums, then (max, sum)
     int B, Hq, Hkv, G, splits;
     float scale_log2;   // scale * log2(e): logits in base-2 units
 };
 
-template <int CPL>
-struct RowLoad;
-template <>
-struct RowLoad<4> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&f)[4])
-    {
-        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
-        f[0] = bf16_lo(w.x);
-        f[1] = bf16_hi(w.x);
-        f[2] = bf16_lo(w.y);
-        f[3] = bf16_hi(w.y);
-    }
-};
-template <>
-struct RowLoad<2> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&f)[2])
-    {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(p));
-        f[0] = bf16_lo(w);
-        f[1] = bf16_hi(w);
-    }
-};
+template <int D, int NB>
+constexpr size_t attn_smem_bytes()
+{
+    return (size_t)2 * R * (D * 2 + 16) + (size_t)R * NB * 8 * 4 + (size_t)2 * NB * 8 * R * 2;
+}
 
-template <int D, int GM>
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x)
+{
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <int D, int NB>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_split(const AttnArgs a)
 {
-    constexpr int CPL = D / 32;
-    __shared__ float s_m[kAttnWarps][GM], s_l[kAttnWarps][GM];
-    __shared__ float s_acc[kAttnWarps][GM][D];
+    constexpr int GM = NB * 8;
+    constexpr int RS = D * 2 + 16;          // shared-memory row stride: conflict-free ldmatrix
+    constexpr int PS = D + 4;               // partial row: D sums, max, sum, 2 pad (16-byte rows)
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *sK = smem;
+    uint8_t *sV = sK + R * RS;
+    float *sS = reinterpret_cast<float *>(sV + R * RS);          // [R][GM] logits (base 2)
+    uint16_t *sPh = reinterpret_cast<uint16_t *>(sS + R * GM);   // [GM][R] weights, bf16 high part
+    uint16_t *sPl = sPh + GM * R;                                 // [GM][R] bf16 remainder
+    __shared__ float s_m[GM], s_l[GM], s_M[GM], s_Linv[GM];
+    __shared__ int32_t s_id[R];
+    __shared__ uint8_t s_valid[R];
     __shared__ int s_last;
 
+    pdl_wait();                 // ids and count come from the selection kernel
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.G;
+    // splits cut the id row's capacity, not its count, so the ids can be
+    // fetched in the same round trip as the count
+    const int lo = (int)((int64_t)a.cap * sp / a.splits);
+    const int hi_cap = (int)((int64_t)a.cap * (sp + 1) / a.splits);
+    const int32_t id_pref = (threadIdx.x < (unsigned)(hi_cap - lo))
+                                ? __ldg(a.ids + (int64_t)b * a.cap + lo + threadIdx.x) : -1;
     int m_b = a.count[b];
     m_b = max(0, min(m_b, a.cap));
-    const int lo = (int)((int64_t)m_b * sp / a.splits);
-    const int hi = (int)((int64_t)m_b * (sp + 1) / a.splits);
+    const int nrows = max(0, min(min(hi_cap, m_b) - lo, R));
     const int64_t off = a.seq_off[b];
     const int64_t n_b = a.seq_off[b + 1] - off;
+    const int r0 = lane >> 2, c0 = (lane & 3) * 2;
 
-    float qf[GM][CPL];
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-            float t[CPL];
-            RowLoad<CPL>::load(a.q + ((int64_t)b * a.Hq + g * G + h) * D + lane * CPL, t);
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                qf[h][c] = t[c];
-        } else {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                qf[h][c] = 0.0f;
+    // ---- 1. gather: ids to shared memory, then every K and V row of the split
+    //         with coalesced 16-byte async copies (CPR consecutive threads per row)
+    if (tid < R) {
+        int32_t id = -1;
+        if (tid < nrows) {
+            id = id_pref;
+            if (id < 0 || (int64_t)id >= n_b)
+                id = -1;                            // ids outside the sequence are ignored
         }
-    }
-    float mr[GM], lr[GM], acc[GM][CPL];
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-        mr[h] = -INFINITY;
-        lr[h] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c)
-            acc[h][c] = 0.0f;
-    }
-
-    const int32_t *idrow = a.ids + (int64_t)b * a.cap;
-    const __nv_bfloat16 *kb = a.k + (int64_t)g * a.sh + lane * CPL;
-    const __nv_bfloat16 *vb = a.v + (int64_t)g * a.sh + lane * CPL;
-    for (int j = lo + warp; j < hi; j += kAttnWarps) {
-        const int32_t id = __ldg(idrow + j);
-        if (id < 0 || (int64_t)id >= n_b)
-            continue;                       // outside the sequence: ignored, never read
-        const int64_t tok = off + id;
-        float kf[CPL], vf[CPL];
-        RowLoad<CPL>::load(kb + tok * a.st, kf);
-        RowLoad<CPL>::load(vb + tok * a.st, vf);
-#pragma unroll
-        for (int h = 0; h < GM; ++h) {
-            if (h < G) {
-                float d = 0.0f;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    d = fmaf(qf[h][c], kf[c], d);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    d += __shfl_xor_sync(0xffffffffu, d, o);
-                const float s = d * a.scale_log2;
-                const float mn = fmaxf(mr[h], s);
-                const float corr = exp2f(mr[h] - mn);
-                const float p = exp2f(s - mn);
-                lr[h] = lr[h] * corr + p;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    acc[h][c] = fmaf(acc[h][c], corr, p * vf[c]);
-                mr[h] = mn;
-            }
-        }
-    }
-
-    // ---- merge the warps of this CTA ---------------------------------------
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-            if (lane == 0) {
-                s_m[warp][h] = mr[h];
-                s_l[warp][h] = lr[h];
-            }
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                s_acc[warp][h][lane * CPL + c] = acc[h][c];
-        }
+        s_id[tid] = id;
+        s_valid[tid] = id >= 0 ? 1 : 0;
     }
     __syncthreads();
-    const int stride = D + 2;
-    float *mypart = a.part + (((int64_t)b * a.Hkv + g) * a.splits + sp) * (int64_t)(G * stride);
-    for (int idx = threadIdx.x; idx < G * D; idx += kAttnThreads) {
-        const int h = idx / D, c = idx - h * D;
-        float M = -INFINITY;
+    {
+        constexpr int CPR = D * 2 / 16;             // 16-byte chunks per row
+        for (int idx = tid; idx < 2 * R * CPR; idx += kAttnThreads) {
+            const int row = idx / CPR, chunk = idx - row * CPR;
+            const bool isV = row >= R;
+            const int r = isV ? row - R : row;
+            uint8_t *dst = (isV ? sV : sK) + r * RS + chunk * 16;
+            const int32_t id = s_id[r];
+            if (id >= 0) {
+                const __nv_bfloat16 *src = (isV ? a.v : a.k) + (off + id) * a.st + (int64_t)g * a.sh;
+                cp_async_16(dst, reinterpret_cast<const uint8_t *>(src) + chunk * 16);
+            } else if (isV) {
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);   // P is 0 there; V must be finite
+            }
+        }
+    }
+
+    uint32_t bq[D / 16][NB][2];
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w)
-            M = fmaxf(M, s_m[w][h]);
-        float A = 0.0f, Lsum = 0.0f;
-        if (M != -INFINITY) {
+    for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) {
-                if (s_m[w][h] != -INFINITY) {
-                    const float e = exp2f(s_m[w][h] - M);
-                    A = fmaf(s_acc[w][h][c], e, A);
-                    Lsum = fmaf(s_l[w][h], e, Lsum);
+        for (int nb = 0; nb < NB; ++nb) {
+            const int j = nb * 8 + r0;
+            if (j < G) {
+                const uint32_t *qp = reinterpret_cast<const uint32_t *>(
+                    a.q + ((int64_t)b * a.Hq + g * G + j) * D + ks * 16 + c0);
+                bq[ks][nb][0] = __ldg(qp);
+                bq[ks][nb][1] = __ldg(qp + 4);
+            } else {
+                bq[ks][nb][0] = 0u;
+                bq[ks][nb][1] = 0u;
+            }
+        }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- 2. logits S = Q K^T (base-2 units) ----------------------------------
+    const int nmb = (nrows + 15) / 16;
+    for (int mb = warp; mb < nmb; mb += kAttnWarps) {
+        float acc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[nb][e] = 0.0f;
+        const int trow = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const uint32_t row_addr = smem_u32(sK + trow * RS) + (uint32_t)((lane >> 4) * 16);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, row_addr + ks * 32);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                mma_16816(acc[nb], a0, a1, a2, a3, bq[ks][nb][0], bq[ks][nb][1]);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int r = mb * 16 + r0 + rr * 8;
+            const bool rv = r < nrows && s_valid[r];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int j = nb * 8 + c0 + cc;
+                    sS[r * GM + j] = (rv && j < G) ? acc[nb][rr * 2 + cc] * a.scale_log2 : -INFINITY;
                 }
-            }
-        }
-        mypart[h * stride + c] = A;
-        if (c == 0) {
-            mypart[h * stride + D] = M;
-            mypart[h * stride + D + 1] = Lsum;
         }
     }
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t t = atomicAdd(&a.tickets[b * a.Hkv + g], 1u);
-        s_last = (t == (uint32_t)a.splits - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!s_last)
-        return;
 
-    // ---- last split of (b, g): merge the splits ---------------------------
-    __threadfence();
-    const float *parts = a.part + ((int64_t)b * a.Hkv + g) * a.splits * (int64_t)(G * stride);
-    for (int idx = threadIdx.x; idx < G * D; idx += kAttnThreads) {
-        const int h = idx / D, c = idx - h * D;
-        float M = -INFINITY;
-        for (int q = 0; q < a.splits; ++q)
-            M = fmaxf(M, __ldcg(parts + (int64_t)q * G * stride + h * stride + D));
-        float A = 0.0f, Lsum = 0.0f;
-        if (M != -INFINITY) {
-            for (int q = 0; q < a.splits; ++q) {
-                const float *pq = parts + (int64_t)q * G * stride + h * stride;
-                const float mq = __ldcg(pq + D);
-                if (mq != -INFINITY) {
-                    const float e = exp2f(mq - M);
-                    A = fmaf(__ldcg(pq + c), e, A);
-                    Lsum = fmaf(__ldcg(pq + D + 1), e, Lsum);
-                }
+    // ---- 3. softmax of each head over this split's rows ---------------------
+    for (int h = warp; h < GM; h += kAttnWarps) {
+        float x[R / 32];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < R / 32; ++i) {
+            const int r = lane + 32 * i;
+            x[i] = (r < nrows && h < G) ? sS[r * GM + h] : -INFINITY;
+            mx = fmaxf(mx, x[i]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.0f;
+#pragma unroll
+        for (int i = 0; i < R / 32; ++i) {
+            const int r = lane + 32 * i;
+            const float p = (mx == -INFINITY) ? 0.0f : exp2f(x[i] - mx);
+            sum += p;
+            const uint16_t hb = bf16_bits_rn(p);
+            sPh[h * R + r] = hb;
+            sPl[h * R + r] = bf16_bits_rn(p - __uint_as_float((uint32_t)hb << 16));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+            s_m[h] = mx;
+            s_l[h] = sum;
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. O^T = V^T P^T: warp w owns channels [16w, 16w + 16) --------------
+    float o[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o[nb][e] = 0.0f;
+    if (warp < D / 16) {
+        const int cw = warp * 16;
+        const int nks = (nrows + 15) / 16;
+        for (int ks = 0; ks < nks; ++ks) {
+            const int rb = ks * 16;
+            const uint32_t addr = smem_u32(sV + (rb + (lane & 7) + ((lane >> 4) & 1) * 8) * RS) +
+                                  (uint32_t)((cw + ((lane >> 3) & 1) * 8) * 2);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(a0, a1, a2, a3, addr);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int h = nb * 8 + r0;
+                const int rr = rb + c0;
+                const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr);
+                const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr + 8);
+                const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr);
+                const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr + 8);
+                mma_16816(o[nb], a0, a1, a2, a3, bh0, bh1);
+                mma_16816(o[nb], a0, a1, a2, a3, bl0, bl1);
             }
         }
-        a.out[((int64_t)b * a.Hq + g * G + h) * D + c] = (Lsum > 0.0f) ? A / Lsum : 0.0f;
     }
-    if (threadIdx.x == 0)
-        a.tickets[b * a.Hkv + g] = 0u;
+
+    // ---- 5. this split's partial ---------------------------------------------
+    const int64_t GS = (int64_t)G * PS;
+    float *mypart = a.part + (((int64_t)b * a.Hkv + g) * a.splits + sp) * GS;
+    if (warp < D / 16) {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int ch = warp * 16 + r0 + (e >= 2 ? 8 : 0);
+                const int h = nb * 8 + c0 + (e & 1);
+                if (h < G)
+                    mypart[h * PS + ch] = o[nb][e];
+            }
+    }
+    if (tid < G) {
+        mypart[tid * PS + D] = s_m[tid];
+        mypart[tid * PS + D + 1] = s_l[tid];
+    }
 }
 
-template <int D, int GM>
+// out[b, g*G + h, :] from the splits of (b, g).  Thread: 4 channels of one head.
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads)
+attn_merge(const AttnArgs a)
+{
+    constexpr int PS = D + 4;
+    constexpr int kBatch = 16;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int G = a.G;
+    const int64_t GS = (int64_t)G * PS;
+    const float *parts = a.part + ((int64_t)b * a.Hkv + g) * a.splits * GS;
+    for (int item = threadIdx.x; item < G * (D / 4); item += kAttnThreads) {
+        const int h = item / (D / 4), c = (item - h * (D / 4)) * 4;
+        float M = -INFINITY, L = 0.0f;
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int q0 = 0; q0 < a.splits; q0 += kBatch) {
+            float4 v4[kBatch];
+            float2 ml[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (q0 + i < a.splits) {
+                    const float *pq = parts + (int64_t)(q0 + i) * GS + h * PS;
+                    v4[i] = __ldcg(reinterpret_cast<const float4 *>(pq + c));
+                    ml[i] = __ldcg(reinterpret_cast<const float2 *>(pq + D));
+                } else {
+                    v4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    ml[i] = make_float2(-INFINITY, 0.0f);
+                }
+            }
+            float Mb = M;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                Mb = fmaxf(Mb, ml[i].x);
+            if (Mb == -INFINITY)
+                continue;
+            const float r = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
+            L *= r;
+            acc.x *= r;
+            acc.y *= r;
+            acc.z *= r;
+            acc.w *= r;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (ml[i].x != -INFINITY) {
+                    const float w = exp2f(ml[i].x - Mb);
+                    L = fmaf(ml[i].y, w, L);
+                    acc.x = fmaf(w, v4[i].x, acc.x);
+                    acc.y = fmaf(w, v4[i].y, acc.y);
+                    acc.z = fmaf(w, v4[i].z, acc.z);
+                    acc.w = fmaf(w, v4[i].w, acc.w);
+                }
+            }
+            M = Mb;
+        }
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        *reinterpret_cast<float4 *>(a.out + ((int64_t)b * a.Hq + g * G + h) * D + c) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+}
+
+template <int D, int NB>
 cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
 {
+    constexpr size_t smem = attn_smem_bytes<D, NB>();
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(attn_split<D, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
     dim3 grid((unsigned)p.attn_splits, (unsigned)p.Hkv, (unsigned)p.B);
-    attn_split<D, GM><<<grid, kAttnThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_ex(attn_split<D, NB>, grid, dim3(kAttnThreads), smem, st, 1, a);
+    if (e != cudaSuccess)
+        return e;
+    return launch_ex(attn_merge<D>, dim3((unsigned)p.Hkv, (unsigned)p.B), dim3(kAttnThreads), 0, st, 1, a);
+}
+
+cudaError_t launch_attn_any(const Plan &p, const AttnArgs &a, cudaStream_t st)
+{
+    if (p.D == 128)
+        return p.G <= 8 ? launch_attn_t<128, 1>(p, a, st) : launch_attn_t<128, 2>(p, a, st);
+    return p.G <= 8 ? launch_attn_t<64, 1>(p, a, st) : launch_attn_t<64, 2>(p, a, st);
+}
+
+AttnArgs make_args(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
+                   float *out)
+{
+    AttnArgs a;
+    a.k = static_cast<const __nv_bfloat16 *>(kv->k);
+    a.v = static_cast<const __nv_bfloat16 *>(kv->v);
+    a.st = kv->stride_tok;
+    a.sh = kv->stride_head;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.seq_off = kv->seq_offsets_dev;
+    a.ids = ids;
+    a.count = count;
+    a.cap = p.capacity;
+    a.out = out;
+    a.part = nullptr;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.splits = p.attn_splits;
+    a.scale_log2 = p.scale * kLog2e;
+    return a;
 }
 
 // ---------------------------------------------------------------------------
@@ -227,8 +379,7 @@ cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
 // every byte of device memory through their own pool and let no library call
 // cudaMalloc or take a workspace after start-up, and deployments whose memory
 // budget is fixed when the process initialises.  For them the split-K
-// partials and the per-(sequence, kv head) tickets live in this file-scope
-// array instead of a caller workspace.  Every GPU that loads the library holds
+// partials live in this file-scope array instead of a caller workspace.  Every GPU that loads the library holds
 // it until the process exits; all calls share it (and it keeps the last call's
 // contents), so calls that can overlap on the GPU race with each other.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
@@ -267,47 +418,22 @@ static uint8_t *noalloc_scratch_ptr(ts_status_t *status)
 ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
                                 const int32_t *count, float *out, cudaStream_t st)
 {
-    const size_t ticket_bytes = align_up(sizeof(uint32_t) * (size_t)p.B * p.Hkv, 256);
-    const size_t part_bytes = sizeof(float) * (size_t)p.B * p.Hkv * p.attn_splits * p.G * (p.D + 2);
-    if (ticket_bytes + part_bytes > kNoAllocScratchBytes) {
+    const size_t part_bytes = sizeof(float) * (size_t)p.B * p.Hkv * p.attn_splits * p.G * (p.D + 4);
+    if (part_bytes > kNoAllocScratchBytes) {
         set_error("ts_sparse_attn_noalloc: this shape needs %zu bytes of scratch, more than the fixed %zu; "
                   "use ts_sparse_attn with a workspace",
-                  ticket_bytes + part_bytes, kNoAllocScratchBytes);
+                  part_bytes, kNoAllocScratchBytes);
         return TS_ERR_UNSUPPORTED;
     }
     ts_status_t status;
     uint8_t *scratch = noalloc_scratch_ptr(&status);
     if (scratch == nullptr)
         return status;
-    // the tickets must start at zero whatever an earlier call left behind
-    cudaError_t e = cudaMemsetAsync(scratch, 0, ticket_bytes, st);
-    if (e != cudaSuccess) {
-        set_error("ts_sparse_attn_noalloc: clearing the tickets failed: %s", cudaGetErrorString(e));
-        return TS_ERR_CUDA;
-    }
-    AttnArgs a;
-    a.k = static_cast<const __nv_bfloat16 *>(kv->k);
-    a.v = static_cast<const __nv_bfloat16 *>(kv->v);
-    a.st = kv->stride_tok;
-    a.sh = kv->stride_head;
-    a.q = static_cast<const __nv_bfloat16 *>(q);
-    a.seq_off = kv->seq_offsets_dev;
-    a.ids = ids;
-    a.count = count;
-    a.cap = p.capacity;
-    a.out = out;
-    a.tickets = reinterpret_cast<uint32_t *>(scratch);
-    a.part = reinterpret_cast<float *>(scratch + ticket_bytes);
-    a.B = p.B;
-    a.Hq = p.Hq;
-    a.Hkv = p.Hkv;
-    a.G = p.G;
-    a.splits = p.attn_splits;
-    a.scale_log2 = p.scale * kLog2e;
-    if (p.D == 128)
-        e = p.G <= 8 ? launch_attn_t<128, 8>(p, a, st) : launch_attn_t<128, 16>(p, a, st);
-    else
-        e = p.G <= 8 ? launch_attn_t<64, 8>(p, a, st) : launch_attn_t<64, 16>(p, a, st);
+    // every partial the merge reads is written by the same call first, so
+    // nothing in the array has to start at zero
+    AttnArgs a = make_args(p, kv, q, ids, count, out);
+    a.part = reinterpret_cast<float *>(scratch);
+    cudaError_t e = launch_attn_any(p, a, st);
     if (e != cudaSuccess) {
         set_error("ts_sparse_attn_noalloc launch: %s", cudaGetErrorString(e));
         return TS_ERR_CUDA;
@@ -318,28 +444,9 @@ ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q,
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
                         float *out, uint8_t *ws, cudaStream_t st)
 {
-    AttnArgs a;
-    a.k = static_cast<const __nv_bfloat16 *>(kv->k);
-    a.v = static_cast<const __nv_bfloat16 *>(kv->v);
-    a.st = kv->stride_tok;
-    a.sh = kv->stride_head;
-    a.q = static_cast<const __nv_bfloat16 *>(q);
-    a.seq_off = kv->seq_offsets_dev;
-    a.ids = ids;
-    a.count = count;
-    a.cap = p.capacity;
-    a.out = out;
+    AttnArgs a = make_args(p, kv, q, ids, count, out);
     a.part = reinterpret_cast<float *>(ws + p.off_attn_part);
-    a.tickets = reinterpret_cast<uint32_t *>(ws + p.off_attn_tickets);
-    a.B = p.B;
-    a.Hq = p.Hq;
-    a.Hkv = p.Hkv;
-    a.G = p.G;
-    a.splits = p.attn_splits;
-    a.scale_log2 = p.scale * kLog2e;
-    if (p.D == 128)
-        return p.G <= 8 ? launch_attn_t<128, 8>(p, a, st) : launch_attn_t<128, 16>(p, a, st);
-    return p.G <= 8 ? launch_attn_t<64, 8>(p, a, st) : launch_attn_t<64, 16>(p, a, st);
+    return launch_attn_any(p, a, st);
 }
 
 }  // namespace ts

@@ -5,27 +5,33 @@
 //
 // For every active sequence b, KV head g and query head h = g*G + j:
 //   s[h, i] = scale * q[b, h, :] . K[b, i, g, :]        (fp32 accumulation)
-// written to the logits workspace [h_q][n_total], and
-//   L[b, h] = log sum_i exp(s[h, i])                   (float64 merge)
+// written to the logits workspace [h_q][ld], and
+//   L[b, h] = log sum_i exp(s[h, i])                   (score_merge below)
 //
 // Design (B200):
-//  * One CTA per SM, persistent over single-stage chunks of T tokens of the
-//    active sequences, dealt round-robin so that all CTAs sweep K together
-//    and the load is balanced to within one chunk.  A producer warp streams K with 3-D TMA boxes
-//    {64 channels, T tokens, h_kv heads} (128-byte swizzle, L2 evict-first)
-//    into a 6-stage ring of ~32 KB stages guarded by mbarriers.
+//  * One CTA per SM, persistent.  The active sequences' tokens are cut into
+//    chunks of T tokens (one pipeline stage, 32 KB of K); CTA j takes the
+//    contiguous, balanced chunk range [j*C/grid, (j+1)*C/grid), so a CTA
+//    spans one or two sequences and the load is balanced to one chunk.
+//  * A producer warp streams K with 3-D TMA boxes {64 channels, T tokens,
+//    h_kv heads} (128-byte swizzle, L2 evict-first) into a 6-stage ring of
+//    32 KB stages guarded by mbarriers.  Before waiting for the previous
+//    kernel in the stream it already asks L2 for its first tiles, so the
+//    first DRAM round trip overlaps that kernel.
 //  * Eight consumer warps each own one KV head g and a share of the 16-token
 //    row blocks of a stage.  The G query heads of g are the N dimension of a
 //    bf16 m16n8k16 tensor-core tile (N = 8 covers G <= 8; two tiles for
 //    G <= 16), K rows the M dimension, the head dimension K: the Q fragments
-//    live in registers for the whole chunk; K fragments come from shared
-//    memory with ldmatrix (conflict-free thanks to the swizzle).
+//    live in registers; K fragments come from shared memory with ldmatrix
+//    (conflict-free thanks to the swizzle).
 //  * The epilogue scales, stores the logits and keeps an online
-//    (max, sum exp) per head and thread over all of the CTA's chunks of a
-//    sequence; when the CTA leaves the sequence these are reduced over the
-//    CTA and written as one partial per (CTA, sequence, head).
-//  * The CTA that finishes the last chunk of a sequence (atomic ticket, no
-//    waiting) merges that sequence's partials in float64 into L[b, :].
+//    (max, sum exp) per head and thread over the CTA's chunks of a sequence;
+//    when the CTA leaves the sequence these are reduced over the CTA and
+//    written as one partial, at the slot of the CTA's first chunk in that
+//    sequence.  No fences, atomics or waits on other CTAs.
+//  * score_merge (one block per sequence and 8 heads) folds the <= grid
+//    partials of a sequence into L[b, :] after the pass: fp32 terms
+//    exp(m - M) <= 1 summed in float64.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -33,6 +39,7 @@ namespace ts {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPrefetchTiles = kScoreStages;
 
 struct ScoreArgs {
     const __nv_bfloat16 *q;   // [B, Hq, D]
@@ -41,13 +48,11 @@ struct ScoreArgs {
     float *logits;            // [Hq][ld]
     int64_t ld;
     float2 *partials;         // [max_chunks][Hq] (max, sum exp(x - max))
-    uint32_t *tickets;        // [B]
-    double *L;                // [B][Hq]
-    uint32_t *ctrl;
+    int32_t *chunk_table;     // [B + 1] first active chunk of each sequence (for score_merge)
+    uint32_t *ctrl;           // status word
     int B, Hq, Hkv, G;
-    int T;                    // tokens per stage
+    int T;                    // tokens per chunk / stage
     int stage_bytes;
-    int64_t chunk_tokens;
     float scale;
 };
 
@@ -57,8 +62,6 @@ struct __align__(16) ScoreShared {
     int64_t off[kMaxBatch + 1];
     int32_t chunk_start[kMaxBatch + 1];
     float2 red[kScoreConsumerWarps][16];
-    int32_t abort;
-    int32_t last;
 };
 
 __device__ __forceinline__ void online_push(float &m, float &z, float x)
@@ -69,6 +72,46 @@ __device__ __forceinline__ void online_push(float &m, float &z, float x)
     } else {
         z += exp2f((x - m) * kLog2e);
     }
+}
+
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int32_t x, int32_t y, int32_t z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// chunk_start[b] (b <= B): first chunk of sequence b, leaving out sequences
+// that reuse their selection when use_reuse is set.  Every thread calls it.
+__device__ __forceinline__ void build_chunk_table(ScoreShared &sh, const int32_t *reuse, int B, int T, int warp,
+                                                  int lane, bool use_reuse)
+{
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int64_t n = sh.off[b + 1] - sh.off[b];
+        const bool active = !use_reuse || reuse == nullptr || reuse[b] == 0;
+        sh.chunk_start[b + 1] = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int32_t run = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int b = base + lane;
+            int32_t x = (b < B) ? sh.chunk_start[b + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o)
+                    x += y;
+            }
+            if (b < B)
+                sh.chunk_start[b + 1] = run + x;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0)
+            sh.chunk_start[0] = 0;
+    }
+    __syncthreads();
 }
 
 template <int D, int NB>
@@ -83,33 +126,60 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int B = a.B;
+    const int T = a.T;
 
-    // ---- sequence table: chunk_start[b] = first chunk of sequence b -------
-    for (int b = tid; b <= B; b += blockDim.x)
-        sh.off[b] = a.seq_off[b];
     if (tid == 0) {
         for (int s = 0; s < kScoreStages; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], kScoreConsumerWarps);
         }
-        sh.abort = 0;
         mbar_fence_init();
     }
+    // ---- before the previous kernel has finished: only L2 prefetch hints,
+    //      computed as if every sequence were active (a wrong guess costs
+    //      nothing but bandwidth; the data itself is read after the wait) -----
+    for (int b = tid; b <= B; b += blockDim.x)
+        sh.off[b] = a.seq_off[b];
+    __syncthreads();
+    build_chunk_table(sh, a.reuse, B, T, warp, lane, false);
+    if (warp == kScoreConsumerWarps && lane == 0) {
+        tma_prefetch_desc(&kmap);
+        const int32_t total = sh.chunk_start[B];
+        const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
+        const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
+        for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
+            const int b = upper_seq(sh.chunk_start, B, v);
+            const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x)
+                tma_prefetch_l2_3d(&kmap, x * 64, (int32_t)t0, 0);
+        }
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+
+    // ---- the real chunk table (reuse flags come from the previous kernel);
+    //      the offsets are re-read too, in case a caller's kernel wrote them;
+    //      offsets and flags are loaded together: one round trip -------------
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) {
-        int64_t n = sh.off[b + 1] - sh.off[b];
-        bool active = (a.reuse == nullptr) || (a.reuse[b] == 0);
-        sh.chunk_start[b + 1] = (active && n > 0) ? (int32_t)((n + a.chunk_tokens - 1) / a.chunk_tokens) : 0;
+        const int64_t o0 = a.seq_off[b], o1 = a.seq_off[b + 1];
+        const bool active = a.reuse == nullptr || a.reuse[b] == 0;
+        sh.off[b] = o0;
+        if (b == B - 1)
+            sh.off[B] = o1;
+        const int64_t n = o1 - o0;
+        sh.chunk_start[b + 1] = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
     }
     __syncthreads();
     if (warp == 0) {
         int32_t run = 0;
         for (int base = 0; base < B; base += 32) {
-            int b = base + lane;
+            const int b = base + lane;
             int32_t x = (b < B) ? sh.chunk_start[b + 1] : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
                 if (lane >= o)
                     x += y;
             }
@@ -121,39 +191,36 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             sh.chunk_start[0] = 0;
     }
     __syncthreads();
-    const int32_t total_chunks = sh.chunk_start[B];
-    const int T = a.T;
+    if (blockIdx.x == 0)
+        for (int b = tid; b <= B; b += blockDim.x)
+            a.chunk_table[b] = sh.chunk_start[b];
+    const int32_t total = sh.chunk_start[B];
+    const int32_t v_begin = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
+    const int32_t v_end = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
     const int Hkv = a.Hkv;
     const int half_bytes = T * Hkv * 128;   // one 64-channel box
 
     if (warp == kScoreConsumerWarps) {
         // ================= producer: one elected lane issues TMA ==========
         if (lane == 0) {
-            tma_prefetch_desc(&kmap);
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
-            for (int32_t v = blockIdx.x; v < total_chunks; v += gridDim.x) {
+            for (int32_t v = v_begin; v < v_end; ++v, ++it) {
                 const int b = upper_seq(sh.chunk_start, B, v);
-                const int64_t lo = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * a.chunk_tokens;
-                const int64_t hi = min(lo + a.chunk_tokens, sh.off[b + 1]);
-                for (int64_t t0 = lo; t0 < hi; t0 += T, ++it) {
-                    const int s = it % kScoreStages;
-                    if (it >= kScoreStages) {
-                        const uint32_t par = ((it / kScoreStages) - 1) & 1;
-                        if (*(volatile int32_t *)&sh.abort ||
-                            !mbar_wait_bounded(&sh.empty[s], par, kSpinLimit)) {
-                            if (!*(volatile int32_t *)&sh.abort)
-                                report_timeout(a.ctrl, kSiteScoreEmpty);
-                            *(volatile int32_t *)&sh.abort = 1;
-                            continue;
-                        }
+                const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+                const int s = it % kScoreStages;
+                if (it >= kScoreStages) {
+                    const uint32_t par = ((it / kScoreStages) - 1) & 1;
+                    if (!mbar_wait_bounded(&sh.empty[s], par, kSpinLimit)) {
+                        report_timeout(a.ctrl, kSiteScoreEmpty);
+                        break;   // nothing issued after this: the consumers time out on full[] too
                     }
-                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
-#pragma unroll
-                    for (int x = 0; x < D / 64; ++x)
-                        tma_load_3d(stages + (size_t)s * a.stage_bytes + x * half_bytes, &kmap, &sh.full[s],
-                                    x * 64, (int32_t)t0, 0, pol);
                 }
+                mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_3d(stages + (size_t)s * a.stage_bytes + x * half_bytes, &kmap, &sh.full[s], x * 64,
+                                (int32_t)t0, 0, pol);
             }
         }
         return;
@@ -173,13 +240,13 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     uint32_t bq[D / 16][NB][2];
     float m[NB][2], z[NB][2];
     int cur_b = -1;
-    int32_t seg_first = 0, seg_count = 0;
+    int32_t seg_first = 0;
     uint32_t it = 0;
+    bool dead = false;
 
-    // Close this CTA's run of chunks of sequence sb: reduce (max, sum) per
-    // head over the CTA, publish one partial at slot seg_first, and let the
-    // CTA that completes the sequence's last chunk merge its partials.
-    auto flush_segment = [&](int sb) {
+    // Close this CTA's run of chunks of a sequence: reduce (max, sum) per head
+    // over the CTA and publish one partial at slot seg_first.
+    auto flush_segment = [&]() {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -201,56 +268,19 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
                 lse_merge(M, Z, sh.red[w2][j].x, sh.red[w2][j].y);
             a.partials[(int64_t)seg_first * a.Hq + h] = make_float2(M, Z);
         }
-        __threadfence();
-        named_bar_sync(1, kScoreConsumerWarps * 32);
-        if (ctid == 0) {
-            const uint32_t nch = (uint32_t)(sh.chunk_start[sb + 1] - sh.chunk_start[sb]);
-            const uint32_t t = atomicAdd(&a.tickets[sb], (uint32_t)seg_count);
-            sh.last = (t + (uint32_t)seg_count == nch) ? 1 : 0;
-        }
-        named_bar_sync(1, kScoreConsumerWarps * 32);
-        if (sh.last) {
-            // Every CTA that took chunks of sb wrote its partial at the slot of
-            // its first chunk there: slots [cs, cs + min(nc, gridDim.x)).
-            __threadfence();
-            const int32_t cs = sh.chunk_start[sb];
-            const int32_t nslots = min(sh.chunk_start[sb + 1] - cs, (int32_t)gridDim.x);
-            for (int h = warp; h < a.Hq; h += kScoreConsumerWarps) {
-                float M = -INFINITY;
-                for (int c = lane; c < nslots; c += 32)
-                    M = fmaxf(M, __ldcg(&a.partials[(int64_t)(cs + c) * a.Hq + h]).x);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                double Z = 0.0;
-                for (int c = lane; c < nslots; c += 32) {
-                    const float2 p = __ldcg(&a.partials[(int64_t)(cs + c) * a.Hq + h]);
-                    if (p.y > 0.0f)
-                        Z += (double)p.y * exp((double)p.x - (double)M);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    Z += __shfl_xor_sync(0xffffffffu, Z, o);
-                if (lane == 0)
-                    a.L[(int64_t)sb * a.Hq + h] = (double)M + log(Z);
-            }
-            if (ctid == 0)
-                a.tickets[sb] = 0u;
-        }
-        named_bar_sync(1, kScoreConsumerWarps * 32);
+        named_bar_sync(1, kScoreConsumerWarps * 32);   // sh.red is rewritten by the next flush
     };
 
-    for (int32_t v = blockIdx.x; v < total_chunks; v += gridDim.x) {
+    for (int32_t v = v_begin; v < v_end; ++v, ++it) {
         const int b = upper_seq(sh.chunk_start, B, v);
-        const int64_t lo = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * a.chunk_tokens;
-        const int64_t hi = min(lo + a.chunk_tokens, sh.off[b + 1]);
+        const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+        const int64_t hi = sh.off[b + 1];
 
         if (b != cur_b) {
             if (cur_b >= 0)
-                flush_segment(cur_b);
+                flush_segment();
             cur_b = b;
             seg_first = v;
-            seg_count = 0;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
@@ -274,67 +304,122 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
                     z[nb][cc] = 0.0f;
                 }
         }
-        ++seg_count;
 
-        for (int64_t t0 = lo; t0 < hi; t0 += T, ++it) {
-            const int s = it % kScoreStages;
-            const uint32_t par = (it / kScoreStages) & 1;
-            bool ok = !*(volatile int32_t *)&sh.abort;
-            if (ok && !mbar_wait_bounded(&sh.full[s], par, kSpinLimit)) {
-                report_timeout(a.ctrl, kSiteScoreFull);
-                *(volatile int32_t *)&sh.abort = 1;
-                ok = false;
-            }
-            if (ok) {
-                const uint32_t stage_base = smem_u32(stages + (size_t)s * a.stage_bytes);
-                for (int mb = wsub; mb < mblocks; mb += nsub) {
-                    float acc[NB][4];
+        const int s = it % kScoreStages;
+        const uint32_t par = (it / kScoreStages) & 1;
+        if (!dead && !mbar_wait_bounded(&sh.full[s], par, kSpinLimit)) {
+            report_timeout(a.ctrl, kSiteScoreFull);
+            dead = true;
+        }
+        if (!dead) {
+            const uint32_t stage_base = smem_u32(stages + (size_t)s * a.stage_bytes);
+            for (int mb = wsub; mb < mblocks; mb += nsub) {
+                float acc[NB][4];
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc[nb][e] = 0.0f;
+                const int trow = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t row_addr = stage_base + (uint32_t)((g * T + trow) * 128);
+                const int swz = trow & 7;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int chunk = (ks & 3) * 2 + (lane >> 4);
+                    const uint32_t addr =
+                        row_addr + (uint32_t)((ks >> 2) * half_bytes) + (uint32_t)((chunk ^ swz) << 4);
+                    uint32_t a0, a1, a2, a3;
+                    ldmatrix_x4(a0, a1, a2, a3, addr);
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb)
+                        mma_16816(acc[nb], a0, a1, a2, a3, bq[ks][nb][0], bq[ks][nb][1]);
+                }
+                // epilogue: rows r0 and r0 + 8 of this block, columns c0, c0 + 1
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            acc[nb][e] = 0.0f;
-                    const int trow = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t row_addr = stage_base + (uint32_t)((g * T + trow) * 128);
-                    const int swz = trow & 7;
-#pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const int chunk = (ks & 3) * 2 + (lane >> 4);
-                        const uint32_t addr = row_addr + (uint32_t)((ks >> 2) * half_bytes) +
-                                              (uint32_t)((chunk ^ swz) << 4);
-                        uint32_t a0, a1, a2, a3;
-                        ldmatrix_x4(a0, a1, a2, a3, addr);
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int64_t tok = t0 + mb * 16 + r0 + rr * 8;
+                    if (tok < hi) {
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb)
-                            mma_16816(acc[nb], a0, a1, a2, a3, bq[ks][nb][0], bq[ks][nb][1]);
-                    }
-                    // epilogue: rows r0 and r0 + 8 of this block, columns c0, c0 + 1
 #pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int64_t tok = t0 + mb * 16 + r0 + rr * 8;
-                        if (tok < hi) {
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                                for (int cc = 0; cc < 2; ++cc) {
-                                    const int j = nb * 8 + c0 + cc;
-                                    if (j < G) {
-                                        const float x = acc[nb][rr * 2 + cc] * scale;
-                                        a.logits[(int64_t)(g * G + j) * a.ld + tok] = x;
-                                        online_push(m[nb][cc], z[nb][cc], x);
-                                    }
+                            for (int cc = 0; cc < 2; ++cc) {
+                                const int j = nb * 8 + c0 + cc;
+                                if (j < G) {
+                                    const float x = acc[nb][rr * 2 + cc] * scale;
+                                    a.logits[(int64_t)(g * G + j) * a.ld + tok] = x;
+                                    online_push(m[nb][cc], z[nb][cc], x);
                                 }
-                        }
+                            }
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sh.empty[s]);
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sh.empty[s]);
     }
     if (cur_b >= 0)
-        flush_segment(cur_b);
+        flush_segment();
+}
+
+// L[b, h] from the partials of sequence b: every CTA whose chunk range meets
+// [cs, ce) wrote one partial, at slot max(start_j, cs).
+__global__ void __launch_bounds__(256)
+score_merge(const float2 *partials, const int32_t *chunk_table, double *L, int B, int Hq, int grid_a)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.x;
+    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    __shared__ int32_t s_start[257];
+    const int32_t cs = chunk_table[b], ce = chunk_table[b + 1], total = chunk_table[B];
+    if (cs == ce)
+        return;   // reused or empty sequence: its L is not needed
+    for (int j = threadIdx.x; j <= grid_a; j += blockDim.x)
+        s_start[j] = (int32_t)((int64_t)j * total / grid_a);   // CTA j's chunk range starts here
+    __syncthreads();
+    if (h >= Hq)
+        return;
+    auto start_of = [&](int j) { return s_start[j]; };
+    auto owner = [&](int32_t v) {   // largest j with start_of(j) <= v
+        int lo = 0, hi = grid_a;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (start_of(mid) <= v)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        return lo;
+    };
+    const int j0 = owner(cs), j1 = owner(ce - 1);
+    constexpr int kPer = 8;   // slots per lane: grid_a <= 256
+    float2 pv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int j = j0 + lane + 32 * i;
+        pv[i] = make_float2(-INFINITY, 0.0f);
+        if (j <= j1 && start_of(j) < start_of(j + 1))   // CTAs with empty ranges wrote nothing
+            pv[i] = __ldcg(&partials[(int64_t)max(start_of(j), cs) * Hq + h]);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        M = fmaxf(M, pv[i].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    double Z = 0.0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        if (pv[i].y > 0.0f)
+            Z += (double)(pv[i].y * exp2f((pv[i].x - M) * kLog2e));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        Z += __shfl_xor_sync(0xffffffffu, Z, o);
+    if (lane == 0)
+        L[(int64_t)b * Hq + h] = (double)M + log(Z);
 }
 
 template <int D, int NB>
@@ -351,8 +436,8 @@ cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, const ScoreAr
             return e;
         configured_dev = dev;
     }
-    score_pass_a<D, NB><<<p.score_grid, kScoreThreads, dyn, st>>>(kmap, args);
-    return cudaGetLastError();
+    return launch_ex(score_pass_a<D, NB>, dim3((unsigned)p.score_grid), dim3(kScoreThreads), dyn, st, 1, kmap,
+                     args);
 }
 
 }  // namespace
@@ -365,10 +450,9 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.seq_off = seq_off;
     a.reuse = reuse;
     a.logits = reinterpret_cast<float *>(ws + p.off_logits);
-    a.ld = p.n_total;
+    a.ld = p.ld_logits;
     a.partials = reinterpret_cast<float2 *>(ws + p.off_partials);
-    a.tickets = reinterpret_cast<uint32_t *>(ws + p.off_score_tickets);
-    a.L = reinterpret_cast<double *>(ws + p.off_L);
+    a.chunk_table = reinterpret_cast<int32_t *>(ws + p.off_chunk_table);
     a.ctrl = reinterpret_cast<uint32_t *>(ws + p.off_ctrl);
     a.B = p.B;
     a.Hq = p.Hq;
@@ -376,11 +460,18 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.G = p.G;
     a.T = p.tile_tokens;
     a.stage_bytes = p.stage_bytes;
-    a.chunk_tokens = p.chunk_tokens;
     a.scale = p.scale;
+    cudaError_t e;
     if (p.D == 128)
-        return p.G <= 8 ? launch_score_t<128, 1>(p, kmap, a, st) : launch_score_t<128, 2>(p, kmap, a, st);
-    return p.G <= 8 ? launch_score_t<64, 1>(p, kmap, a, st) : launch_score_t<64, 2>(p, kmap, a, st);
+        e = p.G <= 8 ? launch_score_t<128, 1>(p, kmap, a, st) : launch_score_t<128, 2>(p, kmap, a, st);
+    else
+        e = p.G <= 8 ? launch_score_t<64, 1>(p, kmap, a, st) : launch_score_t<64, 2>(p, kmap, a, st);
+    if (e != cudaSuccess)
+        return e;
+    return launch_ex(score_merge, dim3((unsigned)p.B, (unsigned)((p.Hq + 7) / 8)), dim3(256), 0, st, 1,
+                     reinterpret_cast<const float2 *>(ws + p.off_partials),
+                     reinterpret_cast<const int32_t *>(ws + p.off_chunk_table),
+                     reinterpret_cast<double *>(ws + p.off_L), p.B, p.Hq, p.score_grid);
 }
 
 }  // namespace ts

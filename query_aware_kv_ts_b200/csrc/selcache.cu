@@ -14,22 +14,40 @@ namespace {
 constexpr int kSelcacheThreads = 256;
 
 __global__ void __launch_bounds__(kSelcacheThreads)
-selcache_kernel(const uint32_t *q, uint32_t *q_prev, int32_t *reuse, double *cos_out, int first_step,
+selcache_kernel(const uint32_t *__restrict__ q, uint32_t *__restrict__ q_prev, int32_t *reuse, double *cos_out, int first_step,
                 int len_pairs, double theta)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     const int b = blockIdx.x;
-    const uint32_t *qb = q + (int64_t)b * len_pairs;
-    uint32_t *pb = q_prev + (int64_t)b * len_pairs;
+    const uint32_t *__restrict__ qb = q + (int64_t)b * len_pairs;
+    uint32_t *__restrict__ pb = q_prev + (int64_t)b * len_pairs;
+    // Loads are issued in batches before any store, so that a thread waits
+    // on memory once per batch instead of once per element.
     double ab = 0.0, aa = 0.0, bb = 0.0;
-    for (int i = threadIdx.x; i < len_pairs; i += blockDim.x) {
-        const uint32_t x = qb[i];
-        const uint32_t y = pb[i];
-        const double x0 = bf16_lo(x), x1 = bf16_hi(x);
-        const double y0 = bf16_lo(y), y1 = bf16_hi(y);
-        ab += x0 * y0 + x1 * y1;
-        aa += x0 * x0 + x1 * x1;
-        bb += y0 * y0 + y1 * y1;
-        pb[i] = x;
+    constexpr int kBatch = 8;
+    for (int i0 = threadIdx.x; i0 < len_pairs; i0 += kBatch * kSelcacheThreads) {
+        uint32_t xs[kBatch], ys[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kSelcacheThreads;
+            xs[u] = i < len_pairs ? __ldcg(qb + i) : 0u;
+            ys[u] = i < len_pairs ? __ldcg(pb + i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const double x0 = bf16_lo(xs[u]), x1 = bf16_hi(xs[u]);
+            const double y0 = bf16_lo(ys[u]), y1 = bf16_hi(ys[u]);
+            ab += x0 * y0 + x1 * y1;
+            aa += x0 * x0 + x1 * x1;
+            bb += y0 * y0 + y1 * y1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kSelcacheThreads;
+            if (i < len_pairs)
+                pb[i] = xs[u];
+        }
     }
     __shared__ double red[3][kSelcacheThreads / 32];
 #pragma unroll
@@ -45,13 +63,19 @@ selcache_kernel(const uint32_t *q, uint32_t *q_prev, int32_t *reuse, double *cos
         red[2][warp] = bb;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        double sab = 0.0, saa = 0.0, sbb = 0.0;
-        for (int w = 0; w < kSelcacheThreads / 32; ++w) {
-            sab += red[0][w];
-            saa += red[1][w];
-            sbb += red[2][w];
+    if (warp == 0) {
+        constexpr int kW = kSelcacheThreads / 32;
+        double sab = lane < kW ? red[0][lane] : 0.0;
+        double saa = lane < kW ? red[1][lane] : 0.0;
+        double sbb = lane < kW ? red[2][lane] : 0.0;
+#pragma unroll
+        for (int o = kW / 2; o > 0; o >>= 1) {
+            sab += __shfl_xor_sync(0xffffffffu, sab, o);
+            saa += __shfl_xor_sync(0xffffffffu, saa, o);
+            sbb += __shfl_xor_sync(0xffffffffu, sbb, o);
         }
+        if (lane != 0)
+            return;
         double c = 0.0;
         int r = 0;
         if (!first_step) {
@@ -69,10 +93,9 @@ selcache_kernel(const uint32_t *q, uint32_t *q_prev, int32_t *reuse, double *cos
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step, int B,
                             int len, double theta, cudaStream_t st)
 {
-    selcache_kernel<<<B, kSelcacheThreads, 0, st>>>(static_cast<const uint32_t *>(q),
-                                                    static_cast<uint32_t *>(q_prev), reuse, cos_out, first_step,
-                                                    len / 2, theta);
-    return cudaGetLastError();
+    return launch_ex(selcache_kernel, dim3((unsigned)B), dim3(kSelcacheThreads), 0, st, 1,
+                     static_cast<const uint32_t *>(q), static_cast<uint32_t *>(q_prev), reuse, cos_out, first_step,
+                     len / 2, theta);
 }
 
 }  // namespace ts

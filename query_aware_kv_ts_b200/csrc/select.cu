@@ -2,60 +2,94 @@
 // (TokenSelect README summary: a small number of critical KV tokens take part
 // in attention; the vote ordering with ties to the lower token id).
 //
-// One thread-block cluster (8 CTAs, 1024 threads each) per sequence.  The
-// candidates [s', l0) are split into 8 contiguous ranges, one per CTA.
+// Order.  Candidate token i of a sequence gets the 64-bit key
+//   key(i) = (bits(v_i) << 32) | (0xffffffff - i)
+// Votes are non-negative fp32, so their bit patterns order like the values,
+// and the low word makes equal votes order by ascending id: the top k keys
+// are exactly the top k tokens with ties to the lower id, and "token i is
+// selected" is key(i) >= T, T the k-th largest key.
 //
-// Exact radix select of the k-th largest vote.  Votes are non-negative fp32,
-// so their bit patterns order like the values.  Three digit levels
-// (bits 31..20, 19..8, 7..0): each CTA builds a shared-memory histogram of
-// its range (restricted to keys matching the digits found so far), the
-// cluster reduces it through distributed shared memory (CTA r owns bin slice
-// r), and every CTA locates the bin holding the k-th largest key.  After three
-// levels the k-th largest key vk is known exactly, together with r = the
-// number of tokens equal to vk that belong to the top k (the lowest-id ties).
-//
-// Ordered compaction: token i of the candidates is selected iff
-// key(i) > vk, or key(i) == vk and fewer than r ties precede it.  Per-CTA
-// counts exchanged over the cluster give each CTA its output offset; a
-// block-wide scan places ids in ascending order.  CTA 0 writes the sink and
-// local windows and the count; the tail of the id row is padded with -1.
-// Cluster barriers are hardware barriers: there is no software spin here.
-#include <cooperative_groups.h>
-
+// Four short kernels spread over the whole GPU (grid: ranges of kTPC
+// candidates x sequences), except the per-sequence resolve step:
+//  S0 sel_hist     histogram of the top 12 vote bits of the candidates
+//                  (shared-memory histogram per range, then global atomics)
+//  S2 sel_collect  every range finds the bin b1 that holds the k-th largest
+//                  vote, counts its candidates above b1 and appends the ones
+//                  inside b1 to the sequence's candidate list
+//  S3 sel_resolve  one CTA per sequence: exact radix select of T among the
+//                  (few) b1 candidates, 8-bit digits over the 52 key bits
+//                  below b1; range offsets = each range's candidates above b1
+//                  plus its b1 candidates >= T, prefix-summed; clears the
+//                  histogram and the list counter for the next call
+//  S4 sel_write    every range writes its selected ids in ascending order at
+//                  its offset (one block scan); range 0 also writes the sink
+//                  and local windows, the count and the -1 padding
+// No kernel waits on another CTA: the four steps are ordered by the stream.
 #include "ts_device.cuh"
 #include "ts_internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace ts {
 namespace {
 
-constexpr int CS = kSelectClusterSize;
-constexpr int NT = kSelectThreads;
+constexpr int NT = kSelectThreads;          // 256
 constexpr int kWarps = NT / 32;
+constexpr int kTPC = kSelectTokensPerCta;   // candidates per range (per CTA)
+constexpr int kPer = kTPC / NT;             // candidates per thread
+constexpr int kResolveSmem = 2560;          // b1 candidates kept in shared memory by S3
 
-struct SelectArgs {
-    const uint32_t *votes;   // fp32 vote bits [n_total]
+struct SelArgs {
+    const uint32_t *votes;     // fp32 vote bits [n_total]
     const int64_t *seq_off;
     const int32_t *reuse;
-    int32_t *ids;            // [B][cap]
-    int32_t *count;          // [B]
-    int k, n_sink, n_local, cap;
+    int32_t *ids;              // [B][cap]
+    int32_t *count;            // [B]
+    uint32_t *hist;            // [B][4096]
+    uint2 *cand;               // [n_total] (vote bits, token id), sequence b's list at seq_off[b]
+    uint32_t *cand_n;          // [B]
+    uint32_t *above;           // [B][rps] candidates above bin b1, per range
+    uint32_t *range_off;       // [B][rps] output offset of each range within the top-k part
+    unsigned long long *thr;   // [B] threshold key T
+    int32_t *mode;             // [B] 0: none, 1: keys >= T, 2: every candidate
+    int k, n_sink, n_local, cap, B, rps;
 };
 
-struct SelectShared {
-    uint32_t hist[4096];
-    uint32_t red[4096 / CS];      // this CTA's cluster-reduced bin slice
-    uint32_t rev[4096 / CS];      // copy of the slice holding the target
-    uint32_t warp_tmp[kWarps + 1];
-    uint32_t slice_total;
-    uint32_t cnt[2];              // this CTA's (above, ties)
-    uint32_t bcast[4];
+struct Window {
+    int64_t off, n, s_end, l0, nc, keff;
 };
 
-// Exclusive scan over the block of one value per thread; returns the
-// exclusive prefix and sets `total`.  Every thread of the block must call it.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *warp_tmp, uint32_t &total)
+__device__ __forceinline__ Window window_of(const SelArgs &a, int b)
+{
+    Window w;
+    w.off = a.seq_off[b];
+    w.n = a.seq_off[b + 1] - w.off;
+    w.s_end = min((int64_t)a.n_sink, w.n);
+    w.l0 = max(w.n - (int64_t)a.n_local, w.s_end);
+    w.nc = w.l0 - w.s_end;
+    w.keff = min((int64_t)a.k, w.nc);
+    return w;
+}
+
+__device__ __forceinline__ unsigned long long make_key(uint32_t vbits, int64_t id)
+{
+    return ((unsigned long long)vbits << 32) | (unsigned long long)(0xffffffffu - (uint32_t)id);
+}
+
+// Copy the 4096-bin histogram of sequence b into shared memory, every load of
+// the thread issued before the first store.
+__device__ __forceinline__ void load_hist(uint32_t *h, const uint32_t *gh)
+{
+    constexpr int kPerThread = 4096 / NT;
+    uint32_t v[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u)
+        v[u] = __ldcg(gh + u * NT + threadIdx.x);
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u)
+        h[u * NT + threadIdx.x] = v[u];
+}
+
+// Exclusive scan over the block of one value per thread (all threads call).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *tmp, uint32_t &total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t incl = x;
@@ -66,10 +100,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *warp_t
             incl += y;
     }
     if (lane == 31)
-        warp_tmp[warp] = incl;
+        tmp[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const uint32_t w = (lane < kWarps) ? warp_tmp[lane] : 0u;
+        const uint32_t w = lane < kWarps ? tmp[lane] : 0u;
         uint32_t wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -78,229 +112,373 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *warp_t
                 wi += y;
         }
         if (lane < kWarps)
-            warp_tmp[lane] = wi - w;
+            tmp[lane] = wi - w;
         if (lane == kWarps - 1)
-            warp_tmp[kWarps] = wi;
+            tmp[kWarps] = wi;
     }
     __syncthreads();
-    const uint32_t excl = warp_tmp[warp] + incl - x;
-    total = warp_tmp[kWarps];
+    const uint32_t ex = tmp[warp] + incl - x;
+    total = tmp[kWarps];
     __syncthreads();
-    return excl;
+    return ex;
 }
 
-// Sum over the block; every thread gets the result.
-__device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t *warp_tmp)
+// In a histogram of nb bins (bin nb-1 on top, nb a multiple of NT), the bin
+// holding the need-th key counted from the top, and the keys above it.
+// Each thread owns nb / NT consecutive bins from the top.  All threads call.
+__device__ __forceinline__ void bin_from_top(const uint32_t *h, int nb, int64_t need, uint32_t *tmp,
+                                             uint32_t *bc, uint32_t &bin, uint32_t &above)
 {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        x += __shfl_xor_sync(0xffffffffu, x, o);
-    if ((threadIdx.x & 31) == 0)
-        warp_tmp[threadIdx.x >> 5] = x;
+    const int per = nb / NT;
+    const int r0 = threadIdx.x * per;   // reversed index r: bin nb-1-r
+    uint32_t local = 0;
+    for (int r = r0; r < r0 + per; ++r)
+        local += h[nb - 1 - r];
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(local, tmp, tot);
+    int64_t cum = ex;
+    if (cum < need && cum + (int64_t)local >= need) {
+        for (int r = r0; r < r0 + per; ++r) {
+            const uint32_t c = h[nb - 1 - r];
+            if (cum + (int64_t)c >= need) {
+                bc[0] = (uint32_t)(nb - 1 - r);
+                bc[1] = (uint32_t)cum;
+                break;
+            }
+            cum += c;
+        }
+    }
     __syncthreads();
-    uint32_t t = 0;
-    for (int w = 0; w < kWarps; ++w)
-        t += warp_tmp[w];
+    bin = bc[0];
+    above = bc[1];
     __syncthreads();
-    return t;
 }
 
-__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NT, 1)
-select_kernel(const SelectArgs a)
+// ---------------------------------------------------------------------------
+// S0: level-1 histogram (top 12 bits) of the candidates
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(NT)
+sel_hist(const SelArgs a)
 {
-    __shared__ SelectShared sh;
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = (int)cluster.block_rank();
-    const int b = blockIdx.x / CS;
-    const int tid = threadIdx.x;
-
+    __shared__ uint32_t h[4096];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.y, r = blockIdx.x;
     if (a.reuse != nullptr && a.reuse[b] != 0)
-        return;   // whole cluster: the previous ids stay
-
-    const int64_t off = a.seq_off[b];
-    const int64_t n = a.seq_off[b + 1] - off;
-    const int64_t s_end = min((int64_t)a.n_sink, n);
-    const int64_t l0 = max(n - (int64_t)a.n_local, s_end);
-    const int64_t nc = l0 - s_end;
-    const int64_t keff = min((int64_t)a.k, nc);
-    const uint32_t *vb = a.votes + off;
-    const int64_t my_lo = s_end + nc * rank / CS;
-    const int64_t my_hi = s_end + nc * (rank + 1) / CS;
-    int32_t *idrow = a.ids + (int64_t)b * a.cap;
-
-    // mode 0: radix select, 1: every candidate, 2: none
-    const int mode = (keff == nc) ? 1 : (keff == 0 ? 2 : 0);
-    uint32_t vk = 0;
-    int64_t r_ties = 0;
-    uint32_t my_above = 0, my_ties = 0;   // this CTA's keys > vk and == vk
-
-    if (mode == 0) {
-        uint32_t prefix = 0, pmask = 0;
-        int64_t need = keff;
-#pragma unroll 1
-        for (int level = 0; level < 3; ++level) {
-            const int shift = level == 0 ? 20 : (level == 1 ? 8 : 0);
-            const int bins = level == 2 ? 256 : 4096;
-            const int W = bins / CS;
-            for (int i = tid; i < bins; i += NT)
-                sh.hist[i] = 0u;
-            __syncthreads();
-            for (int64_t i = my_lo + tid; i < my_hi; i += NT) {
-                const uint32_t key = __ldcg(vb + i);
-                if ((key & pmask) == prefix)
-                    atomicAdd(&sh.hist[(key >> shift) & (uint32_t)(bins - 1)], 1u);
-            }
-            __syncthreads();
-            cluster.sync();
-            // reduce my slice of bins over the cluster
-            uint32_t part = 0;
-            for (int j = tid; j < W; j += NT) {
-                uint32_t s = 0;
+        return;
+    const Window w = window_of(a, b);
+    const int64_t lo = w.s_end + (int64_t)r * kTPC;
+    if (w.keff == 0 || w.keff == w.nc || lo >= w.l0)
+        return;
+    const int64_t hi = min(lo + kTPC, w.l0);
+    for (int i = threadIdx.x; i < 4096; i += NT)
+        h[i] = 0u;
+    const uint32_t *vb = a.votes + w.off;
+    uint32_t kk[kPer];
 #pragma unroll
-                for (int q = 0; q < CS; ++q)
-                    s += cluster.map_shared_rank(sh.hist, q)[rank * W + j];
-                sh.red[j] = s;
-                part += s;
-            }
-            part = block_sum(part, sh.warp_tmp);
-            if (tid == 0)
-                sh.slice_total = part;
-            cluster.sync();
-            // which slice (from the top) holds the need-th largest key?
-            if (tid == 0) {
-                int64_t cum = 0;
-                int sel = 0;
-                for (int q = CS - 1; q >= 0; --q) {
-                    const uint32_t t = *cluster.map_shared_rank(&sh.slice_total, q);
-                    if (cum + (int64_t)t >= need) {
-                        sel = q;
-                        break;
-                    }
-                    cum += t;
-                }
-                sh.bcast[0] = (uint32_t)sel;
-                sh.bcast[1] = (uint32_t)cum;
-            }
-            __syncthreads();
-            const int sel = (int)sh.bcast[0];
-            const int64_t cum_slices = (int64_t)sh.bcast[1];
-            // copy that slice reversed (top bin first) and scan it
-            for (int j = tid; j < W; j += NT)
-                sh.rev[j] = cluster.map_shared_rank(sh.red, sel)[W - 1 - j];
-            __syncthreads();
-            const uint32_t c = (tid < W) ? sh.rev[tid] : 0u;
-            uint32_t tot;
-            const uint32_t ex = block_excl_scan(c, sh.warp_tmp, tot);
-            const int64_t before = cum_slices + (int64_t)ex;
-            if (tid < W && before < need && before + (int64_t)c >= need) {
-                sh.bcast[2] = (uint32_t)(sel * W + (W - 1 - tid));
-                sh.bcast[3] = (uint32_t)ex + (uint32_t)cum_slices;
-            }
-            __syncthreads();
-            const uint32_t bin = sh.bcast[2];
-            need -= (int64_t)sh.bcast[3];
-            prefix |= bin << shift;
-            pmask |= (uint32_t)(bins - 1) << shift;
-            // my own keys above the chosen bin (and, at the last level, equal to it)
-            uint32_t mine = 0;
-            for (int j = (int)bin + 1 + tid; j < bins; j += NT)
-                mine += sh.hist[j];
-            my_above += block_sum(mine, sh.warp_tmp);
-            if (level == 2)
-                my_ties = sh.hist[bin];
-            cluster.sync();   // others are done reading my hist / red / slice_total
-        }
-        vk = prefix;
-        r_ties = need;
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = lo + u * NT + threadIdx.x;
+        kk[u] = i < hi ? __ldcg(vb + i) : 0u;
     }
-
-    // ---- counts per CTA --------------------------------------------------
-    if (mode == 1)
-        my_above = (uint32_t)(my_hi - my_lo);
-    if (tid == 0) {
-        sh.cnt[0] = my_above;
-        sh.cnt[1] = my_ties;
-    }
-    cluster.sync();
-    if (tid == 0) {
-        int64_t tie_before = 0, sel_before = 0, tb = 0;
-        for (int q = 0; q < rank; ++q) {
-            const uint32_t *cq = cluster.map_shared_rank(sh.cnt, q);
-            const int64_t ca = cq[0], ct = cq[1];
-            const int64_t take = max((int64_t)0, min(r_ties - tb, ct));
-            sel_before += ca + take;
-            tb += ct;
-        }
-        tie_before = tb;
-        sh.bcast[0] = (uint32_t)tie_before;
-        sh.bcast[1] = (uint32_t)sel_before;
-    }
-    cluster.sync();   // every remote read of cnt is done
-    const int64_t tie_before = (int64_t)sh.bcast[0];
-    const int64_t sel_before = (int64_t)sh.bcast[1];
-
-    // ---- ordered compaction of my range -----------------------------------
-    if (mode != 2) {
-        int64_t run_ties = 0, run_sel = 0;
-        for (int64_t base = my_lo; base < my_hi; base += NT) {
-            const int64_t i = base + tid;
-            bool is_tie = false, flag = false;
-            if (i < my_hi) {
-                if (mode == 1) {
-                    flag = true;
-                } else {
-                    const uint32_t key = __ldcg(vb + i);
-                    flag = key > vk;
-                    is_tie = key == vk;
-                }
-            }
-            if (mode == 0) {
-                uint32_t tot;
-                const uint32_t ex = block_excl_scan((uint32_t)is_tie, sh.warp_tmp, tot);
-                if (is_tie && tie_before + run_ties + (int64_t)ex < r_ties)
-                    flag = true;
-                run_ties += (int64_t)tot;
-            }
-            uint32_t tot2;
-            const uint32_t pos = block_excl_scan((uint32_t)flag, sh.warp_tmp, tot2);
-            const int64_t at = s_end + sel_before + run_sel + (int64_t)pos;
-            if (flag && at < s_end + keff)      // never past the top-k part of the row
-                idrow[at] = (int32_t)i;
-            run_sel += (int64_t)tot2;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = lo + u * NT + threadIdx.x;
+        const uint32_t bin = i < hi ? (kk[u] >> 20) : 0xffffffffu;
+        // one atomic for the warp's most common bin, one per lane for the others
+        const uint32_t act = __ballot_sync(0xffffffffu, bin != 0xffffffffu);
+        if (act) {
+            const int leader = __ffs(act) - 1;
+            const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+            const uint32_t same = __ballot_sync(0xffffffffu, bin == lb);
+            if (lane == leader)
+                atomicAdd(&h[lb], (uint32_t)__popc(same));
+            else if (bin != 0xffffffffu && bin != lb)
+                atomicAdd(&h[bin], 1u);
         }
     }
+    __syncthreads();
+    uint32_t *gh = a.hist + (size_t)b * 4096;
+    for (int i = threadIdx.x; i < 4096; i += NT)
+        if (h[i] != 0u)
+            atomicAdd(&gh[i], h[i]);
+}
 
-    // ---- windows, count and padding (CTA 0) --------------------------------
-    if (rank == 0) {
-        const int64_t m = s_end + keff + (n - l0);
-        for (int64_t i = tid; i < s_end; i += NT)
+// ---------------------------------------------------------------------------
+// S2: bin b1 of the k-th largest vote; count above it, list the keys in it
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(NT)
+sel_collect(const SelArgs a)
+{
+    __shared__ uint32_t h[4096];
+    __shared__ uint32_t tmp[kWarps + 1];
+    __shared__ uint32_t bc[2];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.y, r = blockIdx.x;
+    if (a.reuse != nullptr && a.reuse[b] != 0)
+        return;
+    const Window w = window_of(a, b);
+    const int64_t lo = w.s_end + (int64_t)r * kTPC;
+    if (w.keff == 0 || w.keff == w.nc || lo >= w.l0)
+        return;
+    const int64_t hi = min(lo + kTPC, w.l0);
+    const uint32_t *vb = a.votes + w.off;
+    uint32_t kk[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = lo + u * NT + threadIdx.x;
+        kk[u] = i < hi ? __ldcg(vb + i) : 0u;
+    }
+    load_hist(h, a.hist + (size_t)b * 4096);
+    __syncthreads();
+    uint32_t b1, above_b1;
+    bin_from_top(h, 4096, w.keff, tmp, bc, b1, above_b1);
+
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t mine_above = 0;
+    uint2 *cl = a.cand + w.off;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = lo + u * NT + threadIdx.x;
+        const bool valid = i < hi;
+        const uint32_t bin = kk[u] >> 20;
+        mine_above += (valid && bin > b1) ? 1u : 0u;
+        const bool in = valid && bin == b1;
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        if (bal) {
+            const int leader = __ffs(bal) - 1;
+            uint32_t base = 0;
+            if (lane == leader)
+                base = atomicAdd(&a.cand_n[b], (uint32_t)__popc(bal));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (in)
+                cl[base + __popc(bal & lt)] = make_uint2(kk[u], (uint32_t)i);
+        }
+    }
+    uint32_t tot;
+    block_excl_scan(mine_above, tmp, tot);
+    if (threadIdx.x == 0)
+        a.above[(size_t)b * a.rps + r] = tot;
+}
+
+// ---------------------------------------------------------------------------
+// S3: exact threshold among the b1 candidates; per-range offsets
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(NT)
+sel_resolve(const SelArgs a)
+{
+    __shared__ uint32_t h[4096];
+    __shared__ uint32_t tmp[kWarps + 1];
+    __shared__ uint32_t bc[2];
+    __shared__ unsigned long long keys[kResolveSmem];
+    __shared__ uint32_t rcnt[kMaxSelectRanges];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.x;
+    if (a.reuse != nullptr && a.reuse[b] != 0)
+        return;
+    const Window w = window_of(a, b);
+    const int nranges = (int)((w.nc + kTPC - 1) / kTPC);
+    if (w.keff == 0 || w.keff == w.nc) {
+        if (threadIdx.x == 0) {
+            a.mode[b] = w.keff == 0 ? 0 : 2;
+            a.thr[b] = 0ull;
+        }
+        // every candidate selected: range r starts at r * kTPC
+        for (int r = threadIdx.x; r < nranges; r += NT)
+            a.range_off[(size_t)b * a.rps + r] = w.keff == 0 ? 0u : (uint32_t)((int64_t)r * kTPC);
+        return;
+    }
+    uint32_t *gh = a.hist + (size_t)b * 4096;
+    const uint32_t m = __ldcg(&a.cand_n[b]);
+    load_hist(h, gh);
+    __syncthreads();
+    uint32_t b1, above_b1;
+    bin_from_top(h, 4096, w.keff, tmp, bc, b1, above_b1);
+    for (int i = threadIdx.x; i < 4096; i += NT)
+        gh[i] = 0u;                                  // ready for the next call
+    const uint2 *cl = a.cand + w.off;
+    const bool in_smem = m <= (uint32_t)kResolveSmem;
+    if (in_smem) {
+        constexpr int kBatch = 10;                   // kResolveSmem / NT
+        for (uint32_t j0 = threadIdx.x; j0 < m; j0 += kBatch * NT) {
+            uint2 c[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                c[u] = j0 + u * NT < m ? __ldcg(cl + j0 + u * NT) : make_uint2(0u, 0u);
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (j0 + u * NT < m)
+                    keys[j0 + u * NT] = make_key(c[u].x, c[u].y);
+        }
+    }
+    __syncthreads();
+    auto key_at = [&](uint32_t j) -> unsigned long long {
+        if (in_smem)
+            return keys[j];
+        const uint2 c = __ldcg(cl + j);
+        return make_key(c.x, c.y);
+    };
+
+    // radix select of the need-th largest key among the m candidates: they
+    // share the top 12 bits (b1); 8-bit digits over bits 51..4, then 3..0
+    int64_t need = (int64_t)w.keff - above_b1;
+    unsigned long long prefix = (unsigned long long)b1 << 52;
+    unsigned long long pmask = 0xfffull << 52;
+    for (int shift = 44; shift >= -4; shift -= 8) {
+        const int sh = shift < 0 ? 0 : shift;
+        const int nb = shift < 0 ? 16 : 256;
+        h[threadIdx.x] = 0u;
+        __syncthreads();
+        for (uint32_t j = threadIdx.x; j < m; j += NT) {
+            const unsigned long long key = key_at(j);
+            if ((key & pmask) == prefix)
+                atomicAdd(&h[(uint32_t)(key >> sh) & (uint32_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        const int t = threadIdx.x;
+        const uint32_t c = t < nb ? h[nb - 1 - t] : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan(c, tmp, tot);
+        if (t < nb && (int64_t)ex < need && (int64_t)(ex + c) >= need) {
+            bc[0] = (uint32_t)(nb - 1 - t);
+            bc[1] = ex;
+        }
+        __syncthreads();
+        const uint32_t dig = bc[0];
+        need -= bc[1];
+        __syncthreads();
+        prefix |= (unsigned long long)dig << sh;
+        pmask |= (unsigned long long)(nb - 1) << sh;
+    }
+    const unsigned long long T = prefix;   // the k-th largest key
+
+    // per-range counts of selected b1 candidates, then range offsets
+    for (int r = threadIdx.x; r < nranges; r += NT)
+        rcnt[r] = 0u;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < m; j += NT) {
+        const unsigned long long key = key_at(j);
+        if (key >= T) {
+            const uint32_t id = 0xffffffffu - (uint32_t)(key & 0xffffffffull);
+            atomicAdd(&rcnt[(id - (uint32_t)w.s_end) / kTPC], 1u);
+        }
+    }
+    __syncthreads();
+    uint32_t run = 0;
+    for (int r0 = 0; r0 < nranges; r0 += NT) {
+        const int r = r0 + threadIdx.x;
+        const uint32_t c = r < nranges ? __ldcg(&a.above[(size_t)b * a.rps + r]) + rcnt[r] : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan(c, tmp, tot);
+        if (r < nranges)
+            a.range_off[(size_t)b * a.rps + r] = run + ex;
+        run += tot;
+    }
+    if (threadIdx.x == 0) {
+        a.thr[b] = T;
+        a.mode[b] = 1;
+        a.cand_n[b] = 0u;                            // ready for the next call
+    }
+}
+
+// ---------------------------------------------------------------------------
+// S4: ordered write of the selected ids; windows, count and padding
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(NT)
+sel_write(const SelArgs a)
+{
+    __shared__ uint32_t tmp[kWarps + 1];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.y, r = blockIdx.x;
+    if (a.reuse != nullptr && a.reuse[b] != 0)
+        return;   // the previous ids stay
+    const Window w = window_of(a, b);
+    int32_t *idrow = a.ids + (int64_t)b * a.cap;
+    if (r == 0) {
+        const int64_t mcount = w.s_end + w.keff + (w.n - w.l0);
+        for (int64_t i = threadIdx.x; i < w.s_end; i += NT)
             idrow[i] = (int32_t)i;
-        for (int64_t j = tid; j < n - l0; j += NT)
-            idrow[s_end + keff + j] = (int32_t)(l0 + j);
-        for (int64_t j = m + tid; j < a.cap; j += NT)
+        for (int64_t j = threadIdx.x; j < w.n - w.l0; j += NT)
+            idrow[w.s_end + w.keff + j] = (int32_t)(w.l0 + j);
+        for (int64_t j = mcount + threadIdx.x; j < a.cap; j += NT)
             idrow[j] = -1;
-        if (tid == 0)
-            a.count[b] = (int32_t)m;
+        if (threadIdx.x == 0)
+            a.count[b] = (int32_t)mcount;
+    }
+    const int64_t lo = w.s_end + (int64_t)r * kTPC;
+    if (lo >= w.l0)
+        return;
+    const int md = __ldcg(&a.mode[b]);
+    if (md == 0)
+        return;
+    const int64_t hi = min(lo + kTPC, w.l0);
+    const unsigned long long T = __ldcg(&a.thr[b]);
+    const uint32_t base = __ldcg(&a.range_off[(size_t)b * a.rps + r]);
+    // each thread takes kPer consecutive candidates, so one block scan orders them
+    const int64_t t0 = lo + (int64_t)threadIdx.x * kPer;
+    const uint32_t *vb = a.votes + w.off;
+    bool f[kPer];
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = t0 + u;
+        f[u] = false;
+        if (i < hi)
+            f[u] = md == 2 || make_key(__ldcg(vb + i), i) >= T;
+        cnt += f[u] ? 1u : 0u;
+    }
+    uint32_t tot;
+    uint32_t pos = block_excl_scan(cnt, tmp, tot);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        if (f[u]) {
+            const int64_t at = w.s_end + (int64_t)base + pos;
+            if (at < w.s_end + w.keff)   // never past the top-k part of the row
+                idrow[at] = (int32_t)(t0 + u);
+            ++pos;
+        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,
-                          int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, cudaStream_t st)
+                          int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, uint8_t *ws,
+                          cudaStream_t st)
 {
-    SelectArgs a;
+    SelArgs a;
     a.votes = reinterpret_cast<const uint32_t *>(votes);
     a.seq_off = seq_off;
     a.reuse = reuse;
     a.ids = ids;
     a.count = count;
+    a.hist = reinterpret_cast<uint32_t *>(ws + p.off_sel_hist);
+    a.cand = reinterpret_cast<uint2 *>(ws + p.off_sel_cand);
+    a.cand_n = reinterpret_cast<uint32_t *>(ws + p.off_sel_cand_n);
+    a.above = reinterpret_cast<uint32_t *>(ws + p.off_sel_above);
+    a.range_off = reinterpret_cast<uint32_t *>(ws + p.off_sel_range_off);
+    a.thr = reinterpret_cast<unsigned long long *>(ws + p.off_sel_thr);
+    a.mode = reinterpret_cast<int32_t *>(ws + p.off_sel_mode);
     a.k = k;
     a.n_sink = n_sink;
     a.n_local = n_local;
     a.cap = k + n_sink + n_local;
-    select_kernel<<<p.B * CS, NT, 0, st>>>(a);
-    return cudaGetLastError();
+    a.B = p.B;
+    a.rps = p.sel_ranges;
+    const dim3 grid((unsigned)p.sel_ranges, (unsigned)p.B);
+    cudaError_t e = launch_ex(sel_hist, grid, dim3(NT), 0, st, 1, a);
+    if (e == cudaSuccess)
+        e = launch_ex(sel_collect, grid, dim3(NT), 0, st, 1, a);
+    if (e == cudaSuccess)
+        e = launch_ex(sel_resolve, dim3((unsigned)p.B), dim3(NT), 0, st, 1, a);
+    if (e == cudaSuccess)
+        e = launch_ex(sel_write, grid, dim3(NT), 0, st, 1, a);
+    return e;
 }
 
 }  // namespace ts

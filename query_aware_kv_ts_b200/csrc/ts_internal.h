@@ -17,12 +17,49 @@ constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
 constexpr int kScoreStages = 6;
 constexpr int kStageBytesTarget = 32768;
 constexpr int kVoteThreads = 256;
-constexpr int kVoteTokensPerBlock = 1024;
-constexpr int kSelectClusterSize = 8;
-constexpr int kSelectThreads = 1024;
-constexpr int kAttnThreads = 128;
+constexpr int kVoteTokensPerBlock = kVoteThreads;   // one token per thread
+constexpr int kSelectThreads = 256;
+constexpr int kSelectTokensPerCta = 2048;     // candidates per selection range
+constexpr int kMaxSelectRanges = 2048;        // ranges per sequence: n <= 4M candidates
+constexpr int kAttnThreads = 256;
+constexpr int kAttnRows = 128;        // selected rows per attention CTA (one split)
+constexpr int kMaxCapacity = 128 * kAttnRows;   // k + sink + local
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launch with programmatic stream serialization (the kernel's prologue may
+// overlap the previous kernel in the stream; see pdl_wait) and, when
+// cluster > 1, a thread-block cluster of that many CTAs along x.
+// Programmatic dependent launch is on unless the environment sets TS_NO_PDL=1.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
+                      Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Everything derived from the cache shape that the kernels and the workspace
 // layout need.  Built identically by every entry point.
@@ -35,17 +72,17 @@ struct Plan {
     // score pass A
     int tile_tokens;         // T: tokens per pipeline stage
     int stage_bytes;
-    int64_t chunk_tokens;    // tokens per work chunk (multiple of T)
-    int64_t max_chunks;      // sum_b ceil(n_b / chunk_tokens)
-    int score_grid;
-    // vote pass B
-    int64_t max_vote_blocks; // sum_b ceil(n_b / kVoteTokensPerBlock)
+    int64_t max_chunks;      // sum_b ceil(n_b / T)
+    int score_grid;          // <= 256
+    int64_t ld_logits;       // logits row stride: n_total rounded up to 4
+    // selection
+    int sel_ranges;          // ranges of kSelectTokensPerCta candidates per sequence (grid x)
     // attention
     int capacity;            // ids row length (k + sink + local)
     int attn_splits;
     // workspace layout (byte offsets)
-    size_t off_ctrl, off_score_tickets, off_attn_tickets, off_L, off_partials, off_logits,
-        off_attn_part, total_bytes;
+    size_t off_ctrl, off_chunk_table, off_L, off_partials, off_logits, off_sel_hist, off_sel_cand,
+        off_sel_cand_n, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part, total_bytes;
 };
 
 // Fill `p` from the cache description (capacity < 0: attention part not
@@ -65,7 +102,8 @@ cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *re
                         cudaStream_t st);
 
 cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,
-                          int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, cudaStream_t st);
+                          int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, uint8_t *ws,
+                          cudaStream_t st);
 
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
                         const int32_t *count, float *out, uint8_t *ws, cudaStream_t st);

@@ -4,12 +4,21 @@
 // reading the logits written by pass A (L2-resident for moderate n) and the
 // float64 log-normalisers L.
 //
-// Precision: s - L is formed exactly as an unevaluated float pair (two-sum of
-// s and the high part of L, minus L's low part), and exp(hi + lo) is taken as
-// expf(hi) * (1 + lo) (one fma) with |lo| < 2^-18, so the only rounding left is that of
-// expf itself (a few 1e-8 relative).  A plain fp32 subtraction would lose up
-// to half an ulp of |s - L| (~1e-6 for |s - L| ~ 20), which is larger than the
-// vote band inside which the selection is allowed to differ.
+// Precision: s - L is formed exactly as t + d (two-sum of s and the float
+// high part of L, minus L's low part).  The base-2 exponent u = (t + d) log2(e)
+// is carried as an unevaluated pair too: u_hi = fl(t * log2e_hi) and
+//   u_lo = fma(t, log2e_hi, -u_hi) + t * log2e_lo + d * log2e_hi
+// (the product error recovered with one fma, as in Dekker's exact product,
+// with log2(e) split Cody-Waite style into a float head and tail), so that
+// exp(s - L) = 2^u_hi * (1 + u_lo ln 2) up to second order in |u_lo| < 2^-17.
+// The only rounding left is the hardware 2^x (a few 1e-8 relative) and the
+// sum over heads.  A plain fp32 s - L would lose up to half an ulp of |s - L|
+// (~1e-6 relative for |s - L| ~ 20), the width of the selection band.
+//
+// Work split: grid (groups / threads, B).  Long sequences: a thread takes 4
+// consecutive tokens aligned to 4 in the logits rows (row stride padded to 4),
+// so each head's logits arrive as one 16-byte load, 8 heads at a time; short
+// sequences: one token per thread, 32 heads loaded at a time, 64-thread blocks.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -17,7 +26,7 @@ namespace ts {
 namespace {
 
 struct VoteArgs {
-    const float *logits;   // [Hq][ld]
+    const float *logits;   // [Hq][ld], ld % 4 == 0
     int64_t ld;
     const double *L;       // [B][Hq]
     const int64_t *seq_off;
@@ -27,85 +36,89 @@ struct VoteArgs {
 };
 
 constexpr int kMaxHeadsVote = 256;
+constexpr int kHeadBatch = 8;
+constexpr float kLog2eHi = 1.44269502162933349609375f;   // float nearest log2(e)
+constexpr float kLog2eLo = 1.925963033500011e-08f;       // log2(e) - kLog2eHi
+constexpr float kLn2 = 0.693147180559945309f;
 
+__device__ __forceinline__ float exp_exact_arg(float s, float Lhi, float Llo)
+{
+    const float t = s - Lhi;                       // two-sum: t + e == s - Lhi
+    const float bp = t - s;
+    const float e = (s - (t - bp)) + (-Lhi - bp);
+    const float d = e - Llo;                       // s - L == t + d
+    const float u = t * kLog2eHi;
+    const float u_lo = fmaf(t, kLog2eHi, -u) + fmaf(t, kLog2eLo, d * kLog2eHi);
+    const float p = exp2f(u);
+    return fmaf(p, u_lo * kLn2, p);
+}
+
+template <int TPT>
 __global__ void __launch_bounds__(kVoteThreads)
 vote_pass_b(const VoteArgs a)
 {
-    __shared__ int64_t s_off[kMaxBatch + 1];
-    __shared__ int32_t s_start[kMaxBatch + 1];
     __shared__ float s_hi[kMaxHeadsVote], s_lo[kMaxHeadsVote];
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int B = a.B;
-    for (int b = tid; b <= B; b += blockDim.x)
-        s_off[b] = a.seq_off[b];
-    __syncthreads();
-    for (int b = tid; b < B; b += blockDim.x) {
-        const int64_t n = s_off[b + 1] - s_off[b];
-        const bool active = (a.reuse == nullptr) || (a.reuse[b] == 0);
-        s_start[b + 1] = active ? (int32_t)((n + kVoteTokensPerBlock - 1) / kVoteTokensPerBlock) : 0;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int32_t run = 0;
-        for (int base = 0; base < B; base += 32) {
-            const int b = base + lane;
-            int32_t x = (b < B) ? s_start[b + 1] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o)
-                    x += y;
-            }
-            if (b < B)
-                s_start[b + 1] = run + x;
-            run += __shfl_sync(0xffffffffu, x, 31);
-        }
-        if (lane == 0)
-            s_start[0] = 0;
-    }
-    __syncthreads();
-    const int32_t v = blockIdx.x;
-    if (v >= s_start[B])
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x;
+    if (a.reuse != nullptr && a.reuse[b] != 0)
         return;
-    const int b = upper_seq(s_start, B, v);
-    for (int h = tid; h < a.Hq; h += blockDim.x) {
+    const int64_t off = a.seq_off[b];
+    const int64_t end = a.seq_off[b + 1];
+    const int64_t base = off & ~int64_t(TPT - 1);                  // first aligned group of the sequence
+    const int nt = blockDim.x;
+    const int64_t i0 = base + ((int64_t)blockIdx.x * nt + tid) * TPT;
+    if (base + (int64_t)blockIdx.x * nt * TPT >= end)
+        return;   // the whole block is past this sequence
+    for (int h = tid; h < a.Hq; h += nt) {
         const double L = a.L[(int64_t)b * a.Hq + h];
         const float hi = (float)L;
         s_hi[h] = hi;
         s_lo[h] = (float)(L - (double)hi);
     }
     __syncthreads();
-
-    const int64_t base = s_off[b] + (int64_t)(v - s_start[b]) * kVoteTokensPerBlock;
-    const int64_t end = min(base + kVoteTokensPerBlock, s_off[b + 1]);
-    constexpr int kPer = kVoteTokensPerBlock / kVoteThreads;
-    float acc[kPer];
+    if (i0 >= end)
+        return;
+    float acc[TPT];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j)
+    for (int j = 0; j < TPT; ++j)
         acc[j] = 0.0f;
-    for (int h = 0; h < a.Hq; ++h) {
-        const float Lhi = s_hi[h], Llo = s_lo[h];
-        const float *row = a.logits + (int64_t)h * a.ld;
+    if constexpr (TPT == 4) {
+        for (int h0 = 0; h0 < a.Hq; h0 += kHeadBatch) {
+            float4 sv[kHeadBatch];
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int64_t i = base + tid + j * kVoteThreads;
-            if (i < end) {
-                const float s = __ldcg(row + i);
-                // two-sum: t + e == s - Lhi exactly
-                const float t = s - Lhi;
-                const float bp = t - s;
-                const float e = (s - (t - bp)) + (-Lhi - bp);
-                const float lo = e - Llo;
-                const float et = expf(t);
-                acc[j] += fmaf(et, lo, et);
+            for (int u = 0; u < kHeadBatch; ++u)
+                if (h0 + u < a.Hq)
+                    sv[u] = __ldcg(reinterpret_cast<const float4 *>(a.logits + (int64_t)(h0 + u) * a.ld + i0));
+#pragma unroll
+            for (int u = 0; u < kHeadBatch; ++u) {
+                if (h0 + u < a.Hq) {
+                    const float Lhi = s_hi[h0 + u], Llo = s_lo[h0 + u];
+                    acc[0] += exp_exact_arg(sv[u].x, Lhi, Llo);
+                    acc[1] += exp_exact_arg(sv[u].y, Lhi, Llo);
+                    acc[2] += exp_exact_arg(sv[u].z, Lhi, Llo);
+                    acc[3] += exp_exact_arg(sv[u].w, Lhi, Llo);
+                }
             }
+        }
+    } else {
+        for (int h0 = 0; h0 < a.Hq; h0 += 4 * kHeadBatch) {
+            float sv[4 * kHeadBatch];
+#pragma unroll
+            for (int u = 0; u < 4 * kHeadBatch; ++u)
+                if (h0 + u < a.Hq)
+                    sv[u] = __ldcg(a.logits + (int64_t)(h0 + u) * a.ld + i0);
+#pragma unroll
+            for (int u = 0; u < 4 * kHeadBatch; ++u)
+                if (h0 + u < a.Hq)
+                    acc[0] += exp_exact_arg(sv[u], s_hi[h0 + u], s_lo[h0 + u]);
         }
     }
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int64_t i = base + tid + j * kVoteThreads;
-        if (i < end)
+    for (int j = 0; j < TPT; ++j) {
+        const int64_t i = i0 + j;
+        if (i >= off && i < end)
             a.votes[i] = acc[j];
     }
 }
@@ -115,19 +128,28 @@ vote_pass_b(const VoteArgs a)
 cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
                         cudaStream_t st)
 {
-    if (p.max_vote_blocks <= 0)
+    if (p.n_max <= 0)
         return cudaSuccess;
     VoteArgs a;
     a.logits = reinterpret_cast<const float *>(ws + p.off_logits);
-    a.ld = p.n_total;
+    a.ld = p.ld_logits;
     a.L = reinterpret_cast<const double *>(ws + p.off_L);
     a.seq_off = seq_off;
     a.reuse = reuse;
     a.votes = votes;
     a.B = p.B;
     a.Hq = p.Hq;
-    vote_pass_b<<<(unsigned)p.max_vote_blocks, kVoteThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    // quads of a sequence: its tokens plus up to 3 before the first aligned index
+    // long sequences: 4 tokens per thread (16-byte loads, 256 threads);
+    // short ones: 1 token per thread in 64-thread blocks, so that enough warps
+    // share the latency-bound pass
+    if (p.n_total > 262144) {
+        const int64_t groups = (p.n_max + 3) / 4 + 1;
+        const unsigned gx = (unsigned)((groups + kVoteThreads - 1) / kVoteThreads);
+        return launch_ex(vote_pass_b<4>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
+    }
+    const unsigned gx = (unsigned)((p.n_max + 63) / 64);
+    return launch_ex(vote_pass_b<1>, dim3(gx, (unsigned)p.B), dim3(64), 0, st, 1, a);
 }
 
 }  // namespace ts
