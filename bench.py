@@ -43,7 +43,10 @@ import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
-LAUNCHES_PER_LAYER_STEP = 6     # selcache, score pass A, normaliser merge, score pass B, select, attention
+# ts_decode_step: selection cache 1; score pass A, normaliser merge, pass B
+# (with the selection histogram) 3; selection collect, resolve, write 3;
+# attention split, merge 2
+LAUNCHES_PER_LAYER_STEP = 9
 
 
 def parse_args(argv=None):
@@ -239,15 +242,14 @@ class Workload:
         m = np.minimum(self.lengths, c.k + c.n_sink + c.n_local)
         return self.k_bytes + int(m.sum()) * c.h_kv * c.head_dim * 2 * 2
 
-    # one layer-step through the public C ABI
+    # one layer-step through the public C ABI: the one-call decode step
+    # (selection cache, score, select, sparse attention)
     def layer_step(self, layer: int, i: int):
         ts, b = self.ts, self.bufs[layer]
         kv = self.kvs[layer][i % self.rotate]
         q = self.q[layer][i % self.T]
-        ts.ts_selcache(q, b.q_prev, b.reuse, False, self.theta, b.cos)
-        ts.ts_score(kv, q, b.reuse, b.votes, b.ws)
-        ts.ts_select(kv, b.votes, b.k, b.n_sink, b.n_local, b.reuse, b.ids, b.count, b.ws)
-        ts.ts_sparse_attn(kv, q, b.ids, b.count, b.out, b.ws)
+        ts.ts_decode_step(kv, q, b.q_prev, b.reuse, False, self.theta, b.k, b.n_sink, b.n_local, b.votes, b.ids,
+                          b.count, b.out, b.ws, b.cos)
 
     def step(self, i: int):
         for layer in range(self.cfg.layers):

@@ -209,6 +209,23 @@ TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, cons
                                           void *stream);
 
 /*
+ * One whole decode step of one layer: ts_selcache, ts_score, ts_select and
+ * ts_sparse_attn in that order on `stream`, with the same arguments and the
+ * same results as the four calls (selection capacity k + n_sink + n_local, the
+ * ids row length).  Fewer kernels run: the vote pass also builds the
+ * selection's first-level vote histogram, which ts_select otherwise builds in
+ * a kernel of its own.  Every argument is checked before the first launch.
+ *   reuse      device int32 [batch], required: written by the selection cache
+ *              and read by every later phase (sequences that reuse keep their
+ *              previous ids and count; their votes are left as they were)
+ *   q          16-byte aligned; out 16-byte aligned; ws as ts_workspace_bytes
+ */
+TS_API ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32_t *reuse,
+                                  double *cos_out, int32_t first_step, double threshold, int32_t k,
+                                  int32_t n_sink, int32_t n_local, float *votes, int32_t *ids,
+                                  int32_t *count, float *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Read and clear the device status word of a workspace (synchronises the
  * stream).  Returns TS_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave
  * up since the last read, TS_OK otherwise.  *site_out (may be NULL) receives

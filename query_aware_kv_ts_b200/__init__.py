@@ -65,6 +65,8 @@ _SIGS = {
     "ts_select": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "ts_sparse_attn": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
     "ts_sparse_attn_noalloc": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P]),
+    "ts_decode_step": (ctypes.c_int, [_KV, _P, _P, _P, _P, _I32, _F64, _I32, _I32, _I32, _P, _P, _P, _P, _P,
+                                      _SZ, _P]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -187,6 +189,16 @@ def ts_sparse_attn_noalloc(kv: KVCache, q, ids, count, out, stream=None):
                                        _stream(stream)))
 
 
+def ts_decode_step(kv: KVCache, q, q_prev, reuse, first_step: bool, threshold: float, k: int, n_sink: int,
+                   n_local: int, votes, ids, count, out, ws, cos_out=None, stream=None):
+    """ts_selcache, ts_score, ts_select and ts_sparse_attn of one layer in one
+    call (fewer kernels, same results)."""
+    _check(_lib.ts_decode_step(kv.ref(), _ptr(q), _ptr(q_prev), _ptr(reuse), _ptr(cos_out),
+                               int(bool(first_step)), float(threshold), k, n_sink, n_local, _ptr(votes),
+                               _ptr(ids), _ptr(count), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)))
+
+
 def ts_get_device_status(ws, stream=None):
     """Returns (status, site); status is TS_OK or TS_ERR_DEVICE_TIMEOUT."""
     site = ctypes.c_uint32(0)
@@ -234,9 +246,15 @@ class StepBuffers:
         self.q_prev = torch.zeros((kv.batch, kv.h_q, kv.head_dim), dtype=torch.bfloat16, device=dev)
 
 
-def decode_step(kv: KVCache, q, buf: StepBuffers, *, theta=None, first_step=True, stream=None):
+def decode_step(kv: KVCache, q, buf: StepBuffers, *, theta=None, first_step=True, stream=None, fused=False):
     """One layer-step through the four entry points, in stream order:
-    ts_selcache (when theta is given) -> ts_score -> ts_select -> ts_sparse_attn."""
+    ts_selcache (when theta is given) -> ts_score -> ts_select -> ts_sparse_attn;
+    fused=True makes the same step one ts_decode_step call (a theta that the
+    cosine never reaches when theta is None)."""
+    if fused:
+        ts_decode_step(kv, q, buf.q_prev, buf.reuse, first_step, 2.0 if theta is None else theta, buf.k,
+                       buf.n_sink, buf.n_local, buf.votes, buf.ids, buf.count, buf.out, buf.ws, buf.cos, stream)
+        return buf.out
     reuse = None
     if theta is not None:
         ts_selcache(q, buf.q_prev, buf.reuse, first_step, theta, buf.cos, stream)

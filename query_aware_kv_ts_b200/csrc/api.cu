@@ -186,25 +186,23 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     // every attention CTA takes at most kAttnRows selected rows
     p->attn_splits = capacity > 0 ? (capacity + kAttnRows - 1) / kAttnRows : 0;
 
+    // small per-call tables first (they share a few pages), then the arrays
+    // that grow with the cache, then the attention partials
     size_t o = 0;
     p->off_ctrl = o;
     o += 256;
     // everything above is the control block that ts_workspace_init zeroes
+    const size_t nt1 = (size_t)(n_total > 0 ? n_total : 1);
     p->off_chunk_table = o;
     o = align_up(o + sizeof(int32_t) * (p->B + 1), 256);
     p->off_L = o;
     o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
     p->off_partials = o;
-    o = align_up(o + sizeof(float) * 2 * (size_t)(chunks > 0 ? chunks : 1) * p->Hq, 256);
-    p->off_logits = o;
-    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(p->ld_logits > 0 ? p->ld_logits : 4), 256);
-    const size_t nt1 = (size_t)(n_total > 0 ? n_total : 1);
-    p->off_sel_hist = o;
-    o = align_up(o + sizeof(uint32_t) * 4096 * (size_t)p->B, 256);
-    p->off_sel_cand = o;
-    o = align_up(o + 8 * nt1, 256);
+    o = align_up(o + sizeof(float) * 2 * (size_t)(p->score_grid + p->B) * p->Hq, 256);
     p->off_sel_cand_n = o;
     o = align_up(o + sizeof(uint32_t) * (size_t)p->B, 256);
+    p->off_sel_bin = o;
+    o = align_up(o + sizeof(uint32_t) * 2 * (size_t)p->B, 256);
     p->off_sel_above = o;
     o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
     p->off_sel_range_off = o;
@@ -213,6 +211,14 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     o = align_up(o + sizeof(uint64_t) * (size_t)p->B, 256);
     p->off_sel_mode = o;
     o = align_up(o + sizeof(int32_t) * (size_t)p->B, 256);
+    p->off_sel_hist = o;
+    o = align_up(o + sizeof(uint32_t) * 4096 * (size_t)p->B, 256);
+    p->off_logits = o;
+    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(p->ld_logits > 0 ? p->ld_logits : 4), 256);
+    p->off_sel_cand = o;
+    o = align_up(o + 8 * nt1, 256);
+    // last: the only part whose size depends on the selection capacity, so
+    // every offset above is the same for every entry point
     p->off_attn_part = o;
     if (capacity > 0)
         o = align_up(o + sizeof(float) * (size_t)p->B * p->Hkv * p->attn_splits * p->G * (D + 4), 256);
@@ -449,6 +455,65 @@ ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32
         return TS_ERR_INVALID_ARG;
     }
     return launch_attn_noalloc(p, kv, q, ids, count, out, static_cast<cudaStream_t>(stream));
+}
+
+ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32_t *reuse, double *cos_out,
+                           int32_t first_step, double threshold, int32_t k, int32_t n_sink, int32_t n_local,
+                           float *votes, int32_t *ids, int32_t *count, float *out, void *ws, size_t ws_bytes,
+                           void *stream)
+{
+    // every argument is checked before the first launch
+    if (k < 0 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > (int64_t(1) << 30) ||
+        k + n_sink + n_local < 1) {
+        set_error("k, n_sink, n_local must be non-negative with a sum in [1, 2^30)");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = make_plan(kv, k + n_sink + n_local, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || q_prev == nullptr || reuse == nullptr || votes == nullptr || ids == nullptr ||
+        count == nullptr || out == nullptr) {
+        set_error("q, q_prev, reuse, votes, ids, count and out are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u) ||
+        (reinterpret_cast<uintptr_t>(q_prev) & 3u)) {
+        set_error("q and out must be 16-byte aligned, q_prev 4-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (isnan(threshold)) {
+        set_error("threshold is NaN");
+        return TS_ERR_INVALID_ARG;
+    }
+    s = check_ws(p, ws, ws_bytes);
+    if (s != TS_OK)
+        return s;
+    CUtensorMap kmap;
+    if (p.n_total > 0) {
+        s = encode_kmap(p, kv, &kmap);
+        if (s != TS_OK)
+            return s;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    cudaError_t e = launch_selcache(q, q_prev, reuse, cos_out, first_step != 0, p.B, p.Hq * p.D, threshold, st);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: selection cache launch");
+    if (p.n_total > 0) {
+        e = launch_score(p, kmap, q, kv->seq_offsets_dev, reuse, w, st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ts_decode_step: score pass A launch");
+        const SelectWindow win = {k, n_sink, n_local};
+        e = launch_vote(p, kv->seq_offsets_dev, reuse, votes, w, st, &win);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ts_decode_step: score pass B launch");
+    }
+    e = launch_select(p, kv->seq_offsets_dev, votes, k, n_sink, n_local, reuse, ids, count, w, st, true);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: select launch");
+    e = launch_attn(p, kv, q, ids, count, out, w, st);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_decode_step: sparse attention launch");
 }
 
 ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream)

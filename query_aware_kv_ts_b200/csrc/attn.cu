@@ -15,9 +15,9 @@
 //     high part and a bf16 remainder (two products) so that the weights keep
 //     ~16 significant bits instead of bf16's 8;
 //  5. writes (max, sum, weighted V) per head as its partial.
-// attn_merge (one block per (b, g), launched right after) folds the splits:
-// a thread owns 4 output channels of one head and reads those channels and
-// the (max, sum) of every split, 16 splits at a time, with an online rescale.
+// attn_merge (one block per (b, query head), launched right after) folds the
+// splits: a thread owns 4 output channels and every NG-th split, loads all of
+// them at once, and the NG split groups are combined through shared memory.
 // Each selected K/V row is read from HBM once for all G heads of its group.
 #include <mutex>
 
@@ -84,8 +84,8 @@ attn_split(const AttnArgs a)
     const int lo = (int)((int64_t)a.cap * sp / a.splits);
     const int hi_cap = (int)((int64_t)a.cap * (sp + 1) / a.splits);
     const int32_t id_pref = (threadIdx.x < (unsigned)(hi_cap - lo))
-                                ? __ldg(a.ids + (int64_t)b * a.cap + lo + threadIdx.x) : -1;
-    int m_b = a.count[b];
+                                ? __ldcg(a.ids + (int64_t)b * a.cap + lo + threadIdx.x) : -1;
+    int m_b = __ldcg(a.count + b);
     m_b = max(0, min(m_b, a.cap));
     const int nrows = max(0, min(min(hi_cap, m_b) - lo, R));
     const int64_t off = a.seq_off[b];
@@ -258,66 +258,99 @@ attn_split(const AttnArgs a)
     }
 }
 
-// out[b, g*G + h, :] from the splits of (b, g).  Thread: 4 channels of one head.
+// out[b, h, :] for query head h = g*G + j from the splits of (b, g).  Thread
+// (sg, c): output channels 4c..4c+3 of every split s = sg (mod NG), all loaded
+// in one round trip (kMergeBatch splits per thread per trip); the NG groups'
+// (max, sum, weighted sums) are then combined through shared memory.
+constexpr int kMergeBatch = 8;
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_merge(const AttnArgs a)
 {
     constexpr int PS = D + 4;
-    constexpr int kBatch = 16;
+    constexpr int CQ = D / 4;                    // channel quads
+    constexpr int NG = kAttnThreads / CQ;        // split groups
+    __shared__ float4 s_acc[NG][CQ];
+    __shared__ float2 s_ml[NG][CQ];
     pdl_wait();
     pdl_launch_dependents();
-    const int g = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x, b = blockIdx.y;
     const int G = a.G;
+    const int g = h / G, j = h - g * G;
+    const int c = threadIdx.x % CQ, sg = threadIdx.x / CQ;
     const int64_t GS = (int64_t)G * PS;
-    const float *parts = a.part + ((int64_t)b * a.Hkv + g) * a.splits * GS;
-    for (int item = threadIdx.x; item < G * (D / 4); item += kAttnThreads) {
-        const int h = item / (D / 4), c = (item - h * (D / 4)) * 4;
-        float M = -INFINITY, L = 0.0f;
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        for (int q0 = 0; q0 < a.splits; q0 += kBatch) {
-            float4 v4[kBatch];
-            float2 ml[kBatch];
+    const float *parts = a.part + ((int64_t)b * a.Hkv + g) * a.splits * GS + (int64_t)j * PS;
+    float M = -INFINITY, L = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int s0 = sg; s0 < a.splits; s0 += kMergeBatch * NG) {
+        float4 v4[kMergeBatch];
+        float2 ml[kMergeBatch];
 #pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                if (q0 + i < a.splits) {
-                    const float *pq = parts + (int64_t)(q0 + i) * GS + h * PS;
-                    v4[i] = __ldcg(reinterpret_cast<const float4 *>(pq + c));
-                    ml[i] = __ldcg(reinterpret_cast<const float2 *>(pq + D));
-                } else {
-                    v4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    ml[i] = make_float2(-INFINITY, 0.0f);
-                }
+        for (int i = 0; i < kMergeBatch; ++i) {
+            const int sp = s0 + i * NG;
+            if (sp < a.splits) {
+                const float *pq = parts + (int64_t)sp * GS;
+                v4[i] = __ldcg(reinterpret_cast<const float4 *>(pq + 4 * c));
+                ml[i] = __ldcg(reinterpret_cast<const float2 *>(pq + D));
+            } else {
+                v4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                ml[i] = make_float2(-INFINITY, 0.0f);
             }
-            float Mb = M;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i)
-                Mb = fmaxf(Mb, ml[i].x);
-            if (Mb == -INFINITY)
-                continue;
-            const float r = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
-            L *= r;
-            acc.x *= r;
-            acc.y *= r;
-            acc.z *= r;
-            acc.w *= r;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                if (ml[i].x != -INFINITY) {
-                    const float w = exp2f(ml[i].x - Mb);
-                    L = fmaf(ml[i].y, w, L);
-                    acc.x = fmaf(w, v4[i].x, acc.x);
-                    acc.y = fmaf(w, v4[i].y, acc.y);
-                    acc.z = fmaf(w, v4[i].z, acc.z);
-                    acc.w = fmaf(w, v4[i].w, acc.w);
-                }
-            }
-            M = Mb;
         }
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        *reinterpret_cast<float4 *>(a.out + ((int64_t)b * a.Hq + g * G + h) * D + c) =
-            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        float Mb = M;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i)
+            Mb = fmaxf(Mb, ml[i].x);
+        if (Mb == -INFINITY)
+            continue;
+        const float r = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
+        L *= r;
+        acc.x *= r;
+        acc.y *= r;
+        acc.z *= r;
+        acc.w *= r;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+            if (ml[i].x != -INFINITY) {
+                const float w = exp2f(ml[i].x - Mb);
+                L = fmaf(ml[i].y, w, L);
+                acc.x = fmaf(w, v4[i].x, acc.x);
+                acc.y = fmaf(w, v4[i].y, acc.y);
+                acc.z = fmaf(w, v4[i].z, acc.z);
+                acc.w = fmaf(w, v4[i].w, acc.w);
+            }
+        }
+        M = Mb;
     }
+    s_acc[sg][c] = acc;
+    s_ml[sg][c] = make_float2(M, L);
+    __syncthreads();
+    if (sg != 0)
+        return;
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+        Mt = fmaxf(Mt, s_ml[q][c].x);
+    float Lt = 0.0f;
+    float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (Mt != -INFINITY) {
+#pragma unroll
+        for (int q = 0; q < NG; ++q) {
+            const float2 mlq = s_ml[q][c];
+            if (mlq.x != -INFINITY) {
+                const float w = exp2f(mlq.x - Mt);
+                const float4 aq = s_acc[q][c];
+                Lt = fmaf(mlq.y, w, Lt);
+                o.x = fmaf(w, aq.x, o.x);
+                o.y = fmaf(w, aq.y, o.y);
+                o.z = fmaf(w, aq.z, o.z);
+                o.w = fmaf(w, aq.w, o.w);
+            }
+        }
+    }
+    const float inv = Lt > 0.0f ? 1.0f / Lt : 0.0f;
+    *reinterpret_cast<float4 *>(a.out + ((int64_t)b * a.Hq + h) * D + 4 * c) =
+        make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
 }
 
 template <int D, int NB>
@@ -338,7 +371,7 @@ cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
     cudaError_t e = launch_ex(attn_split<D, NB>, grid, dim3(kAttnThreads), smem, st, 1, a);
     if (e != cudaSuccess)
         return e;
-    return launch_ex(attn_merge<D>, dim3((unsigned)p.Hkv, (unsigned)p.B), dim3(kAttnThreads), 0, st, 1, a);
+    return launch_ex(attn_merge<D>, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(kAttnThreads), 0, st, 1, a);
 }
 
 cudaError_t launch_attn_any(const Plan &p, const AttnArgs &a, cudaStream_t st)

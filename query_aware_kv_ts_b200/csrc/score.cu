@@ -27,10 +27,12 @@
 //  * The epilogue scales, stores the logits and keeps an online
 //    (max, sum exp) per head and thread over the CTA's chunks of a sequence;
 //    when the CTA leaves the sequence these are reduced over the CTA and
-//    written as one partial, at the slot of the CTA's first chunk in that
-//    sequence.  No fences, atomics or waits on other CTAs.
-//  * score_merge (one block per sequence and 8 heads) folds the <= grid
-//    partials of a sequence into L[b, :] after the pass: fp32 terms
+//    written as one partial of head h at slot j + b (CTA j, sequence b).  The
+//    slot is unique: along the chunk order neither j nor b decreases and one
+//    of them grows at every new (CTA, sequence) segment.  No fences, atomics
+//    or waits on other CTAs.
+//  * score_merge (one warp per sequence and head) folds the partials of
+//    CTAs j0..j1, the CTAs that cover the sequence, into L[b, h]: fp32 terms
 //    exp(m - M) <= 1 summed in float64.
 #include "ts_device.cuh"
 #include "ts_internal.h"
@@ -47,7 +49,8 @@ struct ScoreArgs {
     const int32_t *reuse;     // [B] or null
     float *logits;            // [Hq][ld]
     int64_t ld;
-    float2 *partials;         // [max_chunks][Hq] (max, sum exp(x - max))
+    float2 *partials;         // [Hq][S] (max, sum exp(x - max)) at slot CTA + sequence
+    int S;                    // slots per head: grid + B
     int32_t *chunk_table;     // [B + 1] first active chunk of each sequence (for score_merge)
     uint32_t *ctrl;           // status word
     int B, Hq, Hkv, G;
@@ -62,6 +65,7 @@ struct __align__(16) ScoreShared {
     int64_t off[kMaxBatch + 1];
     int32_t chunk_start[kMaxBatch + 1];
     float2 red[kScoreConsumerWarps][16];
+    int32_t pf_start[32];     // all-active chunk table of the prefetch hints (B <= 32)
 };
 
 __device__ __forceinline__ void online_push(float &m, float &z, float x)
@@ -114,6 +118,29 @@ __device__ __forceinline__ void build_chunk_table(ScoreShared &sh, const int32_t
     __syncthreads();
 }
 
+// B <= 32: lane b < B computes c0 = first chunk of sequence b and c1 = one past
+// its last (sequences with reuse set, when reuse is given, have no chunks),
+// with one round trip for the offsets and flags and a warp scan.
+__device__ __forceinline__ void warp_chunk_scan(const int64_t *seq_off, const int32_t *reuse, int B, int T,
+                                                int lane, int32_t &c0, int32_t &c1)
+{
+    int32_t x = 0;
+    if (lane < B) {
+        const int64_t n = __ldcg(seq_off + lane + 1) - __ldcg(seq_off + lane);
+        const bool active = reuse == nullptr || __ldcg(reuse + lane) == 0;
+        x = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
+    }
+    int32_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    c0 = incl - x;
+    c1 = incl;
+}
+
 template <int D, int NB>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
@@ -138,21 +165,47 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     // ---- before the previous kernel has finished: only L2 prefetch hints,
     //      computed as if every sequence were active (a wrong guess costs
     //      nothing but bandwidth; the data itself is read after the wait) -----
-    for (int b = tid; b <= B; b += blockDim.x)
-        sh.off[b] = a.seq_off[b];
-    __syncthreads();
-    build_chunk_table(sh, a.reuse, B, T, warp, lane, false);
-    if (warp == kScoreConsumerWarps && lane == 0) {
-        tma_prefetch_desc(&kmap);
-        const int32_t total = sh.chunk_start[B];
-        const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
-        const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
-        for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
-            const int b = upper_seq(sh.chunk_start, B, v);
-            const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+    if (B <= 32) {
+        if (warp == kScoreConsumerWarps) {
+            if (lane == 0)
+                tma_prefetch_desc(&kmap);
+            int32_t c0, c1;
+            warp_chunk_scan(a.seq_off, nullptr, B, T, lane, c0, c1);
+            if (lane < B)
+                sh.pf_start[lane] = c0;
+            const int32_t total = __shfl_sync(0xffffffffu, c1, B - 1);
+            __syncwarp();
+            if (lane == 0) {
+                const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
+                const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
+                int b = 0;
+                for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
+                    while (b + 1 < B && sh.pf_start[b + 1] <= v)
+                        ++b;
+                    const int64_t t0 = __ldcg(a.seq_off + b) + (int64_t)(v - sh.pf_start[b]) * T;
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x)
-                tma_prefetch_l2_3d(&kmap, x * 64, (int32_t)t0, 0);
+                    for (int x = 0; x < D / 64; ++x)
+                        tma_prefetch_l2_3d(&kmap, x * 64, (int32_t)t0, 0);
+                }
+            }
+        }
+    } else {
+        for (int b = tid; b <= B; b += blockDim.x)
+            sh.off[b] = __ldcg(a.seq_off + b);
+        __syncthreads();
+        build_chunk_table(sh, a.reuse, B, T, warp, lane, false);
+        if (warp == kScoreConsumerWarps && lane == 0) {
+            tma_prefetch_desc(&kmap);
+            const int32_t total = sh.chunk_start[B];
+            const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
+            const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
+            for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
+                const int b = upper_seq(sh.chunk_start, B, v);
+                const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_prefetch_l2_3d(&kmap, x * 64, (int32_t)t0, 0);
+            }
         }
     }
     pdl_wait();
@@ -161,36 +214,52 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     // ---- the real chunk table (reuse flags come from the previous kernel);
     //      the offsets are re-read too, in case a caller's kernel wrote them;
     //      offsets and flags are loaded together: one round trip -------------
-    __syncthreads();
-    for (int b = tid; b < B; b += blockDim.x) {
-        const int64_t o0 = a.seq_off[b], o1 = a.seq_off[b + 1];
-        const bool active = a.reuse == nullptr || a.reuse[b] == 0;
-        sh.off[b] = o0;
-        if (b == B - 1)
-            sh.off[B] = o1;
-        const int64_t n = o1 - o0;
-        sh.chunk_start[b + 1] = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int32_t run = 0;
-        for (int base = 0; base < B; base += 32) {
-            const int b = base + lane;
-            int32_t x = (b < B) ? sh.chunk_start[b + 1] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o)
-                    x += y;
+    if (B <= 32) {
+        if (warp == 0) {
+            int32_t c0, c1;
+            warp_chunk_scan(a.seq_off, a.reuse, B, T, lane, c0, c1);
+            if (lane < B) {
+                sh.chunk_start[lane] = c0;
+                sh.off[lane] = __ldcg(a.seq_off + lane);
             }
-            if (b < B)
-                sh.chunk_start[b + 1] = run + x;
-            run += __shfl_sync(0xffffffffu, x, 31);
+            if (lane == B - 1) {
+                sh.chunk_start[B] = c1;
+                sh.off[B] = __ldcg(a.seq_off + B);
+            }
         }
-        if (lane == 0)
-            sh.chunk_start[0] = 0;
+        __syncthreads();
+    } else {
+        __syncthreads();
+        for (int b = tid; b < B; b += blockDim.x) {
+            const int64_t o0 = __ldcg(a.seq_off + b), o1 = __ldcg(a.seq_off + b + 1);
+            const bool active = a.reuse == nullptr || __ldcg(a.reuse + b) == 0;
+            sh.off[b] = o0;
+            if (b == B - 1)
+                sh.off[B] = o1;
+            const int64_t n = o1 - o0;
+            sh.chunk_start[b + 1] = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int32_t run = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int b = base + lane;
+                int32_t x = (b < B) ? sh.chunk_start[b + 1] : 0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o)
+                        x += y;
+                }
+                if (b < B)
+                    sh.chunk_start[b + 1] = run + x;
+                run += __shfl_sync(0xffffffffu, x, 31);
+            }
+            if (lane == 0)
+                sh.chunk_start[0] = 0;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     if (blockIdx.x == 0)
         for (int b = tid; b <= B; b += blockDim.x)
             a.chunk_table[b] = sh.chunk_start[b];
@@ -240,12 +309,11 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     uint32_t bq[D / 16][NB][2];
     float m[NB][2], z[NB][2];
     int cur_b = -1;
-    int32_t seg_first = 0;
     uint32_t it = 0;
     bool dead = false;
 
     // Close this CTA's run of chunks of a sequence: reduce (max, sum) per head
-    // over the CTA and publish one partial at slot seg_first.
+    // over the CTA and publish one partial per head at slot blockIdx.x + cur_b.
     auto flush_segment = [&]() {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -266,7 +334,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             float M = -INFINITY, Z = 0.0f;
             for (int w2 = gh; w2 < kScoreConsumerWarps; w2 += Hkv)
                 lse_merge(M, Z, sh.red[w2][j].x, sh.red[w2][j].y);
-            a.partials[(int64_t)seg_first * a.Hq + h] = make_float2(M, Z);
+            a.partials[(int64_t)h * a.S + blockIdx.x + cur_b] = make_float2(M, Z);
         }
         named_bar_sync(1, kScoreConsumerWarps * 32);   // sh.red is rewritten by the next flush
     };
@@ -280,7 +348,6 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             if (cur_b >= 0)
                 flush_segment();
             cur_b = b;
-            seg_first = v;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
@@ -362,46 +429,40 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
         flush_segment();
 }
 
-// L[b, h] from the partials of sequence b: every CTA whose chunk range meets
-// [cs, ce) wrote one partial, at slot max(start_j, cs).
-__global__ void __launch_bounds__(256)
-score_merge(const float2 *partials, const int32_t *chunk_table, double *L, int B, int Hq, int grid_a)
+// L[b, h] from the partials of sequence b (one warp per sequence and head).
+// CTA j of pass A covers chunks [j*total/grid, (j+1)*total/grid); the CTAs that
+// cover the sequence's chunks [cs, ce) are j0 = owner(cs) .. j1 = owner(ce-1),
+// owner(v) = ((v+1)*grid - 1) / total, and CTA j wrote at slot j + b.  The
+// table entries and every slot the sequence could own are loaded together (one
+// round trip); slots outside j0..j1, or of CTAs without chunks, are dropped.
+__global__ void __launch_bounds__(32)
+score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L, int B, int Hq, int grid_a)
 {
     pdl_wait();
     pdl_launch_dependents();
-    const int b = blockIdx.x;
-    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    __shared__ int32_t s_start[257];
-    const int32_t cs = chunk_table[b], ce = chunk_table[b + 1], total = chunk_table[B];
-    if (cs == ce)
-        return;   // reused or empty sequence: its L is not needed
-    for (int j = threadIdx.x; j <= grid_a; j += blockDim.x)
-        s_start[j] = (int32_t)((int64_t)j * total / grid_a);   // CTA j's chunk range starts here
-    __syncthreads();
-    if (h >= Hq)
-        return;
-    auto start_of = [&](int j) { return s_start[j]; };
-    auto owner = [&](int32_t v) {   // largest j with start_of(j) <= v
-        int lo = 0, hi = grid_a;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (start_of(mid) <= v)
-                lo = mid;
-            else
-                hi = mid;
-        }
-        return lo;
-    };
-    const int j0 = owner(cs), j1 = owner(ce - 1);
-    constexpr int kPer = 8;   // slots per lane: grid_a <= 256
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x;
+    constexpr int kPer = 8;   // grid_a <= 256
+    const int32_t cs = __ldcg(chunk_table + b), ce = __ldcg(chunk_table + b + 1), total = __ldcg(chunk_table + B);
+    const float2 *row = partials + (int64_t)h * S + b;
     float2 pv[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-        const int j = j0 + lane + 32 * i;
-        pv[i] = make_float2(-INFINITY, 0.0f);
-        if (j <= j1 && start_of(j) < start_of(j + 1))   // CTAs with empty ranges wrote nothing
-            pv[i] = __ldcg(&partials[(int64_t)max(start_of(j), cs) * Hq + h]);
+        const int j = lane + 32 * i;
+        pv[i] = j < grid_a ? __ldcg(row + j) : make_float2(-INFINITY, 0.0f);
+    }
+    if (cs == ce)
+        return;   // reused or empty sequence: its L is not needed
+    const int j0 = (int)(((int64_t)(cs + 1) * grid_a - 1) / total);
+    const int j1 = (int)(((int64_t)ce * grid_a - 1) / total);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int j = lane + 32 * i;
+        bool keep = j >= j0 && j <= j1;
+        if (keep && total < grid_a)   // some CTAs had no chunks and wrote nothing
+            keep = (int64_t)j * total / grid_a < (int64_t)(j + 1) * total / grid_a;
+        if (!keep)
+            pv[i] = make_float2(-INFINITY, 0.0f);
     }
     float M = -INFINITY;
 #pragma unroll
@@ -452,6 +513,7 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.logits = reinterpret_cast<float *>(ws + p.off_logits);
     a.ld = p.ld_logits;
     a.partials = reinterpret_cast<float2 *>(ws + p.off_partials);
+    a.S = p.score_grid + p.B;
     a.chunk_table = reinterpret_cast<int32_t *>(ws + p.off_chunk_table);
     a.ctrl = reinterpret_cast<uint32_t *>(ws + p.off_ctrl);
     a.B = p.B;
@@ -468,8 +530,8 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
         e = p.G <= 8 ? launch_score_t<64, 1>(p, kmap, a, st) : launch_score_t<64, 2>(p, kmap, a, st);
     if (e != cudaSuccess)
         return e;
-    return launch_ex(score_merge, dim3((unsigned)p.B, (unsigned)((p.Hq + 7) / 8)), dim3(256), 0, st, 1,
-                     reinterpret_cast<const float2 *>(ws + p.off_partials),
+    return launch_ex(score_merge, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(32), 0, st, 1,
+                     reinterpret_cast<const float2 *>(ws + p.off_partials), p.score_grid + p.B,
                      reinterpret_cast<const int32_t *>(ws + p.off_chunk_table),
                      reinterpret_cast<double *>(ws + p.off_L), p.B, p.Hq, p.score_grid);
 }

@@ -18,13 +18,18 @@
 //                  inside b1 to the sequence's candidate list
 //  S3 sel_resolve  one CTA per sequence: exact radix select of T among the
 //                  (few) b1 candidates, 8-bit digits over the 52 key bits
-//                  below b1; range offsets = each range's candidates above b1
-//                  plus its b1 candidates >= T, prefix-summed; clears the
-//                  histogram and the list counter for the next call
+//                  below b1 until at most 32 keys share the prefix, then one
+//                  warp ranks those directly; range offsets = each range's
+//                  candidates above b1 plus its b1 candidates >= T,
+//                  prefix-summed; clears the histogram and the list counter
+//                  for the next call
 //  S4 sel_write    every range writes its selected ids in ascending order at
 //                  its offset (one block scan); range 0 also writes the sink
 //                  and local windows, the count and the -1 padding
 // No kernel waits on another CTA: the four steps are ordered by the stream.
+// The one-call decode step builds S0's histogram inside the vote pass and
+// starts at S2.  Every kernel fetches what it needs in at most two round trips
+// (the loads that do not depend on one another are issued together).
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -46,6 +51,7 @@ struct SelArgs {
     uint32_t *hist;            // [B][4096]
     uint2 *cand;               // [n_total] (vote bits, token id), sequence b's list at seq_off[b]
     uint32_t *cand_n;          // [B]
+    uint2 *bin;                // [B] (b1, candidates above b1), written by S2
     uint32_t *above;           // [B][rps] candidates above bin b1, per range
     uint32_t *range_off;       // [B][rps] output offset of each range within the top-k part
     unsigned long long *thr;   // [B] threshold key T
@@ -57,11 +63,11 @@ struct Window {
     int64_t off, n, s_end, l0, nc, keff;
 };
 
-__device__ __forceinline__ Window window_of(const SelArgs &a, int b)
+__device__ __forceinline__ Window make_window(const SelArgs &a, int64_t off, int64_t end)
 {
     Window w;
-    w.off = a.seq_off[b];
-    w.n = a.seq_off[b + 1] - w.off;
+    w.off = off;
+    w.n = end - off;
     w.s_end = min((int64_t)a.n_sink, w.n);
     w.l0 = max(w.n - (int64_t)a.n_local, w.s_end);
     w.nc = w.l0 - w.s_end;
@@ -74,17 +80,19 @@ __device__ __forceinline__ unsigned long long make_key(uint32_t vbits, int64_t i
     return ((unsigned long long)vbits << 32) | (unsigned long long)(0xffffffffu - (uint32_t)id);
 }
 
-// Copy the 4096-bin histogram of sequence b into shared memory, every load of
-// the thread issued before the first store.
-__device__ __forceinline__ void load_hist(uint32_t *h, const uint32_t *gh)
+// The 4096-bin histogram of a sequence: loads into registers (issued
+// together), then the copy to shared memory.
+constexpr int kHistPer = 4096 / NT;
+__device__ __forceinline__ void load_hist_regs(uint32_t (&v)[kHistPer], const uint32_t *gh)
 {
-    constexpr int kPerThread = 4096 / NT;
-    uint32_t v[kPerThread];
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u)
+    for (int u = 0; u < kHistPer; ++u)
         v[u] = __ldcg(gh + u * NT + threadIdx.x);
+}
+__device__ __forceinline__ void store_hist(uint32_t *h, const uint32_t (&v)[kHistPer])
+{
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u)
+    for (int u = 0; u < kHistPer; ++u)
         h[u * NT + threadIdx.x] = v[u];
 }
 
@@ -164,15 +172,17 @@ sel_hist(const SelArgs a)
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.y, r = blockIdx.x;
-    if (a.reuse != nullptr && a.reuse[b] != 0)
+    const int32_t re = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+    const int64_t off = __ldcg(a.seq_off + b), end = __ldcg(a.seq_off + b + 1);
+    for (int i = threadIdx.x; i < 4096; i += NT)
+        h[i] = 0u;
+    if (re != 0)
         return;
-    const Window w = window_of(a, b);
+    const Window w = make_window(a, off, end);
     const int64_t lo = w.s_end + (int64_t)r * kTPC;
     if (w.keff == 0 || w.keff == w.nc || lo >= w.l0)
         return;
     const int64_t hi = min(lo + kTPC, w.l0);
-    for (int i = threadIdx.x; i < 4096; i += NT)
-        h[i] = 0u;
     const uint32_t *vb = a.votes + w.off;
     uint32_t kk[kPer];
 #pragma unroll
@@ -217,13 +227,19 @@ sel_collect(const SelArgs a)
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.y, r = blockIdx.x;
-    if (a.reuse != nullptr && a.reuse[b] != 0)
+    // round trip 1: flag, bounds and the sequence's histogram
+    const int32_t re = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+    const int64_t off = __ldcg(a.seq_off + b), end = __ldcg(a.seq_off + b + 1);
+    uint32_t hv[kHistPer];
+    load_hist_regs(hv, a.hist + (size_t)b * 4096);
+    if (re != 0)
         return;
-    const Window w = window_of(a, b);
+    const Window w = make_window(a, off, end);
     const int64_t lo = w.s_end + (int64_t)r * kTPC;
     if (w.keff == 0 || w.keff == w.nc || lo >= w.l0)
         return;
     const int64_t hi = min(lo + kTPC, w.l0);
+    // round trip 2: the range's votes
     const uint32_t *vb = a.votes + w.off;
     uint32_t kk[kPer];
 #pragma unroll
@@ -231,10 +247,12 @@ sel_collect(const SelArgs a)
         const int64_t i = lo + u * NT + threadIdx.x;
         kk[u] = i < hi ? __ldcg(vb + i) : 0u;
     }
-    load_hist(h, a.hist + (size_t)b * 4096);
+    store_hist(h, hv);
     __syncthreads();
     uint32_t b1, above_b1;
     bin_from_top(h, 4096, w.keff, tmp, bc, b1, above_b1);
+    if (r == 0 && threadIdx.x == 0)
+        a.bin[b] = make_uint2(b1, above_b1);   // every range finds the same b1
 
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
@@ -270,17 +288,33 @@ sel_collect(const SelArgs a)
 __global__ void __launch_bounds__(NT)
 sel_resolve(const SelArgs a)
 {
-    __shared__ uint32_t h[4096];
+    constexpr int kAbovePer = kMaxSelectRanges / NT;   // per-range counts held per thread
+    __shared__ uint32_t h[NT];                         // one digit's histogram (<= 256 bins)
     __shared__ uint32_t tmp[kWarps + 1];
-    __shared__ uint32_t bc[2];
+    __shared__ uint32_t bc[3];
     __shared__ unsigned long long keys[kResolveSmem];
     __shared__ uint32_t rcnt[kMaxSelectRanges];
+    __shared__ unsigned long long s_list[32];
+    __shared__ uint32_t s_nlist;
+    __shared__ unsigned long long s_T;
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.x;
-    if (a.reuse != nullptr && a.reuse[b] != 0)
+    // round trip 1: flag, bounds, list length, b1 with the count above it, and
+    // the per-range counts above b1
+    const int32_t re = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+    const int64_t off = __ldcg(a.seq_off + b), end = __ldcg(a.seq_off + b + 1);
+    const uint32_t m = __ldcg(&a.cand_n[b]);
+    const uint2 bn = __ldcg(&a.bin[b]);
+    uint32_t ab[kAbovePer];
+#pragma unroll
+    for (int u = 0; u < kAbovePer; ++u) {
+        const int r = u * NT + threadIdx.x;
+        ab[u] = r < a.rps ? __ldcg(&a.above[(size_t)b * a.rps + r]) : 0u;
+    }
+    if (re != 0)
         return;
-    const Window w = window_of(a, b);
+    const Window w = make_window(a, off, end);
     const int nranges = (int)((w.nc + kTPC - 1) / kTPC);
     if (w.keff == 0 || w.keff == w.nc) {
         if (threadIdx.x == 0) {
@@ -293,13 +327,9 @@ sel_resolve(const SelArgs a)
         return;
     }
     uint32_t *gh = a.hist + (size_t)b * 4096;
-    const uint32_t m = __ldcg(&a.cand_n[b]);
-    load_hist(h, gh);
-    __syncthreads();
-    uint32_t b1, above_b1;
-    bin_from_top(h, 4096, w.keff, tmp, bc, b1, above_b1);
     for (int i = threadIdx.x; i < 4096; i += NT)
         gh[i] = 0u;                                  // ready for the next call
+    // round trip 2: the b1 candidates
     const uint2 *cl = a.cand + w.off;
     const bool in_smem = m <= (uint32_t)kResolveSmem;
     if (in_smem) {
@@ -315,6 +345,8 @@ sel_resolve(const SelArgs a)
                     keys[j0 + u * NT] = make_key(c[u].x, c[u].y);
         }
     }
+    if (threadIdx.x == 0)
+        s_nlist = 0u;
     __syncthreads();
     auto key_at = [&](uint32_t j) -> unsigned long long {
         if (in_smem)
@@ -324,11 +356,13 @@ sel_resolve(const SelArgs a)
     };
 
     // radix select of the need-th largest key among the m candidates: they
-    // share the top 12 bits (b1); 8-bit digits over bits 51..4, then 3..0
-    int64_t need = (int64_t)w.keff - above_b1;
-    unsigned long long prefix = (unsigned long long)b1 << 52;
+    // share the top 12 bits (b1); 8-bit digits over bits 51..4, then 3..0,
+    // while more than 32 keys share the prefix found so far
+    int64_t need = (int64_t)w.keff - bn.y;
+    unsigned long long prefix = (unsigned long long)bn.x << 52;
     unsigned long long pmask = 0xfffull << 52;
-    for (int shift = 44; shift >= -4; shift -= 8) {
+    uint32_t alive = m;
+    for (int shift = 44; alive > 32u && shift >= -4; shift -= 8) {
         const int sh = shift < 0 ? 0 : shift;
         const int nb = shift < 0 ? 16 : 256;
         h[threadIdx.x] = 0u;
@@ -346,15 +380,47 @@ sel_resolve(const SelArgs a)
         if (t < nb && (int64_t)ex < need && (int64_t)(ex + c) >= need) {
             bc[0] = (uint32_t)(nb - 1 - t);
             bc[1] = ex;
+            bc[2] = c;
         }
         __syncthreads();
         const uint32_t dig = bc[0];
         need -= bc[1];
+        alive = bc[2];
         __syncthreads();
         prefix |= (unsigned long long)dig << sh;
         pmask |= (unsigned long long)(nb - 1) << sh;
     }
-    const unsigned long long T = prefix;   // the k-th largest key
+    unsigned long long T;
+    if (pmask == ~0ull) {
+        T = prefix;   // every bit resolved: the one key left
+    } else {
+        // at most 32 keys share the prefix (keys are distinct): list them and
+        // let one warp rank them against each other
+        for (uint32_t j = threadIdx.x; j < m; j += NT) {
+            const unsigned long long key = key_at(j);
+            if ((key & pmask) == prefix) {
+                const uint32_t pos = atomicAdd(&s_nlist, 1u);
+                if (pos < 32u)
+                    s_list[pos] = key;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            const uint32_t c = min(s_nlist, 32u);
+            const unsigned long long mine = lane < (int)c ? s_list[lane] : 0ull;
+            uint32_t rank = 0;
+#pragma unroll
+            for (int l = 0; l < 32; ++l) {
+                const unsigned long long o = __shfl_sync(0xffffffffu, mine, l);
+                rank += (l < (int)c && o > mine) ? 1u : 0u;
+            }
+            if (lane < (int)c && (int64_t)rank == need - 1)
+                s_T = mine;
+        }
+        __syncthreads();
+        T = s_T;
+    }
 
     // per-range counts of selected b1 candidates, then range offsets
     for (int r = threadIdx.x; r < nranges; r += NT)
@@ -369,9 +435,12 @@ sel_resolve(const SelArgs a)
     }
     __syncthreads();
     uint32_t run = 0;
-    for (int r0 = 0; r0 < nranges; r0 += NT) {
-        const int r = r0 + threadIdx.x;
-        const uint32_t c = r < nranges ? __ldcg(&a.above[(size_t)b * a.rps + r]) + rcnt[r] : 0u;
+#pragma unroll
+    for (int u = 0; u < kAbovePer; ++u) {
+        if (u * NT >= nranges)
+            break;
+        const int r = u * NT + threadIdx.x;
+        const uint32_t c = r < nranges ? ab[u] + rcnt[r] : 0u;
         uint32_t tot;
         const uint32_t ex = block_excl_scan(c, tmp, tot);
         if (r < nranges)
@@ -392,12 +461,19 @@ __global__ void __launch_bounds__(NT)
 sel_write(const SelArgs a)
 {
     __shared__ uint32_t tmp[kWarps + 1];
+    __shared__ __align__(16) uint32_t sv[kTPC];
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.y, r = blockIdx.x;
-    if (a.reuse != nullptr && a.reuse[b] != 0)
+    // round trip 1: flag, bounds, mode, threshold and this range's offset
+    const int32_t re = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+    const int64_t off = __ldcg(a.seq_off + b), end = __ldcg(a.seq_off + b + 1);
+    const int md = __ldcg(&a.mode[b]);
+    const unsigned long long T = __ldcg(&a.thr[b]);
+    const uint32_t base = r < a.rps ? __ldcg(&a.range_off[(size_t)b * a.rps + r]) : 0u;
+    if (re != 0)
         return;   // the previous ids stay
-    const Window w = window_of(a, b);
+    const Window w = make_window(a, off, end);
     int32_t *idrow = a.ids + (int64_t)b * a.cap;
     if (r == 0) {
         const int64_t mcount = w.s_end + w.keff + (w.n - w.l0);
@@ -411,25 +487,34 @@ sel_write(const SelArgs a)
             a.count[b] = (int32_t)mcount;
     }
     const int64_t lo = w.s_end + (int64_t)r * kTPC;
-    if (lo >= w.l0)
-        return;
-    const int md = __ldcg(&a.mode[b]);
-    if (md == 0)
+    if (lo >= w.l0 || md == 0)
         return;
     const int64_t hi = min(lo + kTPC, w.l0);
-    const unsigned long long T = __ldcg(&a.thr[b]);
-    const uint32_t base = __ldcg(&a.range_off[(size_t)b * a.rps + r]);
-    // each thread takes kPer consecutive candidates, so one block scan orders them
-    const int64_t t0 = lo + (int64_t)threadIdx.x * kPer;
+    // round trip 2: the range's votes, loaded coalesced and regrouped through
+    // shared memory so that each thread owns kPer consecutive candidates
     const uint32_t *vb = a.votes + w.off;
+    {
+        uint32_t v[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int64_t i = lo + u * NT + threadIdx.x;
+            v[u] = i < hi ? __ldcg(vb + i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u)
+            sv[u * NT + threadIdx.x] = v[u];
+    }
+    __syncthreads();
+    const int64_t t0 = lo + (int64_t)threadIdx.x * kPer;
+    const uint4 va = *reinterpret_cast<const uint4 *>(sv + threadIdx.x * kPer);
+    const uint4 vc = *reinterpret_cast<const uint4 *>(sv + threadIdx.x * kPer + 4);
+    const uint32_t mv[kPer] = {va.x, va.y, va.z, va.w, vc.x, vc.y, vc.z, vc.w};
     bool f[kPer];
     uint32_t cnt = 0;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int64_t i = t0 + u;
-        f[u] = false;
-        if (i < hi)
-            f[u] = md == 2 || make_key(__ldcg(vb + i), i) >= T;
+        f[u] = i < hi && (md == 2 || make_key(mv[u], i) >= T);
         cnt += f[u] ? 1u : 0u;
     }
     uint32_t tot;
@@ -449,7 +534,7 @@ sel_write(const SelArgs a)
 
 cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,
                           int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, uint8_t *ws,
-                          cudaStream_t st)
+                          cudaStream_t st, bool hist_ready)
 {
     SelArgs a;
     a.votes = reinterpret_cast<const uint32_t *>(votes);
@@ -460,6 +545,7 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
     a.hist = reinterpret_cast<uint32_t *>(ws + p.off_sel_hist);
     a.cand = reinterpret_cast<uint2 *>(ws + p.off_sel_cand);
     a.cand_n = reinterpret_cast<uint32_t *>(ws + p.off_sel_cand_n);
+    a.bin = reinterpret_cast<uint2 *>(ws + p.off_sel_bin);
     a.above = reinterpret_cast<uint32_t *>(ws + p.off_sel_above);
     a.range_off = reinterpret_cast<uint32_t *>(ws + p.off_sel_range_off);
     a.thr = reinterpret_cast<unsigned long long *>(ws + p.off_sel_thr);
@@ -471,7 +557,7 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
     a.B = p.B;
     a.rps = p.sel_ranges;
     const dim3 grid((unsigned)p.sel_ranges, (unsigned)p.B);
-    cudaError_t e = launch_ex(sel_hist, grid, dim3(NT), 0, st, 1, a);
+    cudaError_t e = hist_ready ? cudaSuccess : launch_ex(sel_hist, grid, dim3(NT), 0, st, 1, a);
     if (e == cudaSuccess)
         e = launch_ex(sel_collect, grid, dim3(NT), 0, st, 1, a);
     if (e == cudaSuccess)

@@ -82,7 +82,8 @@ struct Plan {
     int attn_splits;
     // workspace layout (byte offsets)
     size_t off_ctrl, off_chunk_table, off_L, off_partials, off_logits, off_sel_hist, off_sel_cand,
-        off_sel_cand_n, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part, total_bytes;
+        off_sel_cand_n, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part,
+        total_bytes;
 };
 
 // Fill `p` from the cache description (capacity < 0: attention part not
@@ -98,12 +99,19 @@ cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double 
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
                          const int32_t *reuse, uint8_t *ws, cudaStream_t st);
 
-cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
-                        cudaStream_t st);
+// Selection parameters, for the vote pass that also builds the selection's
+// level-1 histogram.
+struct SelectWindow {
+    int k, n_sink, n_local;
+};
 
+cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
+                        cudaStream_t st, const SelectWindow *hist_window = nullptr);
+
+// hist_ready: the level-1 histogram was already built by the vote pass.
 cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,
                           int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, uint8_t *ws,
-                          cudaStream_t st);
+                          cudaStream_t st, bool hist_ready = false);
 
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
                         const int32_t *count, float *out, uint8_t *ws, cudaStream_t st);

@@ -19,6 +19,13 @@
 // consecutive tokens aligned to 4 in the logits rows (row stride padded to 4),
 // so each head's logits arrive as one 16-byte load, 8 heads at a time; short
 // sequences: one token per thread, 32 heads loaded at a time, 64-thread blocks.
+// The reuse flag, the sequence bounds and the normalisers L are fetched in one
+// round trip, the logits in the next.
+//
+// With a histogram buffer (the one-call decode step) the pass also builds the
+// selection's level-1 histogram of its candidates' votes (top 12 bits of the
+// fp32 pattern, the bins the selection starts from): a shared-memory
+// histogram per block, merged into the sequence's global one with atomics.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -32,6 +39,8 @@ struct VoteArgs {
     const int64_t *seq_off;
     const int32_t *reuse;
     float *votes;
+    uint32_t *hist;        // [B][4096] level-1 selection histogram, or null
+    int k, n_sink, n_local;
     int B, Hq;
 };
 
@@ -53,80 +62,130 @@ __device__ __forceinline__ float exp_exact_arg(float s, float Lhi, float Llo)
     return fmaf(p, u_lo * kLn2, p);
 }
 
-template <int TPT>
+template <int TPT, bool HIST>
 __global__ void __launch_bounds__(kVoteThreads)
 vote_pass_b(const VoteArgs a)
 {
     __shared__ float s_hi[kMaxHeadsVote], s_lo[kMaxHeadsVote];
+    __shared__ uint32_t s_hist[HIST ? 4096 : 1];
+    const int tid = threadIdx.x;
+    const int nt = blockDim.x;
+    if (HIST)
+        for (int i = tid; i < 4096; i += nt)
+            s_hist[i] = 0u;
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.y;
-    const int tid = threadIdx.x;
-    if (a.reuse != nullptr && a.reuse[b] != 0)
+    // one round trip: flag, bounds and normalisers (h_q <= 2 * blockDim)
+    const int32_t r = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+    const int64_t off = __ldcg(a.seq_off + b);
+    const int64_t end = __ldcg(a.seq_off + b + 1);
+    double Lv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int h = tid + u * nt;
+        Lv[u] = h < a.Hq ? __ldcg(a.L + (int64_t)b * a.Hq + h) : 0.0;
+    }
+    if (r != 0)
         return;
-    const int64_t off = a.seq_off[b];
-    const int64_t end = a.seq_off[b + 1];
     const int64_t base = off & ~int64_t(TPT - 1);                  // first aligned group of the sequence
-    const int nt = blockDim.x;
     const int64_t i0 = base + ((int64_t)blockIdx.x * nt + tid) * TPT;
     if (base + (int64_t)blockIdx.x * nt * TPT >= end)
         return;   // the whole block is past this sequence
-    for (int h = tid; h < a.Hq; h += nt) {
-        const double L = a.L[(int64_t)b * a.Hq + h];
-        const float hi = (float)L;
-        s_hi[h] = hi;
-        s_lo[h] = (float)(L - (double)hi);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int h = tid + u * nt;
+        if (h < a.Hq) {
+            const float hi = (float)Lv[u];
+            s_hi[h] = hi;
+            s_lo[h] = (float)(Lv[u] - (double)hi);
+        }
     }
     __syncthreads();
-    if (i0 >= end)
-        return;
     float acc[TPT];
 #pragma unroll
     for (int j = 0; j < TPT; ++j)
         acc[j] = 0.0f;
-    if constexpr (TPT == 4) {
-        for (int h0 = 0; h0 < a.Hq; h0 += kHeadBatch) {
-            float4 sv[kHeadBatch];
+    if (i0 < end) {
+        if constexpr (TPT == 4) {
+            for (int h0 = 0; h0 < a.Hq; h0 += kHeadBatch) {
+                float4 sv[kHeadBatch];
 #pragma unroll
-            for (int u = 0; u < kHeadBatch; ++u)
-                if (h0 + u < a.Hq)
-                    sv[u] = __ldcg(reinterpret_cast<const float4 *>(a.logits + (int64_t)(h0 + u) * a.ld + i0));
+                for (int u = 0; u < kHeadBatch; ++u)
+                    if (h0 + u < a.Hq)
+                        sv[u] = __ldcg(reinterpret_cast<const float4 *>(a.logits + (int64_t)(h0 + u) * a.ld + i0));
 #pragma unroll
-            for (int u = 0; u < kHeadBatch; ++u) {
-                if (h0 + u < a.Hq) {
-                    const float Lhi = s_hi[h0 + u], Llo = s_lo[h0 + u];
-                    acc[0] += exp_exact_arg(sv[u].x, Lhi, Llo);
-                    acc[1] += exp_exact_arg(sv[u].y, Lhi, Llo);
-                    acc[2] += exp_exact_arg(sv[u].z, Lhi, Llo);
-                    acc[3] += exp_exact_arg(sv[u].w, Lhi, Llo);
+                for (int u = 0; u < kHeadBatch; ++u) {
+                    if (h0 + u < a.Hq) {
+                        const float Lhi = s_hi[h0 + u], Llo = s_lo[h0 + u];
+                        acc[0] += exp_exact_arg(sv[u].x, Lhi, Llo);
+                        acc[1] += exp_exact_arg(sv[u].y, Lhi, Llo);
+                        acc[2] += exp_exact_arg(sv[u].z, Lhi, Llo);
+                        acc[3] += exp_exact_arg(sv[u].w, Lhi, Llo);
+                    }
                 }
             }
+        } else {
+            for (int h0 = 0; h0 < a.Hq; h0 += 4 * kHeadBatch) {
+                float sv[4 * kHeadBatch];
+#pragma unroll
+                for (int u = 0; u < 4 * kHeadBatch; ++u)
+                    if (h0 + u < a.Hq)
+                        sv[u] = __ldcg(a.logits + (int64_t)(h0 + u) * a.ld + i0);
+#pragma unroll
+                for (int u = 0; u < 4 * kHeadBatch; ++u)
+                    if (h0 + u < a.Hq)
+                        acc[0] += exp_exact_arg(sv[u], s_hi[h0 + u], s_lo[h0 + u]);
+            }
         }
-    } else {
-        for (int h0 = 0; h0 < a.Hq; h0 += 4 * kHeadBatch) {
-            float sv[4 * kHeadBatch];
 #pragma unroll
-            for (int u = 0; u < 4 * kHeadBatch; ++u)
-                if (h0 + u < a.Hq)
-                    sv[u] = __ldcg(a.logits + (int64_t)(h0 + u) * a.ld + i0);
-#pragma unroll
-            for (int u = 0; u < 4 * kHeadBatch; ++u)
-                if (h0 + u < a.Hq)
-                    acc[0] += exp_exact_arg(sv[u], s_hi[h0 + u], s_lo[h0 + u]);
+        for (int j = 0; j < TPT; ++j) {
+            const int64_t i = i0 + j;
+            if (i >= off && i < end)
+                a.votes[i] = acc[j];
         }
     }
+    if constexpr (HIST) {
+        // candidates [s', l0) of the sequence; nothing to rank when the
+        // selection takes none or all of them (block-uniform)
+        const int64_t n = end - off;
+        const int64_t s_end = min((int64_t)a.n_sink, n);
+        const int64_t l0 = max(n - (int64_t)a.n_local, s_end);
+        const int64_t keff = min((int64_t)a.k, l0 - s_end);
+        if (keff == 0 || keff == l0 - s_end)
+            return;
+        const int lane = tid & 31;
 #pragma unroll
-    for (int j = 0; j < TPT; ++j) {
-        const int64_t i = i0 + j;
-        if (i >= off && i < end)
-            a.votes[i] = acc[j];
+        for (int j = 0; j < TPT; ++j) {
+            const int64_t li = i0 + j - off;   // sequence-local id
+            const bool cand = i0 < end && li >= s_end && li < l0;
+            const uint32_t bin = cand ? (__float_as_uint(acc[j]) >> 20) : 0xffffffffu;
+            // one atomic for the warp's first bin, one per lane for the others
+            const uint32_t act = __ballot_sync(0xffffffffu, cand);
+            if (act) {
+                const int leader = __ffs(act) - 1;
+                const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+                const uint32_t same = __ballot_sync(0xffffffffu, bin == lb);
+                if (lane == leader)
+                    atomicAdd(&s_hist[lb], (uint32_t)__popc(same));
+                else if (cand && bin != lb)
+                    atomicAdd(&s_hist[bin], 1u);
+            }
+        }
+        __syncthreads();
+        uint32_t *gh = a.hist + (size_t)b * 4096;
+        for (int i = tid; i < 4096; i += nt) {
+            const uint32_t c = s_hist[i];
+            if (c != 0u)
+                atomicAdd(&gh[i], c);
+        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
-                        cudaStream_t st)
+                        cudaStream_t st, const SelectWindow *hist_window)
 {
     if (p.n_max <= 0)
         return cudaSuccess;
@@ -137,19 +196,28 @@ cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *re
     a.seq_off = seq_off;
     a.reuse = reuse;
     a.votes = votes;
+    a.hist = hist_window != nullptr ? reinterpret_cast<uint32_t *>(ws + p.off_sel_hist) : nullptr;
+    a.k = hist_window != nullptr ? hist_window->k : 0;
+    a.n_sink = hist_window != nullptr ? hist_window->n_sink : 0;
+    a.n_local = hist_window != nullptr ? hist_window->n_local : 0;
     a.B = p.B;
     a.Hq = p.Hq;
-    // quads of a sequence: its tokens plus up to 3 before the first aligned index
     // long sequences: 4 tokens per thread (16-byte loads, 256 threads);
-    // short ones: 1 token per thread in 64-thread blocks, so that enough warps
-    // share the latency-bound pass
+    // short ones: 1 token per thread, in 64-thread blocks so that enough warps
+    // share the latency-bound pass (256 with the histogram, whose per-block
+    // clear and merge cost 4096 bins)
     if (p.n_total > 262144) {
         const int64_t groups = (p.n_max + 3) / 4 + 1;
         const unsigned gx = (unsigned)((groups + kVoteThreads - 1) / kVoteThreads);
-        return launch_ex(vote_pass_b<4>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
+        if (a.hist != nullptr)
+            return launch_ex(vote_pass_b<4, true>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
+        return launch_ex(vote_pass_b<4, false>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
     }
-    const unsigned gx = (unsigned)((p.n_max + 63) / 64);
-    return launch_ex(vote_pass_b<1>, dim3(gx, (unsigned)p.B), dim3(64), 0, st, 1, a);
+    const int nt = a.hist != nullptr ? kVoteThreads : 64;
+    const unsigned gx = (unsigned)((p.n_max + nt) / nt);
+    if (a.hist != nullptr)
+        return launch_ex(vote_pass_b<1, true>, dim3(gx, (unsigned)p.B), dim3(nt), 0, st, 1, a);
+    return launch_ex(vote_pass_b<1, false>, dim3(gx, (unsigned)p.B), dim3(nt), 0, st, 1, a);
 }
 
 }  // namespace ts
