@@ -199,8 +199,8 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
     p->off_partials = o;
     o = align_up(o + sizeof(float) * 2 * (size_t)(p->score_grid + p->B) * p->Hq, 256);
-    p->off_sel_cand_n = o;
-    o = align_up(o + sizeof(uint32_t) * (size_t)p->B, 256);
+    p->off_sel_inb1 = o;
+    o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
     p->off_sel_bin = o;
     o = align_up(o + sizeof(uint32_t) * 2 * (size_t)p->B, 256);
     p->off_sel_above = o;

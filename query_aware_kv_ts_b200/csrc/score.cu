@@ -66,6 +66,7 @@ struct __align__(16) ScoreShared {
     int32_t chunk_start[kMaxBatch + 1];
     float2 red[kScoreConsumerWarps][16];
     int32_t pf_start[32];     // all-active chunk table of the prefetch hints (B <= 32)
+    int64_t pf_off[32];       // and the sequence offsets it was built from
 };
 
 __device__ __forceinline__ void online_push(float &m, float &z, float x)
@@ -122,11 +123,14 @@ __device__ __forceinline__ void build_chunk_table(ScoreShared &sh, const int32_t
 // its last (sequences with reuse set, when reuse is given, have no chunks),
 // with one round trip for the offsets and flags and a warp scan.
 __device__ __forceinline__ void warp_chunk_scan(const int64_t *seq_off, const int32_t *reuse, int B, int T,
-                                                int lane, int32_t &c0, int32_t &c1)
+                                                int lane, int32_t &c0, int32_t &c1, int64_t &o0, int64_t &o1)
 {
     int32_t x = 0;
+    o0 = o1 = 0;
     if (lane < B) {
-        const int64_t n = __ldcg(seq_off + lane + 1) - __ldcg(seq_off + lane);
+        o0 = __ldcg(seq_off + lane);
+        o1 = __ldcg(seq_off + lane + 1);
+        const int64_t n = o1 - o0;
         const bool active = reuse == nullptr || __ldcg(reuse + lane) == 0;
         x = (active && n > 0) ? (int32_t)((n + T - 1) / T) : 0;
     }
@@ -170,9 +174,12 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             if (lane == 0)
                 tma_prefetch_desc(&kmap);
             int32_t c0, c1;
-            warp_chunk_scan(a.seq_off, nullptr, B, T, lane, c0, c1);
-            if (lane < B)
+            int64_t o0, o1;
+            warp_chunk_scan(a.seq_off, nullptr, B, T, lane, c0, c1, o0, o1);
+            if (lane < B) {
                 sh.pf_start[lane] = c0;
+                sh.pf_off[lane] = o0;
+            }
             const int32_t total = __shfl_sync(0xffffffffu, c1, B - 1);
             __syncwarp();
             if (lane == 0) {
@@ -182,7 +189,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
                 for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
                     while (b + 1 < B && sh.pf_start[b + 1] <= v)
                         ++b;
-                    const int64_t t0 = __ldcg(a.seq_off + b) + (int64_t)(v - sh.pf_start[b]) * T;
+                    const int64_t t0 = sh.pf_off[b] + (int64_t)(v - sh.pf_start[b]) * T;
 #pragma unroll
                     for (int x = 0; x < D / 64; ++x)
                         tma_prefetch_l2_3d(&kmap, x * 64, (int32_t)t0, 0);
@@ -217,14 +224,15 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     if (B <= 32) {
         if (warp == 0) {
             int32_t c0, c1;
-            warp_chunk_scan(a.seq_off, a.reuse, B, T, lane, c0, c1);
+            int64_t o0, o1;
+            warp_chunk_scan(a.seq_off, a.reuse, B, T, lane, c0, c1, o0, o1);
             if (lane < B) {
                 sh.chunk_start[lane] = c0;
-                sh.off[lane] = __ldcg(a.seq_off + lane);
+                sh.off[lane] = o0;
             }
             if (lane == B - 1) {
                 sh.chunk_start[B] = c1;
-                sh.off[B] = __ldcg(a.seq_off + B);
+                sh.off[B] = o1;
             }
         }
         __syncthreads();

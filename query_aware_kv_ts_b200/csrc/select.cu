@@ -14,15 +14,15 @@
 //  S0 sel_hist     histogram of the top 12 vote bits of the candidates
 //                  (shared-memory histogram per range, then global atomics)
 //  S2 sel_collect  every range finds the bin b1 that holds the k-th largest
-//                  vote, counts its candidates above b1 and appends the ones
-//                  inside b1 to the sequence's candidate list
+//                  vote, counts its candidates above b1 and inside b1, and
+//                  writes the ones inside b1 to its own slots of the
+//                  candidate list (no atomics: slots [r*2048, r*2048 + count))
 //  S3 sel_resolve  one CTA per sequence: exact radix select of T among the
 //                  (few) b1 candidates, 8-bit digits over the 52 key bits
 //                  below b1 until at most 32 keys share the prefix, then one
 //                  warp ranks those directly; range offsets = each range's
 //                  candidates above b1 plus its b1 candidates >= T,
-//                  prefix-summed; clears the histogram and the list counter
-//                  for the next call
+//                  prefix-summed; clears the histogram for the next call
 //  S4 sel_write    every range writes its selected ids in ascending order at
 //                  its offset (one block scan); range 0 also writes the sink
 //                  and local windows, the count and the -1 padding
@@ -49,8 +49,8 @@ struct SelArgs {
     int32_t *ids;              // [B][cap]
     int32_t *count;            // [B]
     uint32_t *hist;            // [B][4096]
-    uint2 *cand;               // [n_total] (vote bits, token id), sequence b's list at seq_off[b]
-    uint32_t *cand_n;          // [B]
+    uint2 *cand;               // [n_total] (vote bits, token id); range r of sequence b at seq_off[b] + r*2048
+    uint32_t *inb1;            // [B][rps] candidates inside bin b1, per range
     uint2 *bin;                // [B] (b1, candidates above b1), written by S2
     uint32_t *above;           // [B][rps] candidates above bin b1, per range
     uint32_t *range_off;       // [B][rps] output offset of each range within the top-k part
@@ -96,7 +96,8 @@ __device__ __forceinline__ void store_hist(uint32_t *h, const uint32_t (&v)[kHis
         h[u * NT + threadIdx.x] = v[u];
 }
 
-// Exclusive scan over the block of one value per thread (all threads call).
+// Exclusive scan over the block of one value per thread (all threads call):
+// warp scans, one barrier, then every warp scans the warp totals itself.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *tmp, uint32_t &total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -110,56 +111,56 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *tmp, u
     if (lane == 31)
         tmp[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        const uint32_t w = lane < kWarps ? tmp[lane] : 0u;
-        uint32_t wi = w;
+    const uint32_t w = lane < kWarps ? tmp[lane] : 0u;
+    uint32_t wi = w;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o)
-                wi += y;
-        }
-        if (lane < kWarps)
-            tmp[lane] = wi - w;
-        if (lane == kWarps - 1)
-            tmp[kWarps] = wi;
+    for (int o = 1; o < kWarps; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o)
+            wi += y;
     }
-    __syncthreads();
-    const uint32_t ex = tmp[warp] + incl - x;
-    total = tmp[kWarps];
-    __syncthreads();
-    return ex;
+    const uint32_t before = __shfl_sync(0xffffffffu, wi - w, warp);
+    total = __shfl_sync(0xffffffffu, wi, kWarps - 1);
+    __syncthreads();   // tmp is rewritten by the next scan
+    return before + incl - x;
 }
 
-// In a histogram of nb bins (bin nb-1 on top, nb a multiple of NT), the bin
-// holding the need-th key counted from the top, and the keys above it.
-// Each thread owns nb / NT consecutive bins from the top.  All threads call.
-__device__ __forceinline__ void bin_from_top(const uint32_t *h, int nb, int64_t need, uint32_t *tmp,
-                                             uint32_t *bc, uint32_t &bin, uint32_t &above)
+// In the 4096-bin histogram (bin 4095 on top), the bin holding the need-th key
+// counted from the top, and the keys above it.  Thread t owns the 16
+// consecutive bins 4095-16t .. 4080-16t, kept in registers.  All threads call.
+__device__ __forceinline__ void bin_from_top(const uint32_t *h, int64_t need, uint32_t *tmp, uint32_t *bc,
+                                             uint32_t &bin, uint32_t &above)
 {
-    const int per = nb / NT;
-    const int r0 = threadIdx.x * per;   // reversed index r: bin nb-1-r
+    constexpr int kNb = 4096, kOwn = kNb / NT;
+    const int top = kNb - 1 - threadIdx.x * kOwn;
+    uint32_t c[kOwn];
     uint32_t local = 0;
-    for (int r = r0; r < r0 + per; ++r)
-        local += h[nb - 1 - r];
+#pragma unroll
+    for (int i = 0; i < kOwn; ++i) {
+        c[i] = h[top - i];
+        local += c[i];
+    }
     uint32_t tot;
     const uint32_t ex = block_excl_scan(local, tmp, tot);
-    int64_t cum = ex;
-    if (cum < need && cum + (int64_t)local >= need) {
-        for (int r = r0; r < r0 + per; ++r) {
-            const uint32_t c = h[nb - 1 - r];
-            if (cum + (int64_t)c >= need) {
-                bc[0] = (uint32_t)(nb - 1 - r);
-                bc[1] = (uint32_t)cum;
-                break;
+    if ((int64_t)ex < need && (int64_t)ex + local >= need) {
+        int64_t cum = ex;
+        uint32_t found = 0, at = 0;
+        bool done = false;
+#pragma unroll
+        for (int i = 0; i < kOwn; ++i) {
+            if (!done && cum + c[i] >= need) {
+                found = (uint32_t)(top - i);
+                at = (uint32_t)cum;
+                done = true;
             }
-            cum += c;
+            cum += c[i];
         }
+        bc[0] = found;
+        bc[1] = at;
     }
     __syncthreads();
     bin = bc[0];
     above = bc[1];
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -250,36 +251,34 @@ sel_collect(const SelArgs a)
     store_hist(h, hv);
     __syncthreads();
     uint32_t b1, above_b1;
-    bin_from_top(h, 4096, w.keff, tmp, bc, b1, above_b1);
+    bin_from_top(h, w.keff, tmp, bc, b1, above_b1);
     if (r == 0 && threadIdx.x == 0)
         a.bin[b] = make_uint2(b1, above_b1);   // every range finds the same b1
 
-    const int lane = threadIdx.x & 31;
-    const unsigned lt = (1u << lane) - 1u;
-    uint32_t mine_above = 0;
-    uint2 *cl = a.cand + w.off;
+    uint32_t mine_above = 0, mine_in = 0;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int64_t i = lo + u * NT + threadIdx.x;
         const bool valid = i < hi;
         const uint32_t bin = kk[u] >> 20;
         mine_above += (valid && bin > b1) ? 1u : 0u;
-        const bool in = valid && bin == b1;
-        const uint32_t bal = __ballot_sync(0xffffffffu, in);
-        if (bal) {
-            const int leader = __ffs(bal) - 1;
-            uint32_t base = 0;
-            if (lane == leader)
-                base = atomicAdd(&a.cand_n[b], (uint32_t)__popc(bal));
-            base = __shfl_sync(0xffffffffu, base, leader);
-            if (in)
-                cl[base + __popc(bal & lt)] = make_uint2(kk[u], (uint32_t)i);
-        }
+        mine_in += (valid && bin == b1) ? 1u : 0u;
     }
+    // one scan of both counts (each total <= 2048, so the low field never carries)
     uint32_t tot;
-    block_excl_scan(mine_above, tmp, tot);
-    if (threadIdx.x == 0)
-        a.above[(size_t)b * a.rps + r] = tot;
+    const uint32_t ex = block_excl_scan((mine_above << 16) | mine_in, tmp, tot);
+    uint2 *cl = a.cand + w.off + (lo - w.s_end);
+    uint32_t pos = ex & 0xffffu;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = lo + u * NT + threadIdx.x;
+        if (i < hi && (kk[u] >> 20) == b1)
+            cl[pos++] = make_uint2(kk[u], (uint32_t)i);
+    }
+    if (threadIdx.x == 0) {
+        a.above[(size_t)b * a.rps + r] = tot >> 16;
+        a.inb1[(size_t)b * a.rps + r] = tot & 0xffffu;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -297,20 +296,21 @@ sel_resolve(const SelArgs a)
     __shared__ unsigned long long s_list[32];
     __shared__ uint32_t s_nlist;
     __shared__ unsigned long long s_T;
+    __shared__ uint32_t s_rstart[kMaxSelectRanges + 1];   // first list index of each range
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.x;
-    // round trip 1: flag, bounds, list length, b1 with the count above it, and
-    // the per-range counts above b1
+    // round trip 1: flag, bounds, b1 with the count above it, and the
+    // per-range counts above and inside b1
     const int32_t re = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
     const int64_t off = __ldcg(a.seq_off + b), end = __ldcg(a.seq_off + b + 1);
-    const uint32_t m = __ldcg(&a.cand_n[b]);
     const uint2 bn = __ldcg(&a.bin[b]);
-    uint32_t ab[kAbovePer];
+    uint32_t ab[kAbovePer], ib[kAbovePer];
 #pragma unroll
     for (int u = 0; u < kAbovePer; ++u) {
         const int r = u * NT + threadIdx.x;
         ab[u] = r < a.rps ? __ldcg(&a.above[(size_t)b * a.rps + r]) : 0u;
+        ib[u] = r < a.rps ? __ldcg(&a.inb1[(size_t)b * a.rps + r]) : 0u;
     }
     if (re != 0)
         return;
@@ -329,8 +329,38 @@ sel_resolve(const SelArgs a)
     uint32_t *gh = a.hist + (size_t)b * 4096;
     for (int i = threadIdx.x; i < 4096; i += NT)
         gh[i] = 0u;                                  // ready for the next call
-    // round trip 2: the b1 candidates
+    // list index of each range's first b1 candidate
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kAbovePer; ++u) {
+        if (u * NT >= nranges)
+            break;
+        const int r = u * NT + threadIdx.x;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan(r < nranges ? ib[u] : 0u, tmp, tot);
+        if (r < nranges)
+            s_rstart[r] = m + ex;
+        m += tot;
+    }
+    if (threadIdx.x == 0) {
+        s_rstart[nranges] = m;
+        s_nlist = 0u;
+    }
+    __syncthreads();
+    // candidate j of the list: range r with s_rstart[r] <= j < s_rstart[r+1]
     const uint2 *cl = a.cand + w.off;
+    auto addr_of = [&](uint32_t j) -> const uint2 * {
+        int lo_r = 0, hi_r = nranges;
+        while (hi_r - lo_r > 1) {
+            const int mid = (lo_r + hi_r) >> 1;
+            if (s_rstart[mid] <= j)
+                lo_r = mid;
+            else
+                hi_r = mid;
+        }
+        return cl + (int64_t)lo_r * kTPC + (j - s_rstart[lo_r]);
+    };
+    // round trip 2: the b1 candidates
     const bool in_smem = m <= (uint32_t)kResolveSmem;
     if (in_smem) {
         constexpr int kBatch = 10;                   // kResolveSmem / NT
@@ -338,20 +368,18 @@ sel_resolve(const SelArgs a)
             uint2 c[kBatch];
 #pragma unroll
             for (int u = 0; u < kBatch; ++u)
-                c[u] = j0 + u * NT < m ? __ldcg(cl + j0 + u * NT) : make_uint2(0u, 0u);
+                c[u] = j0 + u * NT < m ? __ldcg(addr_of(j0 + u * NT)) : make_uint2(0u, 0u);
 #pragma unroll
             for (int u = 0; u < kBatch; ++u)
                 if (j0 + u * NT < m)
                     keys[j0 + u * NT] = make_key(c[u].x, c[u].y);
         }
     }
-    if (threadIdx.x == 0)
-        s_nlist = 0u;
     __syncthreads();
     auto key_at = [&](uint32_t j) -> unsigned long long {
         if (in_smem)
             return keys[j];
-        const uint2 c = __ldcg(cl + j);
+        const uint2 c = __ldcg(addr_of(j));
         return make_key(c.x, c.y);
     };
 
@@ -450,7 +478,6 @@ sel_resolve(const SelArgs a)
     if (threadIdx.x == 0) {
         a.thr[b] = T;
         a.mode[b] = 1;
-        a.cand_n[b] = 0u;                            // ready for the next call
     }
 }
 
@@ -544,7 +571,7 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
     a.count = count;
     a.hist = reinterpret_cast<uint32_t *>(ws + p.off_sel_hist);
     a.cand = reinterpret_cast<uint2 *>(ws + p.off_sel_cand);
-    a.cand_n = reinterpret_cast<uint32_t *>(ws + p.off_sel_cand_n);
+    a.inb1 = reinterpret_cast<uint32_t *>(ws + p.off_sel_inb1);
     a.bin = reinterpret_cast<uint2 *>(ws + p.off_sel_bin);
     a.above = reinterpret_cast<uint32_t *>(ws + p.off_sel_above);
     a.range_off = reinterpret_cast<uint32_t *>(ws + p.off_sel_range_off);

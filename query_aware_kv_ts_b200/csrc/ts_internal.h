@@ -82,7 +82,7 @@ struct Plan {
     int attn_splits;
     // workspace layout (byte offsets)
     size_t off_ctrl, off_chunk_table, off_L, off_partials, off_logits, off_sel_hist, off_sel_cand,
-        off_sel_cand_n, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part,
+        off_sel_inb1, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part,
         total_bytes;
 };
 

@@ -18,7 +18,8 @@
 // Work split: grid (groups / threads, B).  Long sequences: a thread takes 4
 // consecutive tokens aligned to 4 in the logits rows (row stride padded to 4),
 // so each head's logits arrive as one 16-byte load, 8 heads at a time; short
-// sequences: one token per thread, 32 heads loaded at a time, 64-thread blocks.
+// sequences: four lanes per token, each summing every fourth head (the exp
+// chains are latency-bound: more warps per token hide them), then two shuffles.
 // The reuse flag, the sequence bounds and the normalisers L are fetched in one
 // round trip, the logits in the next.
 //
@@ -68,30 +69,35 @@ vote_pass_b(const VoteArgs a)
 {
     __shared__ float s_hi[kMaxHeadsVote], s_lo[kMaxHeadsVote];
     __shared__ uint32_t s_hist[HIST ? 4096 : 1];
+    __shared__ uint16_t s_used[HIST ? 1024 : 1];   // bins this block touched (<= its tokens)
+    __shared__ uint32_t s_nused;
+    __shared__ int64_t s_bounds[2];
+    __shared__ int32_t s_reuse;
     const int tid = threadIdx.x;
     const int nt = blockDim.x;
-    if (HIST)
+    if (HIST) {
         for (int i = tid; i < 4096; i += nt)
             s_hist[i] = 0u;
+        if (tid == 0)
+            s_nused = 0u;
+    }
     pdl_wait();
     pdl_launch_dependents();
     const int b = blockIdx.y;
-    // one round trip: flag, bounds and normalisers (h_q <= 2 * blockDim)
-    const int32_t r = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
-    const int64_t off = __ldcg(a.seq_off + b);
-    const int64_t end = __ldcg(a.seq_off + b + 1);
+    // one round trip: flag, bounds and normalisers (h_q <= 2 * blockDim), each
+    // word loaded by one thread of the block and shared (hundreds of blocks
+    // read the same words)
+    if (tid == 0) {
+        s_reuse = a.reuse != nullptr ? __ldcg(a.reuse + b) : 0;
+        s_bounds[0] = __ldcg(a.seq_off + b);
+        s_bounds[1] = __ldcg(a.seq_off + b + 1);
+    }
     double Lv[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int h = tid + u * nt;
         Lv[u] = h < a.Hq ? __ldcg(a.L + (int64_t)b * a.Hq + h) : 0.0;
     }
-    if (r != 0)
-        return;
-    const int64_t base = off & ~int64_t(TPT - 1);                  // first aligned group of the sequence
-    const int64_t i0 = base + ((int64_t)blockIdx.x * nt + tid) * TPT;
-    if (base + (int64_t)blockIdx.x * nt * TPT >= end)
-        return;   // the whole block is past this sequence
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int h = tid + u * nt;
@@ -102,6 +108,17 @@ vote_pass_b(const VoteArgs a)
         }
     }
     __syncthreads();
+    if (s_reuse != 0)
+        return;
+    const int64_t off = s_bounds[0];
+    const int64_t end = s_bounds[1];
+    // TPT == 4: thread = 4 consecutive tokens; TPT == 1: 4 lanes per token
+    const int tpb = TPT == 1 ? nt / 4 : nt * TPT;                  // tokens per block
+    const int q4 = TPT == 1 ? (tid & 3) : 0;
+    const int64_t base = off & ~int64_t(TPT - 1);                  // first aligned group of the sequence
+    const int64_t i0 = base + (int64_t)blockIdx.x * tpb + (TPT == 1 ? (tid >> 2) : (int64_t)tid * TPT);
+    if (base + (int64_t)blockIdx.x * tpb >= end)
+        return;   // the whole block is past this sequence
     float acc[TPT];
 #pragma unroll
     for (int j = 0; j < TPT; ++j)
@@ -126,18 +143,25 @@ vote_pass_b(const VoteArgs a)
                 }
             }
         } else {
-            for (int h0 = 0; h0 < a.Hq; h0 += 4 * kHeadBatch) {
-                float sv[4 * kHeadBatch];
+            // four lanes per token, each summing every fourth head
+            for (int h0 = q4; h0 < a.Hq; h0 += 4 * kHeadBatch) {
+                float sv[kHeadBatch];
 #pragma unroll
-                for (int u = 0; u < 4 * kHeadBatch; ++u)
-                    if (h0 + u < a.Hq)
-                        sv[u] = __ldcg(a.logits + (int64_t)(h0 + u) * a.ld + i0);
+                for (int u = 0; u < kHeadBatch; ++u)
+                    if (h0 + 4 * u < a.Hq)
+                        sv[u] = __ldcg(a.logits + (int64_t)(h0 + 4 * u) * a.ld + i0);
 #pragma unroll
-                for (int u = 0; u < 4 * kHeadBatch; ++u)
-                    if (h0 + u < a.Hq)
-                        acc[0] += exp_exact_arg(sv[u], s_hi[h0 + u], s_lo[h0 + u]);
+                for (int u = 0; u < kHeadBatch; ++u)
+                    if (h0 + 4 * u < a.Hq)
+                        acc[0] += exp_exact_arg(sv[u], s_hi[h0 + 4 * u], s_lo[h0 + 4 * u]);
             }
         }
+    }
+    if constexpr (TPT == 1) {
+        acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+        acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+    }
+    if (i0 < end && (TPT > 1 || q4 == 0)) {
 #pragma unroll
         for (int j = 0; j < TPT; ++j) {
             const int64_t i = i0 + j;
@@ -158,26 +182,33 @@ vote_pass_b(const VoteArgs a)
 #pragma unroll
         for (int j = 0; j < TPT; ++j) {
             const int64_t li = i0 + j - off;   // sequence-local id
-            const bool cand = i0 < end && li >= s_end && li < l0;
+            const bool cand = i0 < end && li >= s_end && li < l0 && q4 == 0;
             const uint32_t bin = cand ? (__float_as_uint(acc[j]) >> 20) : 0xffffffffu;
-            // one atomic for the warp's first bin, one per lane for the others
+            // one atomic for the warp's first bin, one per lane for the others;
+            // whoever finds a bin empty lists it
             const uint32_t act = __ballot_sync(0xffffffffu, cand);
             if (act) {
                 const int leader = __ffs(act) - 1;
                 const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
                 const uint32_t same = __ballot_sync(0xffffffffu, bin == lb);
+                uint32_t mine = 0xffffffffu;
                 if (lane == leader)
-                    atomicAdd(&s_hist[lb], (uint32_t)__popc(same));
+                    mine = lb;
                 else if (cand && bin != lb)
-                    atomicAdd(&s_hist[bin], 1u);
+                    mine = bin;
+                if (mine != 0xffffffffu) {
+                    const uint32_t add = (lane == leader) ? (uint32_t)__popc(same) : 1u;
+                    if (atomicAdd(&s_hist[mine], add) == 0u)
+                        s_used[atomicAdd(&s_nused, 1u)] = (uint16_t)mine;
+                }
             }
         }
         __syncthreads();
         uint32_t *gh = a.hist + (size_t)b * 4096;
-        for (int i = tid; i < 4096; i += nt) {
-            const uint32_t c = s_hist[i];
-            if (c != 0u)
-                atomicAdd(&gh[i], c);
+        const uint32_t nused = s_nused;
+        for (uint32_t u = tid; u < nused; u += nt) {
+            const uint32_t bin = s_used[u];
+            atomicAdd(&gh[bin], s_hist[bin]);
         }
     }
 }
@@ -203,9 +234,7 @@ cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *re
     a.B = p.B;
     a.Hq = p.Hq;
     // long sequences: 4 tokens per thread (16-byte loads, 256 threads);
-    // short ones: 1 token per thread, in 64-thread blocks so that enough warps
-    // share the latency-bound pass (256 with the histogram, whose per-block
-    // clear and merge cost 4096 bins)
+    // short ones: 64 tokens per 256-thread block, four lanes per token
     if (p.n_total > 262144) {
         const int64_t groups = (p.n_max + 3) / 4 + 1;
         const unsigned gx = (unsigned)((groups + kVoteThreads - 1) / kVoteThreads);
@@ -213,8 +242,8 @@ cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *re
             return launch_ex(vote_pass_b<4, true>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
         return launch_ex(vote_pass_b<4, false>, dim3(gx, (unsigned)p.B), dim3(kVoteThreads), 0, st, 1, a);
     }
-    const int nt = a.hist != nullptr ? kVoteThreads : 64;
-    const unsigned gx = (unsigned)((p.n_max + nt) / nt);
+    const int nt = kVoteThreads;                 // 64 tokens x 4 lanes
+    const unsigned gx = (unsigned)((p.n_max + nt / 4) / (nt / 4));
     if (a.hist != nullptr)
         return launch_ex(vote_pass_b<1, true>, dim3(gx, (unsigned)p.B), dim3(nt), 0, st, 1, a);
     return launch_ex(vote_pass_b<1, false>, dim3(gx, (unsigned)p.B), dim3(nt), 0, st, 1, a);
