@@ -127,7 +127,7 @@ TS_API ts_status_t ts_selcache(const void *q, void *q_prev, int32_t *reuse, doub
  *   votes[seq_offsets[b] + i] = sum_h exp(s[h,i] - L[b,h])
  * so the votes of a sequence sum to h_q.  Sequences with reuse[b] != 0 are
  * skipped (their votes are left as they were).
- *   q          device bf16 [batch, h_q, head_dim] contiguous
+ *   q          device bf16 [batch, h_q, head_dim] contiguous, 16-byte aligned
  *   reuse      device int32 [batch] or NULL (NULL: score every sequence)
  *   votes      device float32 [seq_offsets[batch]], written
  * The float32 votes carry a relative error of a few 1e-7.

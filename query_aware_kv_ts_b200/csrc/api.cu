@@ -166,8 +166,8 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->n_max = n_max;
     p->scale = kv->scale != 0.0f ? kv->scale : (float)(1.0 / sqrt((double)D));
     p->sms = sms;
-    p->tile_tokens = (kStageBytesTarget / 2) / (kv->h_kv * D);
-    p->stage_bytes = p->tile_tokens * kv->h_kv * D * 2;
+    p->tile_tokens = kScoreRows / kv->h_kv;          // one stage = 128 K rows (h_kv heads x T tokens)
+    p->stage_bytes = kScoreRows * D * 2;
     int64_t chunks = 0;
     for (int b = 0; b < kv->batch; ++b) {
         const int64_t n = off[b + 1] - off[b];
@@ -176,6 +176,12 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->max_chunks = chunks;
     const int grid_cap = sms < 256 ? sms : 256;
     p->score_grid = (int)(chunks < grid_cap ? chunks : grid_cap);
+    {
+        // two stage parities x the lane quarters (32 rows each) one kv head's
+        // T = 128 / h_kv rows span
+        const int qph = p->tile_tokens > 32 ? p->tile_tokens / 32 : 1;
+        p->score_partials_per_slot = 2 * qph;
+    }
     p->ld_logits = (n_total + 3) / 4 * 4;
     p->sel_ranges = (int)((n_max + kSelectTokensPerCta - 1) / kSelectTokensPerCta) + 1;
     p->capacity = capacity;
@@ -198,7 +204,8 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->off_L = o;
     o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
     p->off_partials = o;
-    o = align_up(o + sizeof(float) * 2 * (size_t)(p->score_grid + p->B) * p->Hq, 256);
+    o = align_up(o + sizeof(float) * 2 * (size_t)(p->score_grid + p->B) * p->score_partials_per_slot * p->Hq,
+                 256);
     p->off_sel_inb1 = o;
     o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
     p->off_sel_bin = o;
@@ -338,8 +345,8 @@ ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reu
     ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
     if (s != TS_OK)
         return s;
-    if (q == nullptr || (reinterpret_cast<uintptr_t>(q) & 3u)) {
-        set_error("q is required and must be 4-byte aligned");
+    if (q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15u)) {
+        set_error("q is required and must be 16-byte aligned");
         return TS_ERR_INVALID_ARG;
     }
     if (p.n_total == 0)
@@ -348,7 +355,7 @@ ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reu
     s = encode_kmap(p, kv, &kmap);
     if (s != TS_OK)
         return s;
-    cudaError_t e = launch_score(p, kmap, q, kv->seq_offsets_dev, reuse, static_cast<uint8_t *>(ws),
+    cudaError_t e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, static_cast<uint8_t *>(ws),
                                  static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass A launch");
 }
@@ -501,7 +508,7 @@ ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32
     if (e != cudaSuccess)
         return cuda_fail(e, "ts_decode_step: selection cache launch");
     if (p.n_total > 0) {
-        e = launch_score(p, kmap, q, kv->seq_offsets_dev, reuse, w, st);
+        e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, st);
         if (e != cudaSuccess)
             return cuda_fail(e, "ts_decode_step: score pass A launch");
         const SelectWindow win = {k, n_sink, n_local};

@@ -10,27 +10,38 @@
 //
 // Design (B200):
 //  * One CTA per SM, persistent.  The active sequences' tokens are cut into
-//    chunks of T tokens (one pipeline stage, 32 KB of K); CTA j takes the
-//    contiguous, balanced chunk range [j*C/grid, (j+1)*C/grid), so a CTA
-//    spans one or two sequences and the load is balanced to one chunk.
-//  * A producer warp streams K with 3-D TMA boxes {64 channels, T tokens,
-//    h_kv heads} (128-byte swizzle, L2 evict-first) into a 6-stage ring of
-//    32 KB stages guarded by mbarriers.  Before waiting for the previous
-//    kernel in the stream it already asks L2 for its first tiles, so the
-//    first DRAM round trip overlaps that kernel.
-//  * Eight consumer warps each own one KV head g and a share of the 16-token
-//    row blocks of a stage.  The G query heads of g are the N dimension of a
-//    bf16 m16n8k16 tensor-core tile (N = 8 covers G <= 8; two tiles for
-//    G <= 16), K rows the M dimension, the head dimension K: the Q fragments
-//    live in registers; K fragments come from shared memory with ldmatrix
-//    (conflict-free thanks to the swizzle).
-//  * The epilogue scales, stores the logits and keeps an online
-//    (max, sum exp) per head and thread over the CTA's chunks of a sequence;
-//    when the CTA leaves the sequence these are reduced over the CTA and
-//    written as one partial of head h at slot j + b (CTA j, sequence b).  The
-//    slot is unique: along the chunk order neither j nor b decreases and one
-//    of them grows at every new (CTA, sequence) segment.  No fences, atomics
-//    or waits on other CTAs.
+//    chunks of T = 128 / h_kv tokens, so that a chunk holds 128 K rows (h_kv
+//    heads x T tokens, one pipeline stage); CTA j takes the contiguous,
+//    balanced chunk range [j*C/grid, (j+1)*C/grid).
+//  * Warp 8 streams K with 3-D TMA boxes {64 channels, T tokens, h_kv heads}
+//    (128-byte swizzle, L2 evict-first) into a ring of stages guarded by
+//    mbarriers.  Before waiting for the previous kernel in the stream it
+//    already asks L2 for its first tiles.
+//  * Warp 9 owns the tensor cores: it allocates TMEM, writes the sequence's
+//    queries into shared memory in the same swizzled K-major layout (row
+//    g*GP + j = query head g*G + j, rows j >= G zero; GP = 4, 8 or 16), and one
+//    lane issues, per stage, the tcgen05.mma chain
+//        D[128 x N] = Kstage[128 x d] . Q[N x d]^T,   N = h_kv * GP,
+//    d/16 instructions of K = 16 into one of four TMEM accumulators, then
+//    commits to the stage's "empty" barrier (the ring slot is free once the
+//    MMAs have read it) and to the accumulator's "full" barrier.  Row g*T + t
+//    of D holds token t's logits against every query head; the columns
+//    g*GP .. g*GP+G-1 are the ones of its own group.
+//  * Warps 0-7 are the epilogue: thread i of warps w and w+4 owns TMEM lane
+//    32w + i, i.e. one (kv head, token) row; warp w takes the even stages and
+//    warp w+4 the odd ones (two warps per TMEM lane quarter hide the load and
+//    exp latencies for any group size).  A thread loads its group's G
+//    columns with tcgen05.ld, frees the accumulator, scales, stores the
+//    logits (a warp writes 32 consecutive tokens of a head: coalesced) and
+//    keeps an online (max, sum exp) per head; when the CTA leaves a sequence
+//    each warp reduces these over its lanes and writes them as its own
+//    partial of each head (R per (CTA, sequence) segment), with no barrier;
+//    they are
+//    reduced over the threads of each head and written as one partial of
+//    head h at slot j + b (CTA j, sequence b).  The slot is unique: along the
+//    chunk order neither j nor b decreases and one of them grows at every new
+//    (CTA, sequence) segment.  No fences, atomics or waits on other CTAs;
+//    every wait on a barrier is bounded.
 //  * score_merge (one warp per sequence and head) folds the partials of
 //    CTAs j0..j1, the CTAs that cover the sequence, into L[b, h]: fp32 terms
 //    exp(m - M) <= 1 summed in float64.
@@ -41,7 +52,9 @@ namespace ts {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kPrefetchTiles = kScoreStages;
+constexpr int kMaxPrefetchTiles = 6;
+constexpr int kProducerWarp = kScoreEpiWarps;       // 8
+constexpr int kMmaWarp = kScoreEpiWarps + 1;        // 9
 
 struct ScoreArgs {
     const __nv_bfloat16 *q;   // [B, Hq, D]
@@ -49,22 +62,29 @@ struct ScoreArgs {
     const int32_t *reuse;     // [B] or null
     float *logits;            // [Hq][ld]
     int64_t ld;
-    float2 *partials;         // [Hq][S] (max, sum exp(x - max)) at slot CTA + sequence
-    int S;                    // slots per head: grid + B
+    float2 *partials;         // [Hq][S][R] (max, sum exp(x - max)) at slot CTA + sequence, entry per warp
+    int S;                    // segment slots per head: grid + B
+    int R;                    // partials per segment slot: epilogue warps that see one head
     int32_t *chunk_table;     // [B + 1] first active chunk of each sequence (for score_merge)
     uint32_t *ctrl;           // status word
     int B, Hq, Hkv, G;
     int T;                    // tokens per chunk / stage
     int stage_bytes;
+    int nstages;              // ring depth
+    int64_t pf_off[33];       // B <= 32: the host copy of the offsets, for the prefetch hints only
+    uint32_t tmem_cols;       // TMEM columns allocated (power of 2 >= 4 * N)
     float scale;
 };
 
 struct __align__(16) ScoreShared {
-    uint64_t full[kScoreStages];
-    uint64_t empty[kScoreStages];
+    uint64_t full[kScoreMaxStages];
+    uint64_t empty[kScoreMaxStages];
+    uint64_t acc_full[kScoreAccBufs];
+    uint64_t acc_empty[kScoreAccBufs];
+    uint64_t mma_done;        // every MMA issued so far has completed
     int64_t off[kMaxBatch + 1];
     int32_t chunk_start[kMaxBatch + 1];
-    float2 red[kScoreConsumerWarps][16];
+    uint32_t tmem_base;
     int32_t pf_start[32];     // all-active chunk table of the prefetch hints (B <= 32)
     int64_t pf_off[32];       // and the sequence offsets it was built from
 };
@@ -119,6 +139,15 @@ __device__ __forceinline__ void build_chunk_table(ScoreShared &sh, const int32_t
     __syncthreads();
 }
 
+// floor(j * total / grid) for j <= grid <= 256 and total < 2^31: a double
+// quotient is exact enough (a non-integer quotient is at least 1/grid away
+// from an integer, far above the rounding error) and much cheaper than a
+// 64-bit integer division.
+__device__ __forceinline__ int32_t chunk_split(uint32_t j, int32_t total, uint32_t grid)
+{
+    return (int32_t)floor((double)j * (double)total / (double)grid);
+}
+
 // B <= 32: lane b < B computes c0 = first chunk of sequence b and c1 = one past
 // its last (sequences with reuse set, when reuse is given, have no chunks),
 // with one round trip for the offsets and flags and a warp scan.
@@ -145,37 +174,152 @@ __device__ __forceinline__ void warp_chunk_scan(const int64_t *seq_off, const in
     c1 = incl;
 }
 
-template <int D, int NB>
+// The queries of sequence b as the UMMA B operand: N = h_kv*GP rows of d
+// channels, bf16, K-major with the 128-byte swizzle (64-channel halves of
+// N * 128 bytes).  Whole warp.
+// MMA N: one GP-row block per kv head, at least 16 (the M = 128 shapes need
+// N to be a multiple of 16).
+template <int GP>
+__host__ __device__ constexpr int score_mma_n(int Hkv)
+{
+    return Hkv * GP < 16 ? 16 : Hkv * GP;
+}
+
+template <int D, int GP>
+__device__ __forceinline__ void stage_queries(uint8_t *qs, const __nv_bfloat16 *qb, int G, int Hkv, int lane)
+{
+    const int N = score_mma_n<GP>(Hkv);
+    constexpr int kChunks = D / 8;           // 16-byte chunks per row
+    constexpr int kBatch = 8;
+    for (int c0 = lane; c0 < N * kChunks; c0 += 32 * kBatch) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int c = c0 + u * 32;
+            const int n = c / kChunks, cc = c - n * kChunks;
+            const int g = n / GP, j = n - g * GP;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (c < N * kChunks && g < Hkv && j < G)   // rows past the last head stay zero
+                v[u] = __ldg(reinterpret_cast<const uint4 *>(qb + (int64_t)(g * G + j) * D) + cc);
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int c = c0 + u * 32;
+            if (c < N * kChunks) {
+                const int n = c / kChunks, cc = c - n * kChunks;
+                const int half = cc >> 3, ci = cc & 7;
+                *reinterpret_cast<uint4 *>(qs + (size_t)half * N * 128 + n * 128 + ((ci ^ (n & 7)) << 4)) = v[u];
+            }
+        }
+    }
+}
+
+// Order-preserving map of a float to a signed integer (and back), for the
+// integer warp max reduction.
+__device__ __forceinline__ int32_t float_order_key(float x)
+{
+    const int32_t b = __float_as_int(x);
+    return b >= 0 ? b : (b ^ 0x7fffffff);
+}
+__device__ __forceinline__ float float_from_order_key(int32_t k)
+{
+    return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff));
+}
+
+// End of a (CTA, sequence) segment in the epilogue: reduce each head's
+// (max, sum exp) over the lanes of this warp that hold it (one integer max
+// reduction, one exp2 per lane, a fixed shuffle tree of adds: deterministic)
+// and write it as this warp's partial of the head.  A (CTA, sequence) segment
+// owns R partial slots per head, one per epilogue warp that sees the head
+// (two stage parities x the lane quarters the head spans); score_merge folds
+// them.  No barrier: the warps of the CTA never wait for each other here.
+// (m, z) are consumed: on return they hold the warp's (max, sum) per head.
+template <int GP>
+__device__ __forceinline__ void score_flush(float (&m)[GP], float (&z)[GP], int G, int T, int span, int lane,
+                                            int warp, int g, float2 *partials, int64_t stride, int64_t slot_base)
+{
+    const int quarter = warp & 3, hs = warp >> 2;
+    const int qph = T > 32 ? T / 32 : 1;   // lane quarters per head
+    const uint32_t grp = span == 32 ? 0xffffffffu : (lane < 16 ? 0x0000ffffu : 0xffff0000u);
+#pragma unroll
+    for (int j = 0; j < GP; ++j) {
+        const float M = float_from_order_key(__reduce_max_sync(grp, float_order_key(m[j])));
+        z[j] = (m[j] == -INFINITY) ? 0.0f : z[j] * exp2f((m[j] - M) * kLog2e);
+        m[j] = M;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        if (o < span) {
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+                z[j] += __shfl_xor_sync(0xffffffffu, z[j], o);
+        }
+    if ((lane % span) == 0) {
+        const int r = hs * qph + (quarter % qph);
+#pragma unroll
+        for (int j = 0; j < GP; ++j)
+            if (j < G)
+                partials[(int64_t)(g * G + j) * stride + slot_base + r] = make_float2(m[j], z[j]);
+    }
+}
+
+template <int D, int GP>
 __global__ void __launch_bounds__(kScoreThreads, 1)
-score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
+score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ ScoreArgs a)
 {
     extern __shared__ uint8_t dyn_smem[];
     __shared__ ScoreShared sh;
     uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    const int NS = a.nstages;
+    uint8_t *qs = stages + (size_t)NS * a.stage_bytes;      // 1024-byte aligned: stages are multiples of 16 KB
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int B = a.B;
     const int T = a.T;
+    const int Hkv = a.Hkv;
+    const int N = score_mma_n<GP>(Hkv);
 
     if (tid == 0) {
-        for (int s = 0; s < kScoreStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&sh.full[s], 1);
-            mbar_init(&sh.empty[s], kScoreConsumerWarps);
+            mbar_init(&sh.empty[s], 1);
         }
+        for (int s = 0; s < kScoreAccBufs; ++s) {
+            mbar_init(&sh.acc_full[s], 1);
+            mbar_init(&sh.acc_empty[s], kScoreEpiWarps / 2);   // the four warps of that stage parity
+        }
+        mbar_init(&sh.mma_done, 1);
         mbar_fence_init();
     }
+    if (warp == kMmaWarp)
+        tmem_alloc(&sh.tmem_base, a.tmem_cols);
     // ---- before the previous kernel has finished: only L2 prefetch hints,
     //      computed as if every sequence were active (a wrong guess costs
     //      nothing but bandwidth; the data itself is read after the wait) -----
+    const int npf = NS < kMaxPrefetchTiles ? NS : kMaxPrefetchTiles;
     if (B <= 32) {
-        if (warp == kScoreConsumerWarps) {
+        if (warp == kProducerWarp) {
             if (lane == 0)
                 tma_prefetch_desc(&kmap);
-            int32_t c0, c1;
-            int64_t o0, o1;
-            warp_chunk_scan(a.seq_off, nullptr, B, T, lane, c0, c1, o0, o1);
+            // all-active chunk table from the host offsets (kernel parameters:
+            // no memory round trip before the wait)
+            int32_t x = 0;
+            int64_t o0 = 0;
+            if (lane < B) {
+                o0 = a.pf_off[lane];
+                const int64_t n = a.pf_off[lane + 1] - o0;
+                x = n > 0 ? (int32_t)((n + T - 1) / T) : 0;
+            }
+            int32_t c1 = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, c1, o);
+                if (lane >= o)
+                    c1 += y;
+            }
+            const int32_t c0 = c1 - x;
             if (lane < B) {
                 sh.pf_start[lane] = c0;
                 sh.pf_off[lane] = o0;
@@ -183,10 +327,10 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             const int32_t total = __shfl_sync(0xffffffffu, c1, B - 1);
             __syncwarp();
             if (lane == 0) {
-                const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
-                const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
+                const int32_t v0 = chunk_split(blockIdx.x, total, gridDim.x);
+                const int32_t v1 = chunk_split(blockIdx.x + 1, total, gridDim.x);
                 int b = 0;
-                for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
+                for (int32_t v = v0; v < v1 && v < v0 + npf; ++v) {
                     while (b + 1 < B && sh.pf_start[b + 1] <= v)
                         ++b;
                     const int64_t t0 = sh.pf_off[b] + (int64_t)(v - sh.pf_start[b]) * T;
@@ -201,12 +345,12 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
             sh.off[b] = __ldcg(a.seq_off + b);
         __syncthreads();
         build_chunk_table(sh, a.reuse, B, T, warp, lane, false);
-        if (warp == kScoreConsumerWarps && lane == 0) {
+        if (warp == kProducerWarp && lane == 0) {
             tma_prefetch_desc(&kmap);
             const int32_t total = sh.chunk_start[B];
-            const int32_t v0 = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
-            const int32_t v1 = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
-            for (int32_t v = v0; v < v1 && v < v0 + kPrefetchTiles; ++v) {
+            const int32_t v0 = chunk_split(blockIdx.x, total, gridDim.x);
+            const int32_t v1 = chunk_split(blockIdx.x + 1, total, gridDim.x);
+            for (int32_t v = v0; v < v1 && v < v0 + npf; ++v) {
                 const int b = upper_seq(sh.chunk_start, B, v);
                 const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
 #pragma unroll
@@ -221,6 +365,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
     // ---- the real chunk table (reuse flags come from the previous kernel);
     //      the offsets are re-read too, in case a caller's kernel wrote them;
     //      offsets and flags are loaded together: one round trip -------------
+    tmem_fence_before();
     if (B <= 32) {
         if (warp == 0) {
             int32_t c0, c1;
@@ -268,29 +413,30 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
         }
         __syncthreads();
     }
+    tmem_fence_after();
     if (blockIdx.x == 0)
         for (int b = tid; b <= B; b += blockDim.x)
             a.chunk_table[b] = sh.chunk_start[b];
     const int32_t total = sh.chunk_start[B];
-    const int32_t v_begin = (int32_t)((int64_t)blockIdx.x * total / gridDim.x);
-    const int32_t v_end = (int32_t)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
-    const int Hkv = a.Hkv;
-    const int half_bytes = T * Hkv * 128;   // one 64-channel box
+    const int32_t v_begin = chunk_split(blockIdx.x, total, gridDim.x);
+    const int32_t v_end = chunk_split(blockIdx.x + 1, total, gridDim.x);
+    const uint32_t tmem = sh.tmem_base;
+    const int half_bytes = kScoreRows * 128;   // one 64-channel box
 
-    if (warp == kScoreConsumerWarps) {
-        // ================= producer: one elected lane issues TMA ==========
+    if (warp == kProducerWarp) {
+        // ================= TMA producer: one elected lane ==================
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
             for (int32_t v = v_begin; v < v_end; ++v, ++it) {
                 const int b = upper_seq(sh.chunk_start, B, v);
                 const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
-                const int s = it % kScoreStages;
-                if (it >= kScoreStages) {
-                    const uint32_t par = ((it / kScoreStages) - 1) & 1;
+                const int s = it % NS;
+                if (it >= (uint32_t)NS) {
+                    const uint32_t par = ((it / NS) - 1) & 1;
                     if (!mbar_wait_bounded(&sh.empty[s], par, kSpinLimit)) {
                         report_timeout(a.ctrl, kSiteScoreEmpty);
-                        break;   // nothing issued after this: the consumers time out on full[] too
+                        break;   // nothing issued after this: the MMA warp times out on full[] too
                     }
                 }
                 mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
@@ -300,149 +446,160 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a)
                                 (int32_t)t0, 0, pol);
             }
         }
-        return;
+        return;   // takes no part in the final barrier
     }
 
-    // ===================== consumers (warps 0..7) =========================
-    const int ctid = tid;                       // 0..255
-    const int g = warp % Hkv;
-    const int wsub = warp / Hkv;
-    const int nsub = kScoreConsumerWarps / Hkv;
-    const int mblocks = T / 16;
-    const int G = a.G;
-    const int r0 = lane >> 2;
-    const int c0 = (lane & 3) * 2;
-    const float scale = a.scale;
-
-    uint32_t bq[D / 16][NB][2];
-    float m[NB][2], z[NB][2];
-    int cur_b = -1;
-    uint32_t it = 0;
-    bool dead = false;
-
-    // Close this CTA's run of chunks of a sequence: reduce (max, sum) per head
-    // over the CTA and publish one partial per head at slot blockIdx.x + cur_b.
-    auto flush_segment = [&]() {
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    const float m2 = __shfl_xor_sync(0xffffffffu, m[nb][cc], o);
-                    const float z2 = __shfl_xor_sync(0xffffffffu, z[nb][cc], o);
-                    lse_merge(m[nb][cc], z[nb][cc], m2, z2);
+    if (warp == kMmaWarp) {
+        // ================= tensor cores: queries, MMA chain ===============
+        constexpr uint32_t kIdescM = 128;
+        const uint32_t idesc = umma_idesc_bf16_f32(kIdescM, N);
+        int cur_b = -1;
+        bool dead = false;
+        uint32_t done_par = 0;
+        uint32_t it = 0;
+        for (int32_t v = v_begin; v < v_end && !dead; ++v, ++it) {
+            const int b = upper_seq(sh.chunk_start, B, v);
+            if (b != cur_b) {
+                if (cur_b >= 0) {   // the old queries may still be read by MMAs in flight
+                    if (lane == 0)
+                        umma_commit(&sh.mma_done);
+                    __syncwarp();
+                    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.mma_done, done_par, kSpinLimit));
+                    done_par ^= 1u;
+                    if (!ok) {
+                        if (lane == 0)
+                            report_timeout(a.ctrl, kSiteScoreMma);
+                        dead = true;
+                        break;
+                    }
                 }
-                if (lane < 4)
-                    sh.red[warp][nb * 8 + c0 + cc] = make_float2(m[nb][cc], z[nb][cc]);
+                stage_queries<D, GP>(qs, a.q + (int64_t)b * a.Hq * D, a.G, Hkv, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                cur_b = b;
             }
-        named_bar_sync(1, kScoreConsumerWarps * 32);
-        for (int h = ctid; h < a.Hq; h += kScoreConsumerWarps * 32) {
-            const int gh = h / G, j = h - gh * G;
-            float M = -INFINITY, Z = 0.0f;
-            for (int w2 = gh; w2 < kScoreConsumerWarps; w2 += Hkv)
-                lse_merge(M, Z, sh.red[w2][j].x, sh.red[w2][j].y);
-            a.partials[(int64_t)h * a.S + blockIdx.x + cur_b] = make_float2(M, Z);
+            const int s = it % NS;
+            const uint32_t par = (it / NS) & 1;
+            const int buf = it % kScoreAccBufs;
+            bool ok = true;
+            if (lane == 0) {
+                ok = mbar_wait_bounded(&sh.full[s], par, kSpinLimit);
+                if (ok && it >= (uint32_t)kScoreAccBufs)
+                    ok = mbar_wait_bounded(&sh.acc_empty[buf], ((it / kScoreAccBufs) - 1) & 1, kSpinLimit);
+                if (ok) {
+                    tmem_fence_after();
+                    const uint32_t a_base = smem_u32(stages + (size_t)s * a.stage_bytes);
+                    const uint32_t b_base = smem_u32(qs);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t koff = (uint32_t)((ks & 3) * 32);
+                        const uint64_t ad = umma_desc_sw128(a_base + (uint32_t)((ks >> 2) * half_bytes) + koff);
+                        const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)((ks >> 2) * N * 128) + koff);
+                        umma_bf16(tmem + (uint32_t)(buf * N), ad, bd, idesc, ks > 0);
+                    }
+                    umma_commit(&sh.empty[s]);        // the ring slot is free once these MMAs have read it
+                    umma_commit(&sh.acc_full[buf]);   // the accumulator is ready for the epilogue
+                } else {
+                    report_timeout(a.ctrl, kSiteScoreMma);
+                }
+            }
+            dead = !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
+            __syncwarp();
         }
-        named_bar_sync(1, kScoreConsumerWarps * 32);   // sh.red is rewritten by the next flush
-    };
+        // every MMA this warp issued has completed before TMEM is released
+        if (it > 0) {
+            if (lane == 0)
+                umma_commit(&sh.mma_done);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&sh.mma_done, done_par, kSpinLimit)) && lane == 0)
+                report_timeout(a.ctrl, kSiteScoreMma);
+        }
+    } else {
+        // ================= epilogue: warps 0-3, one TMEM lane each =========
+        const int quarter = warp & 3, hs = warp >> 2;
+        const int r = quarter * 32 + lane;         // accumulator row
+        const int g = r / T, t = r - g * T;        // kv head, token within the chunk
+        const int g_lo = (quarter * 32) / T;       // first kv head of this warp's rows
+        const int span = T < 32 ? T : 32;          // lanes of this warp with the same head
+        const int G = a.G;
+        const float scale = a.scale;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        float m[GP], z[GP];
+        int cur_b = -1;
+        bool dead = false;
+        uint32_t it = 0;
 
-    for (int32_t v = v_begin; v < v_end; ++v, ++it) {
-        const int b = upper_seq(sh.chunk_start, B, v);
-        const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
-        const int64_t hi = sh.off[b + 1];
+        auto flush_segment = [&]() {
+            score_flush<GP>(m, z, G, T, span, lane, warp, g, a.partials, (int64_t)a.S * a.R,
+                            ((int64_t)blockIdx.x + cur_b) * a.R);
+        };
 
-        if (b != cur_b) {
-            if (cur_b >= 0)
-                flush_segment();
-            cur_b = b;
+        for (int32_t v = v_begin; v < v_end; ++v, ++it) {
+            const int b = upper_seq(sh.chunk_start, B, v);
+            if (b != cur_b) {
+                if (cur_b >= 0)
+                    flush_segment();
+                cur_b = b;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
+                for (int j = 0; j < GP; ++j) {
+                    m[j] = -INFINITY;
+                    z[j] = 0.0f;
+                }
+            }
+            if (dead || (int)(it & 1u) != hs)
+                continue;                          // the other warp of this lane quarter takes it
+            const int buf = it % kScoreAccBufs;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&sh.acc_full[buf], (it / kScoreAccBufs) & 1, kSpinLimit))) {
+                if (lane == 0)
+                    report_timeout(a.ctrl, kSiteScoreAcc);
+                dead = true;
+                continue;
+            }
+            tmem_fence_after();
+            uint32_t raw[GP], raw2[GP];
+            const uint32_t taddr = lane_base + (uint32_t)(buf * N + g_lo * GP);
+            tmem_ld_32x32b<GP>(taddr, raw);
+            if (T < 32)
+                tmem_ld_32x32b<GP>(taddr + GP, raw2);   // h_kv = 8: two heads per lane quarter
+            tmem_wait_ld();
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sh.acc_empty[buf]);
+            const bool second = g != g_lo;           // only with two heads per lane quarter
+            const int64_t tok = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T + t;
+            if (tok < sh.off[b + 1]) {
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int j = nb * 8 + r0;
+                for (int j = 0; j < GP; ++j) {
                     if (j < G) {
-                        const uint32_t *qp = reinterpret_cast<const uint32_t *>(
-                            a.q + ((int64_t)b * a.Hq + g * G + j) * D + ks * 16 + c0);
-                        bq[ks][nb][0] = __ldg(qp);
-                        bq[ks][nb][1] = __ldg(qp + 4);
-                    } else {
-                        bq[ks][nb][0] = 0u;
-                        bq[ks][nb][1] = 0u;
-                    }
-                }
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    m[nb][cc] = -INFINITY;
-                    z[nb][cc] = 0.0f;
-                }
-        }
-
-        const int s = it % kScoreStages;
-        const uint32_t par = (it / kScoreStages) & 1;
-        if (!dead && !mbar_wait_bounded(&sh.full[s], par, kSpinLimit)) {
-            report_timeout(a.ctrl, kSiteScoreFull);
-            dead = true;
-        }
-        if (!dead) {
-            const uint32_t stage_base = smem_u32(stages + (size_t)s * a.stage_bytes);
-            for (int mb = wsub; mb < mblocks; mb += nsub) {
-                float acc[NB][4];
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        acc[nb][e] = 0.0f;
-                const int trow = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t row_addr = stage_base + (uint32_t)((g * T + trow) * 128);
-                const int swz = trow & 7;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const int chunk = (ks & 3) * 2 + (lane >> 4);
-                    const uint32_t addr =
-                        row_addr + (uint32_t)((ks >> 2) * half_bytes) + (uint32_t)((chunk ^ swz) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(a0, a1, a2, a3, addr);
-#pragma unroll
-                    for (int nb = 0; nb < NB; ++nb)
-                        mma_16816(acc[nb], a0, a1, a2, a3, bq[ks][nb][0], bq[ks][nb][1]);
-                }
-                // epilogue: rows r0 and r0 + 8 of this block, columns c0, c0 + 1
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int64_t tok = t0 + mb * 16 + r0 + rr * 8;
-                    if (tok < hi) {
-#pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                            for (int cc = 0; cc < 2; ++cc) {
-                                const int j = nb * 8 + c0 + cc;
-                                if (j < G) {
-                                    const float x = acc[nb][rr * 2 + cc] * scale;
-                                    a.logits[(int64_t)(g * G + j) * a.ld + tok] = x;
-                                    online_push(m[nb][cc], z[nb][cc], x);
-                                }
-                            }
+                        const float x = __uint_as_float(second ? raw2[j] : raw[j]) * scale;
+                        a.logits[(int64_t)(g * G + j) * a.ld + tok] = x;
+                        online_push(m[j], z[j], x);
                     }
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sh.empty[s]);
+        if (cur_b >= 0)
+            flush_segment();
     }
-    if (cur_b >= 0)
-        flush_segment();
+    // epilogue and MMA warps: every accumulator has been read and every MMA
+    // has completed before the MMA warp frees TMEM
+    tmem_fence_before();
+    named_bar_sync(2, (kScoreEpiWarps + 1) * 32);
+    tmem_fence_after();
+    if (warp == kMmaWarp)
+        tmem_dealloc(tmem, a.tmem_cols);
 }
 
 // L[b, h] from the partials of sequence b (one warp per sequence and head).
-// CTA j of pass A covers chunks [j*total/grid, (j+1)*total/grid); the CTAs that
-// cover the sequence's chunks [cs, ce) are j0 = owner(cs) .. j1 = owner(ce-1),
-// owner(v) = ((v+1)*grid - 1) / total, and CTA j wrote at slot j + b.  The
-// table entries and every slot the sequence could own are loaded together (one
-// round trip); slots outside j0..j1, or of CTAs without chunks, are dropped.
+// CTA j of pass A covers chunks [j*total/grid, (j+1)*total/grid); the CTAs
+// that cover the sequence's chunks [cs, ce) are j0 = owner(cs) ..
+// j1 = owner(ce-1), owner(v) = ((v+1)*grid - 1) / total, and CTA j wrote the
+// R partials of its segment at slot j + b.  The table entries and every
+// partial the sequence could own are loaded together (one round trip);
+// entries of CTAs outside j0..j1, or without chunks, are dropped.  fp32
+// terms exp(m - M) <= 1 summed in float64 in a fixed order.
+template <int R>
 __global__ void __launch_bounds__(32)
 score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L, int B, int Hq, int grid_a)
 {
@@ -450,14 +607,15 @@ score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L
     pdl_launch_dependents();
     const int h = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x;
-    constexpr int kPer = 8;   // grid_a <= 256
+    constexpr int kPer = 8 * R;   // grid_a * R <= 256 * R entries over 32 lanes
+    const int n = grid_a * R;
     const int32_t cs = __ldcg(chunk_table + b), ce = __ldcg(chunk_table + b + 1), total = __ldcg(chunk_table + B);
-    const float2 *row = partials + (int64_t)h * S + b;
+    const float2 *row = partials + ((int64_t)h * S + b) * R;
     float2 pv[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-        const int j = lane + 32 * i;
-        pv[i] = j < grid_a ? __ldcg(row + j) : make_float2(-INFINITY, 0.0f);
+        const int e = lane + 32 * i;
+        pv[i] = e < n ? __ldcg(row + e) : make_float2(-INFINITY, 0.0f);
     }
     if (cs == ce)
         return;   // reused or empty sequence: its L is not needed
@@ -465,10 +623,11 @@ score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L
     const int j1 = (int)(((int64_t)ce * grid_a - 1) / total);
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-        const int j = lane + 32 * i;
-        bool keep = j >= j0 && j <= j1;
+        const int e = lane + 32 * i;
+        const int j = e / R;   // R is a power of 2: a shift
+        bool keep = e < n && j >= j0 && j <= j1;
         if (keep && total < grid_a)   // some CTAs had no chunks and wrote nothing
-            keep = (int64_t)j * total / grid_a < (int64_t)(j + 1) * total / grid_a;
+            keep = chunk_split(j, total, grid_a) < chunk_split(j + 1, total, grid_a);
         if (!keep)
             pv[i] = make_float2(-INFINITY, 0.0f);
     }
@@ -491,30 +650,41 @@ score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L
         L[(int64_t)b * Hq + h] = (double)M + log(Z);
 }
 
-template <int D, int NB>
-cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, const ScoreArgs &args, cudaStream_t st)
+template <int D, int GP>
+cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, ScoreArgs args, cudaStream_t st)
 {
-    const size_t dyn = (size_t)kScoreStages * p.stage_bytes + 1024;
+    const int N = score_mma_n<GP>(p.Hkv);
+    const size_t q_bytes = (size_t)N * D * 2;
+    int ns = (int)((kScoreDynSmemBudget - q_bytes) / (size_t)p.stage_bytes);
+    ns = ns < kScoreMaxStages ? ns : kScoreMaxStages;
+    args.nstages = ns;
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(kScoreAccBufs * N))
+        cols <<= 1;
+    args.tmem_cols = cols;
+    const size_t dyn = (size_t)ns * p.stage_bytes + q_bytes + 1024;
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(score_pass_a<D, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)dyn);
+        cudaError_t e = cudaFuncSetAttribute(score_pass_a<D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(kScoreDynSmemBudget + 1024));
         if (e != cudaSuccess)
             return e;
         configured_dev = dev;
     }
-    return launch_ex(score_pass_a<D, NB>, dim3((unsigned)p.score_grid), dim3(kScoreThreads), dyn, st, 1, kmap,
+    return launch_ex(score_pass_a<D, GP>, dim3((unsigned)p.score_grid), dim3(kScoreThreads), dyn, st, 1, kmap,
                      args);
 }
 
 }  // namespace
 
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
-                         const int32_t *reuse, uint8_t *ws, cudaStream_t st)
+                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st)
 {
     ScoreArgs a;
+    for (int b = 0; b <= 32; ++b)
+        a.pf_off[b] = (p.B <= 32 && b <= p.B) ? seq_off_host[b] : 0;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.seq_off = seq_off;
     a.reuse = reuse;
@@ -522,6 +692,7 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.ld = p.ld_logits;
     a.partials = reinterpret_cast<float2 *>(ws + p.off_partials);
     a.S = p.score_grid + p.B;
+    a.R = p.score_partials_per_slot;
     a.chunk_table = reinterpret_cast<int32_t *>(ws + p.off_chunk_table);
     a.ctrl = reinterpret_cast<uint32_t *>(ws + p.off_ctrl);
     a.B = p.B;
@@ -532,16 +703,30 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.stage_bytes = p.stage_bytes;
     a.scale = p.scale;
     cudaError_t e;
+    // GP: columns per kv head in the MMA's N (the smallest of 4, 8, 16 that
+    // holds the group); a small N keeps the query tile small and leaves
+    // shared memory to the K ring
     if (p.D == 128)
-        e = p.G <= 8 ? launch_score_t<128, 1>(p, kmap, a, st) : launch_score_t<128, 2>(p, kmap, a, st);
+        e = p.G <= 4 ? launch_score_t<128, 4>(p, kmap, a, st)
+                     : (p.G <= 8 ? launch_score_t<128, 8>(p, kmap, a, st) : launch_score_t<128, 16>(p, kmap, a, st));
     else
-        e = p.G <= 8 ? launch_score_t<64, 1>(p, kmap, a, st) : launch_score_t<64, 2>(p, kmap, a, st);
+        e = p.G <= 4 ? launch_score_t<64, 4>(p, kmap, a, st)
+                     : (p.G <= 8 ? launch_score_t<64, 8>(p, kmap, a, st) : launch_score_t<64, 16>(p, kmap, a, st));
     if (e != cudaSuccess)
         return e;
-    return launch_ex(score_merge, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(32), 0, st, 1,
-                     reinterpret_cast<const float2 *>(ws + p.off_partials), p.score_grid + p.B,
-                     reinterpret_cast<const int32_t *>(ws + p.off_chunk_table),
-                     reinterpret_cast<double *>(ws + p.off_L), p.B, p.Hq, p.score_grid);
+    const float2 *parts = reinterpret_cast<const float2 *>(ws + p.off_partials);
+    const int32_t *table = reinterpret_cast<const int32_t *>(ws + p.off_chunk_table);
+    double *Lp = reinterpret_cast<double *>(ws + p.off_L);
+    const dim3 mgrid((unsigned)p.Hq, (unsigned)p.B);
+    const int S = p.score_grid + p.B;
+    switch (p.score_partials_per_slot) {
+    case 2:
+        return launch_ex(score_merge<2>, mgrid, dim3(32), 0, st, 1, parts, S, table, Lp, p.B, p.Hq, p.score_grid);
+    case 4:
+        return launch_ex(score_merge<4>, mgrid, dim3(32), 0, st, 1, parts, S, table, Lp, p.B, p.Hq, p.score_grid);
+    default:
+        return launch_ex(score_merge<8>, mgrid, dim3(32), 0, st, 1, parts, S, table, Lp, p.B, p.Hq, p.score_grid);
+    }
 }
 
 }  // namespace ts

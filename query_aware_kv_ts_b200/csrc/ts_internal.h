@@ -12,10 +12,12 @@
 namespace ts {
 
 constexpr int kMaxBatch = 1024;        // sequences per call (shared-memory tables)
-constexpr int kScoreConsumerWarps = 8;
-constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
-constexpr int kScoreStages = 6;
-constexpr int kStageBytesTarget = 32768;
+constexpr int kScoreRows = 128;                 // K rows per stage (h_kv heads x T tokens): the MMA's M
+constexpr int kScoreEpiWarps = 8;               // two per TMEM lane quarter (each half of the heads)
+constexpr int kScoreThreads = (kScoreEpiWarps + 2) * 32;   // + TMA producer warp + MMA warp
+constexpr int kScoreMaxStages = 12;
+constexpr int kScoreAccBufs = 4;                // TMEM accumulators in flight
+constexpr size_t kScoreDynSmemBudget = 212 * 1024;   // + the kernel's ~13 KB of static shared memory
 constexpr int kVoteThreads = 256;
 constexpr int kVoteTokensPerBlock = kVoteThreads;   // one token per thread
 constexpr int kSelectThreads = 256;
@@ -74,6 +76,7 @@ struct Plan {
     int stage_bytes;
     int64_t max_chunks;      // sum_b ceil(n_b / T)
     int score_grid;          // <= 256
+    int score_partials_per_slot;   // R: epilogue warps of pass A that see one kv head
     int64_t ld_logits;       // logits row stride: n_total rounded up to 4
     // selection
     int sel_ranges;          // ranges of kSelectTokensPerCta candidates per sequence (grid x)
@@ -96,8 +99,10 @@ void set_error(const char *fmt, ...);
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step,
                             int B, int len, double theta, cudaStream_t st);
 
+// seq_off_host: the host copy of the offsets (prefetch hints before the
+// dependency wait; the device copy decides the work).
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
-                         const int32_t *reuse, uint8_t *ws, cudaStream_t st);
+                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st);
 
 // Selection parameters, for the vote pass that also builds the selection's
 // level-1 histogram.
