@@ -194,7 +194,7 @@ TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_
  * loads the library holds until the process exits.
  *   - Arguments, results and errors as for ts_sparse_attn.  Shapes whose
  *     scratch would exceed 4 MiB (B * h_kv * splits * (h_q/h_kv) * (d+4) * 4
- *     bytes, splits = ceil(ids_capacity / 128)) are rejected with
+ *     bytes, splits = ceil(ids_capacity / 64)) are rejected with
  *     TS_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on each device looks the array up (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream

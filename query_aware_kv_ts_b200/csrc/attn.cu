@@ -2,8 +2,9 @@
 // number of critical KV cache tokens take part in the attention calculation).
 //   out[b, h, :] = sum_j softmax_j(scale * q_h . K[ids_j, g]) * V[ids_j, g]
 //
-// Split-K decode attention: grid (splits, h_kv, B), 256 threads, at most 128
-// selected rows per CTA.  Each CTA:
+// Split-K decode attention: grid (splits, h_kv, B), 256 threads, at most 64
+// selected rows per CTA (small splits spread the gather over many SMs: a
+// block's load phase costs about 10-16 ns per KB it loads).  Each CTA:
 //  1. gathers its K and V rows into shared memory with coalesced 16-byte
 //     asynchronous copies (every row of the CTA in flight at once);
 //  2. computes the logits of the G query heads of kv head g on tensor cores

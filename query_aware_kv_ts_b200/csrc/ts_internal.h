@@ -24,8 +24,8 @@ constexpr int kSelectThreads = 256;
 constexpr int kSelectTokensPerCta = 2048;     // candidates per selection range
 constexpr int kMaxSelectRanges = 2048;        // ranges per sequence: n <= 4M candidates
 constexpr int kAttnThreads = 256;
-constexpr int kAttnRows = 128;        // selected rows per attention CTA (one split)
-constexpr int kMaxCapacity = 128 * kAttnRows;   // k + sink + local
+constexpr int kAttnRows = 64;         // selected rows per attention CTA (one split)
+constexpr int kMaxCapacity = 16384;   // k + sink + local
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
