@@ -327,10 +327,12 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
             const int32_t total = __shfl_sync(0xffffffffu, c1, B - 1);
             __syncwarp();
             if (lane == 0) {
-                const int32_t v0 = chunk_split(blockIdx.x, total, gridDim.x);
-                const int32_t v1 = chunk_split(blockIdx.x + 1, total, gridDim.x);
+                const bool il = B == 1;
+                const int32_t v0 = il ? (int32_t)blockIdx.x : chunk_split(blockIdx.x, total, gridDim.x);
+                const int32_t v1 = il ? total : chunk_split(blockIdx.x + 1, total, gridDim.x);
+                const int32_t vs = il ? (int32_t)gridDim.x : 1;
                 int b = 0;
-                for (int32_t v = v0; v < v1 && v < v0 + npf; ++v) {
+                for (int32_t v = v0; v < v1 && v < v0 + npf * vs; v += vs) {
                     while (b + 1 < B && sh.pf_start[b + 1] <= v)
                         ++b;
                     const int64_t t0 = sh.pf_off[b] + (int64_t)(v - sh.pf_start[b]) * T;
@@ -418,8 +420,14 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
         for (int b = tid; b <= B; b += blockDim.x)
             a.chunk_table[b] = sh.chunk_start[b];
     const int32_t total = sh.chunk_start[B];
-    const int32_t v_begin = chunk_split(blockIdx.x, total, gridDim.x);
-    const int32_t v_end = chunk_split(blockIdx.x + 1, total, gridDim.x);
+    // chunks of this CTA: v_begin, v_begin + v_step, ... < v_end.  A single
+    // sequence is dealt round-robin (CTA j: j, j + grid, ...), so every SM
+    // reads from every part of the cache; several sequences keep contiguous
+    // ranges [j*C/grid, (j+1)*C/grid) (one segment per CTA and sequence).
+    const bool interleave = B == 1;
+    const int32_t v_begin = interleave ? (int32_t)blockIdx.x : chunk_split(blockIdx.x, total, gridDim.x);
+    const int32_t v_end = interleave ? total : chunk_split(blockIdx.x + 1, total, gridDim.x);
+    const int32_t v_step = interleave ? (int32_t)gridDim.x : 1;
     const uint32_t tmem = sh.tmem_base;
     const int half_bytes = kScoreRows * 128;   // one 64-channel box
 
@@ -428,7 +436,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
-            for (int32_t v = v_begin; v < v_end; ++v, ++it) {
+            for (int32_t v = v_begin; v < v_end; v += v_step, ++it) {
                 const int b = upper_seq(sh.chunk_start, B, v);
                 const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
                 const int s = it % NS;
@@ -457,7 +465,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
         bool dead = false;
         uint32_t done_par = 0;
         uint32_t it = 0;
-        for (int32_t v = v_begin; v < v_end && !dead; ++v, ++it) {
+        for (int32_t v = v_begin; v < v_end && !dead; v += v_step, ++it) {
             const int b = upper_seq(sh.chunk_start, B, v);
             if (b != cur_b) {
                 if (cur_b >= 0) {   // the old queries may still be read by MMAs in flight
@@ -534,7 +542,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
                             ((int64_t)blockIdx.x + cur_b) * a.R);
         };
 
-        for (int32_t v = v_begin; v < v_end; ++v, ++it) {
+        for (int32_t v = v_begin; v < v_end; v += v_step, ++it) {
             const int b = upper_seq(sh.chunk_start, B, v);
             if (b != cur_b) {
                 if (cur_b >= 0)
@@ -625,9 +633,14 @@ score_merge(const float2 *partials, int S, const int32_t *chunk_table, double *L
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
         const int j = e / R;   // R is a power of 2: a shift
-        bool keep = e < n && j >= j0 && j <= j1;
-        if (keep && total < grid_a)   // some CTAs had no chunks and wrote nothing
-            keep = chunk_split(j, total, grid_a) < chunk_split(j + 1, total, grid_a);
+        bool keep;
+        if (B == 1) {   // round-robin chunks: CTA j has some iff j < total
+            keep = e < n && j < total;
+        } else {
+            keep = e < n && j >= j0 && j <= j1;
+            if (keep && total < grid_a)   // some CTAs had no chunks and wrote nothing
+                keep = chunk_split(j, total, grid_a) < chunk_split(j + 1, total, grid_a);
+        }
         if (!keep)
             pv[i] = make_float2(-INFINITY, 0.0f);
     }
