@@ -72,3 +72,33 @@ def test_host_side_argument_errors(lib):
     assert lib.ts_workspace_init(None, 0, None) == 3
     lib.ts_selftest_expire_wait.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]
     assert lib.ts_selftest_expire_wait(None, 0, 10, None) == 3
+
+
+class _KV(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("seq_offsets_dev", ctypes.c_void_p),
+                ("seq_offsets_host", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64), ("scale", ctypes.c_float)]
+
+
+def test_decode_step_checks_everything_before_launching(lib):
+    """ts_decode_step validates its whole argument list on the host: nothing
+    is launched (no GPU is touched here) when any argument is wrong."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    P, I32, F64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_double, ctypes.c_size_t
+    lib.ts_decode_step.argtypes = [ctypes.POINTER(_KV), P, P, P, P, I32, F64, I32, I32, I32, P, P, P, P, P, SZ, P]
+
+    def call(kv, k=16, s=4, l=8):
+        return lib.ts_decode_step(kv, None, None, None, None, 1, 0.9, k, s, l, None, None, None, None, None, 0,
+                                  None)
+
+    assert call(None, k=-1) == 1 and b"non-negative" in lib.ts_last_error()
+    assert call(None, k=0, s=0, l=0) == 1                     # empty selection capacity
+    assert call(None) == 1 and b"kv" in lib.ts_last_error()
+    off = (ctypes.c_int64 * 2)(0, 64)
+    kv = _KV(1, 6, 4, 64, ctypes.addressof(off), ctypes.addressof(off), 16, 16, 256, 64, 0.0)
+    assert call(ctypes.byref(kv)) == 1 and b"multiple" in lib.ts_last_error()   # h_q % h_kv
+    kv = _KV(1, 8, 4, 96, ctypes.addressof(off), ctypes.addressof(off), 16, 16, 384, 96, 0.0)
+    assert call(ctypes.byref(kv)) == 2                         # head_dim 96: unsupported
+    kv = _KV(1, 8, 4, 64, ctypes.addressof(off), ctypes.addressof(off), 8, 16, 256, 64, 0.0)
+    assert call(ctypes.byref(kv)) == 1 and b"16-byte" in lib.ts_last_error()    # misaligned K
