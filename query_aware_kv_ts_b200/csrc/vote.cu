@@ -17,7 +17,8 @@
 //
 // Work split: grid (groups / threads, B).  Long sequences: a thread takes 4
 // consecutive tokens aligned to 4 in the logits rows (row stride padded to 4),
-// so each head's logits arrive as one 16-byte load, 8 heads at a time; short
+// so each head's logits arrive as one 16-byte load, the next 4 heads' loads in
+// flight while 4 heads are computed; short
 // sequences: four lanes per token, each summing every fourth head (the exp
 // chains are latency-bound: more warps per token hide them), then two shuffles.
 // The reuse flag, the sequence bounds and the normalisers L are fetched in one
@@ -125,22 +126,34 @@ vote_pass_b(const VoteArgs a)
         acc[j] = 0.0f;
     if (i0 < end) {
         if constexpr (TPT == 4) {
-            for (int h0 = 0; h0 < a.Hq; h0 += kHeadBatch) {
-                float4 sv[kHeadBatch];
+            // software-pipelined over batches of kPipe heads: the next batch's
+            // loads are in flight while this one is computed
+            constexpr int kPipe = 4;
+            const float4 *lg = reinterpret_cast<const float4 *>(a.logits + i0);
+            const int64_t ld4 = a.ld / 4;
+            float4 cur[kPipe], nxt[kPipe];
 #pragma unroll
-                for (int u = 0; u < kHeadBatch; ++u)
-                    if (h0 + u < a.Hq)
-                        sv[u] = __ldcg(reinterpret_cast<const float4 *>(a.logits + (int64_t)(h0 + u) * a.ld + i0));
+            for (int u = 0; u < kPipe; ++u)
+                cur[u] = u < a.Hq ? __ldcg(lg + (int64_t)u * ld4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int h0 = 0; h0 < a.Hq; h0 += kPipe) {
 #pragma unroll
-                for (int u = 0; u < kHeadBatch; ++u) {
+                for (int u = 0; u < kPipe; ++u) {
+                    const int h = h0 + kPipe + u;
+                    nxt[u] = h < a.Hq ? __ldcg(lg + (int64_t)h * ld4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
+#pragma unroll
+                for (int u = 0; u < kPipe; ++u) {
                     if (h0 + u < a.Hq) {
                         const float Lhi = s_hi[h0 + u], Llo = s_lo[h0 + u];
-                        acc[0] += exp_exact_arg(sv[u].x, Lhi, Llo);
-                        acc[1] += exp_exact_arg(sv[u].y, Lhi, Llo);
-                        acc[2] += exp_exact_arg(sv[u].z, Lhi, Llo);
-                        acc[3] += exp_exact_arg(sv[u].w, Lhi, Llo);
+                        acc[0] += exp_exact_arg(cur[u].x, Lhi, Llo);
+                        acc[1] += exp_exact_arg(cur[u].y, Lhi, Llo);
+                        acc[2] += exp_exact_arg(cur[u].z, Lhi, Llo);
+                        acc[3] += exp_exact_arg(cur[u].w, Lhi, Llo);
                     }
                 }
+#pragma unroll
+                for (int u = 0; u < kPipe; ++u)
+                    cur[u] = nxt[u];
             }
         } else {
             // four lanes per token, each summing every fourth head
