@@ -23,6 +23,7 @@ reference arm.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -58,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run only the first N layers of the workload (a smaller case of the same kernels, "
+                         "for profiler captures); the JSON line's config records it")
     a = ap.parse_args(argv)
     big = a.workload in ("llama8b_b4", "ragged_b32", "qwen7b_1m")
     if a.steps is None:
@@ -204,10 +208,15 @@ def profile_traffic(kernel_src: str, workload: str):
 # ---------------------------------------------------------------------------
 
 class Workload:
-    def __init__(self, name: str, device):
+    def __init__(self, name: str, device, layers=None):
         import query_aware_kv_ts_b200 as ts
         self.ts = ts
-        self.cfg = cfg = W.CONFIGS[name]
+        cfg = W.CONFIGS[name]
+        if layers is not None:
+            if not 1 <= layers <= cfg.layers:
+                raise SystemExit("--layers must be in [1, %d] for %s" % (cfg.layers, name))
+            cfg = dataclasses.replace(cfg, layers=layers)
+        self.cfg = cfg
         self.name = name
         self.device = device
         self.layers = []
@@ -343,7 +352,7 @@ def run_ours(a, d: Dist):
     torch.cuda.set_device(d.local)
     dev = torch.device("cuda", d.local)
     d.init("nccl")
-    wl = Workload(a.workload, dev)
+    wl = Workload(a.workload, dev, a.layers)
     cfg = wl.cfg
     ts = wl.ts
 
