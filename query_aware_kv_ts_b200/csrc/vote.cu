@@ -64,11 +64,72 @@ __device__ __forceinline__ float exp_exact_arg(float s, float Lhi, float Llo)
     return fmaf(p, u_lo * kLn2, p);
 }
 
+// Blackwell's packed fp32 instructions: two lanes per instruction, each lane
+// rounded exactly as the scalar IEEE operation.  The low half is the first
+// element (the lower address when loaded from memory).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// exp_exact_arg of two tokens at once: the same operations in the same
+// order, lane by lane (u is carried negated, -u = t * -log2e_hi exactly),
+// so each lane's result is bit-identical to the scalar function's.
+struct PackedL {
+    uint64_t hi, nhi, lo;   // (L_hi, L_hi), (-L_hi, -L_hi), (L_lo, L_lo)
+};
+__device__ __forceinline__ uint64_t exp_exact_arg2(uint64_t s, const PackedL &L)
+{
+    const uint64_t kHi2 = f2_pack(kLog2eHi, kLog2eHi), kNHi2 = f2_pack(-kLog2eHi, -kLog2eHi);
+    const uint64_t kLo2 = f2_pack(kLog2eLo, kLog2eLo), kLn22 = f2_pack(kLn2, kLn2);
+    const uint64_t t = f2_sub(s, L.hi);
+    const uint64_t bp = f2_sub(t, s);
+    const uint64_t e = f2_add(f2_sub(s, f2_sub(t, bp)), f2_sub(L.nhi, bp));
+    const uint64_t d = f2_sub(e, L.lo);
+    const uint64_t nu = f2_mul(t, kNHi2);
+    const uint64_t u_lo = f2_add(f2_fma(t, kHi2, nu), f2_fma(t, kLo2, f2_mul(d, kHi2)));
+    float nu0, nu1;
+    f2_unpack(nu, nu0, nu1);
+    const uint64_t p = f2_pack(exp2f(-nu0), exp2f(-nu1));
+    return f2_fma(p, f2_mul(u_lo, kLn22), p);
+}
+
 template <int TPT, bool HIST>
-__global__ void __launch_bounds__(kVoteThreads)
+__global__ void __launch_bounds__(kVoteThreads, 4)
 vote_pass_b(const VoteArgs a)
 {
     __shared__ float s_hi[kMaxHeadsVote], s_lo[kMaxHeadsVote];
+    __shared__ PackedL s_pl[TPT == 4 ? kMaxHeadsVote : 1];
     __shared__ uint32_t s_hist[HIST ? 4096 : 1];
     __shared__ uint16_t s_used[HIST ? 1024 : 1];   // bins this block touched (<= its tokens)
     __shared__ uint32_t s_nused;
@@ -104,8 +165,11 @@ vote_pass_b(const VoteArgs a)
         const int h = tid + u * nt;
         if (h < a.Hq) {
             const float hi = (float)Lv[u];
+            const float lo = (float)(Lv[u] - (double)hi);
             s_hi[h] = hi;
-            s_lo[h] = (float)(Lv[u] - (double)hi);
+            s_lo[h] = lo;
+            if (TPT == 4)
+                s_pl[TPT == 4 ? h : 0] = PackedL{f2_pack(hi, hi), f2_pack(-hi, -hi), f2_pack(lo, lo)};
         }
     }
     __syncthreads();
@@ -127,34 +191,37 @@ vote_pass_b(const VoteArgs a)
     if (i0 < end) {
         if constexpr (TPT == 4) {
             // software-pipelined over batches of kPipe heads: the next batch's
-            // loads are in flight while this one is computed
+            // loads are in flight while this one is computed; tokens in pairs
+            // on the packed fp32 pipes (a 16-byte load is two packed pairs)
             constexpr int kPipe = 4;
-            const float4 *lg = reinterpret_cast<const float4 *>(a.logits + i0);
+            const ulonglong2 *lg = reinterpret_cast<const ulonglong2 *>(a.logits + i0);
             const int64_t ld4 = a.ld / 4;
-            float4 cur[kPipe], nxt[kPipe];
+            const ulonglong2 zero = make_ulonglong2(0ull, 0ull);
+            ulonglong2 cur[kPipe], nxt[kPipe];
+            uint64_t acc01 = 0ull, acc23 = 0ull;   // +0.0f in both halves
 #pragma unroll
             for (int u = 0; u < kPipe; ++u)
-                cur[u] = u < a.Hq ? __ldcg(lg + (int64_t)u * ld4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                cur[u] = u < a.Hq ? __ldcg(lg + (int64_t)u * ld4) : zero;
             for (int h0 = 0; h0 < a.Hq; h0 += kPipe) {
 #pragma unroll
                 for (int u = 0; u < kPipe; ++u) {
                     const int h = h0 + kPipe + u;
-                    nxt[u] = h < a.Hq ? __ldcg(lg + (int64_t)h * ld4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    nxt[u] = h < a.Hq ? __ldcg(lg + (int64_t)h * ld4) : zero;
                 }
 #pragma unroll
                 for (int u = 0; u < kPipe; ++u) {
                     if (h0 + u < a.Hq) {
-                        const float Lhi = s_hi[h0 + u], Llo = s_lo[h0 + u];
-                        acc[0] += exp_exact_arg(cur[u].x, Lhi, Llo);
-                        acc[1] += exp_exact_arg(cur[u].y, Lhi, Llo);
-                        acc[2] += exp_exact_arg(cur[u].z, Lhi, Llo);
-                        acc[3] += exp_exact_arg(cur[u].w, Lhi, Llo);
+                        const PackedL L = s_pl[h0 + u];
+                        acc01 = f2_add(acc01, exp_exact_arg2(cur[u].x, L));
+                        acc23 = f2_add(acc23, exp_exact_arg2(cur[u].y, L));
                     }
                 }
 #pragma unroll
                 for (int u = 0; u < kPipe; ++u)
                     cur[u] = nxt[u];
             }
+            f2_unpack(acc01, acc[0], acc[1]);
+            f2_unpack(acc23, acc[2], acc[3]);
         } else {
             // four lanes per token, each summing every fourth head
             for (int h0 = q4; h0 < a.Hq; h0 += 4 * kHeadBatch) {
