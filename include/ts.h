@@ -212,9 +212,10 @@ TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, cons
  * One whole decode step of one layer: ts_selcache, ts_score, ts_select and
  * ts_sparse_attn in that order on `stream`, with the same arguments and the
  * same results as the four calls (selection capacity k + n_sink + n_local, the
- * ids row length).  Fewer kernels run: the vote pass also builds the
- * selection's first-level vote histogram, which ts_select otherwise builds in
- * a kernel of its own.  Every argument is checked before the first launch.
+ * ids row length; bit for bit).  Fewer kernels run: the vote pass also builds
+ * the selection's first-level vote histogram, which ts_select otherwise builds
+ * in a kernel of its own (ts_decode_step_kernels gives the count).  Every
+ * argument is checked before the first launch.
  *   reuse      device int32 [batch], required: written by the selection cache
  *              and read by every later phase (sequences that reuse keep their
  *              previous ids and count; their votes are left as they were)
@@ -224,6 +225,14 @@ TS_API ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev
                                   double *cos_out, int32_t first_step, double threshold, int32_t k,
                                   int32_t n_sink, int32_t n_local, float *votes, int32_t *ids,
                                   int32_t *count, float *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Number of kernels one ts_decode_step call on this cache launches (for
+ * launch accounting and profiling), or -1 with ts_last_error set when the
+ * cache description or the selection sizes are invalid.  Host only; touches
+ * no device memory.
+ */
+TS_API int32_t ts_decode_step_kernels(const ts_kv_t *kv, int32_t k, int32_t n_sink, int32_t n_local);
 
 /*
  * Read and clear the device status word of a workspace (synchronises the

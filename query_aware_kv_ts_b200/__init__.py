@@ -67,6 +67,7 @@ _SIGS = {
     "ts_sparse_attn_noalloc": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P]),
     "ts_decode_step": (ctypes.c_int, [_KV, _P, _P, _P, _P, _I32, _F64, _I32, _I32, _I32, _P, _P, _P, _P, _P,
                                       _SZ, _P]),
+    "ts_decode_step_kernels": (_I32, [_KV, _I32, _I32, _I32]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -197,6 +198,14 @@ def ts_decode_step(kv: KVCache, q, q_prev, reuse, first_step: bool, threshold: f
                                int(bool(first_step)), float(threshold), k, n_sink, n_local, _ptr(votes),
                                _ptr(ids), _ptr(count), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                _stream(stream)))
+
+
+def ts_decode_step_kernels(kv: KVCache, k: int, n_sink: int, n_local: int) -> int:
+    """Kernels one ts_decode_step call on this cache launches."""
+    n = _lib.ts_decode_step_kernels(kv.ref(), k, n_sink, n_local)
+    if n < 0:
+        raise TsError(TS_ERR_INVALID_ARG, ts_last_error())
+    return int(n)
 
 
 def ts_get_device_status(ws, stream=None):

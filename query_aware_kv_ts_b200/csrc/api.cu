@@ -523,6 +523,21 @@ ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_decode_step: sparse attention launch");
 }
 
+int32_t ts_decode_step_kernels(const ts_kv_t *kv, int32_t k, int32_t n_sink, int32_t n_local)
+{
+    if (k < 0 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > (int64_t(1) << 30) ||
+        k + n_sink + n_local < 1) {
+        set_error("k, n_sink, n_local must be non-negative with a sum in [1, 2^30)");
+        return -1;
+    }
+    Plan p;
+    if (make_plan(kv, k + n_sink + n_local, &p) != TS_OK)
+        return -1;
+    // selection cache; score pass A, normaliser merge, vote pass (with the
+    // selection histogram); collect, resolve, write; attention split, merge
+    return 1 + (p.n_total > 0 ? 3 : 0) + 3 + 2;
+}
+
 ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream)
 {
     if (ws == nullptr || ws_bytes < 256) {

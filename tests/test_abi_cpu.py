@@ -102,3 +102,14 @@ def test_decode_step_checks_everything_before_launching(lib):
     assert call(ctypes.byref(kv)) == 2                         # head_dim 96: unsupported
     kv = _KV(1, 8, 4, 64, ctypes.addressof(off), ctypes.addressof(off), 8, 16, 256, 64, 0.0)
     assert call(ctypes.byref(kv)) == 1 and b"16-byte" in lib.ts_last_error()    # misaligned K
+
+
+def test_decode_step_kernels_rejects_bad_arguments(lib):
+    """ts_decode_step_kernels answers -1 (with an error message) for invalid
+    selection sizes or a missing cache, before any device query."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    lib.ts_decode_step_kernels.restype = ctypes.c_int32
+    lib.ts_decode_step_kernels.argtypes = [ctypes.POINTER(_KV), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    assert lib.ts_decode_step_kernels(None, -1, 4, 8) == -1 and b"non-negative" in lib.ts_last_error()
+    assert lib.ts_decode_step_kernels(None, 0, 0, 0) == -1
+    assert lib.ts_decode_step_kernels(None, 16, 4, 8) == -1 and b"kv" in lib.ts_last_error()

@@ -105,3 +105,14 @@ def test_trajectory_fused_equals_four_calls(cfg_name, n):
         prev_ids = bf.ids.cpu().numpy().copy()
         reused += int(reuse.sum())
     assert reused > 0, "the trajectory never reused a selection"
+
+
+
+@pytest.mark.parametrize("cfg_name", ["tiny", "qwen7b_32k", "llama8b_b4", "ragged_b32"])
+def test_kernel_count(cfg_name):
+    """ts_decode_step_kernels reports the nine kernels of a step (selection
+    cache; score pass A, merge, vote pass; collect, resolve, write; attention
+    split, merge)."""
+    cfg = W.CONFIGS[cfg_name]
+    case, _ = H.config_case(cfg, n_override=min(cfg.n, 4096))
+    assert H.ts().ts_decode_step_kernels(case.kv, cfg.k, cfg.n_sink, cfg.n_local) == 9
