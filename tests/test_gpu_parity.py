@@ -3,8 +3,10 @@
 Small synthetic cases cover every kernel specialisation (head_dim 64/128,
 group sizes 1..16, h_kv 1..8), ragged batches with empty and one-token
 sequences, tails that are not a multiple of the tile, windows larger than the
-sequence, k = 0 and k >= candidates, tied votes, padded strides and very peaked
-scores.  Each case spans several 16-token tiles and a ragged tail."""
+sequence, k = 0 and k >= candidates, tied votes, padded strides, very peaked
+scores, more than 32 sequences, and the largest batch (1024) and selection
+capacity (16384) the library takes.  Each case spans several tiles and a
+ragged tail."""
 import zlib
 
 import numpy as np
@@ -56,6 +58,12 @@ CASES = {
     "integer_keys_many_ties": ([2000], 28, 4, 128, 200, 4, 64, {"dist": "int"}),
     "padded_strides": ([3000], 28, 4, 128, 256, 4, 64, {"strides": (4 * 128 * 2 + 64, 256)}),
     "peaked_scores": ([2500], 8, 2, 128, 64, 4, 32, {"scale": 1.0}),
+    # more than 32 sequences (score pass A's general chunk-table path)
+    "batch_40_qwen_heads": ([int(x) for x in np.random.default_rng(40).integers(1, 700, 40)], 28, 4, 128, 64, 4,
+                            32, {}),
+    # the largest batch and the largest selection the library takes
+    "max_batch_1024": ([int(x) for x in np.random.default_rng(1024).integers(0, 41, 1024)], 4, 2, 64, 8, 2, 4, {}),
+    "max_capacity_16384": ([20000], 4, 2, 64, 16384 - 4 - 64, 4, 64, {"planted": 32}),
 }
 
 
