@@ -61,6 +61,8 @@ def _declare(lib):
     lib.oracle_windows.restype = None
     lib.oracle_select.argtypes = [P, i64, i64, i64, i64, P]
     lib.oracle_select.restype = i64
+    lib.oracle_reuse_ids.argtypes = [P, i64, i64, i64, i64, i64, i64, P]
+    lib.oracle_reuse_ids.restype = i64
     lib.oracle_sparse_attn.argtypes = [P, P, i32, i32, i64, i64, P, i32, f64, P, i64, P]
     lib.oracle_sparse_attn.restype = None
     lib.oracle_dense_attn.argtypes = [P, P, i64, i32, i32, i64, i64, P, i32, f64, P]
@@ -193,6 +195,18 @@ def select(v, k: int, n_sink: int, n_local: int) -> tuple[np.ndarray, int]:
     return ids, int(m)
 
 
+def reuse_ids(prev_ids, prev_count: int, n_old: int, n_new: int, k: int, n_sink: int,
+              n_local: int) -> tuple[np.ndarray, int]:
+    """The ids of a sequence that reuses its selection after its cache grew from
+    n_old to n_new tokens: the previous top-k part with the current sink and
+    local windows (reading R19; the previous row itself when n_new == n_old).
+    Returns (ids int32 [k + n_sink + n_local] with -1 padding, count)."""
+    prev = np.ascontiguousarray(prev_ids, dtype=np.int32)
+    out = np.empty(k + n_sink + n_local, np.int32)
+    m = lib().oracle_reuse_ids(_ptr(prev), int(prev_count), int(n_old), int(n_new), k, n_sink, n_local, _ptr(out))
+    return out, int(m)
+
+
 def sparse_attn(k, v, q, ids, m: int | None = None, scale: float | None = None) -> np.ndarray:
     k, st, sh = _kv_view(k)
     v, vst, vsh = _kv_view(v)
@@ -284,3 +298,44 @@ def decode_step(k, v, seq_offsets, q, k_top: int, n_sink: int, n_local: int,
         res.count[b] = m
         res.out.append(sparse_attn(kb, vb, qb, ids, m, scale))
     return res
+
+
+# ---------------------------------------------------------------------------
+# A decode loop over one growing sequence
+# ---------------------------------------------------------------------------
+
+def decode_loop(k, v, n0: int, qs, k_top: int, n_sink: int, n_local: int, theta: float,
+                scale=None, reuse_override=None) -> list[dict]:
+    """One layer of one sequence over T decode steps with KV append (reading
+    R19): step t attends over the first n_t = n0 + t tokens of k, v (the token
+    appended before the step included).  The selection cache compares q_t with
+    q_{t-1} (never at t = 0); on reuse the ids are reuse_ids() of the previous
+    step's row, otherwise the full vote and selection over the n_t tokens.
+
+    k, v: uint16 [>= n0 + T - 1, h_kv, d]; qs: uint16 [T, h_q, d].
+    reuse_override: optional bool [T] replacing the cosine decision.
+    Returns one dict per step: reuse, cos, n, ids, count, out (and votes when
+    the selection was recomputed)."""
+    k, v, qs = _u16(k), _u16(v), _u16(qs)
+    T = qs.shape[0]
+    q_prev = np.zeros_like(qs[0])
+    steps = []
+    prev = None
+    for t in range(T):
+        n_t = n0 + t
+        reuse, c = selcache(qs[t], q_prev, t == 0, theta)
+        if reuse_override is not None:
+            reuse = bool(reuse_override[t])
+        kb, vb = k[:n_t], v[:n_t]
+        rec = {"reuse": reuse, "cos": c, "n": n_t}
+        if reuse:
+            ids, m = reuse_ids(prev["ids"], prev["count"], prev["n"], n_t, k_top, n_sink, n_local)
+        else:
+            vt, _ = votes(kb, qs[t], scale)
+            ids, m = select(vt, k_top, n_sink, n_local)
+            rec["votes"] = vt
+        rec["ids"], rec["count"] = ids, m
+        rec["out"] = sparse_attn(kb, vb, qs[t], ids, m, scale)
+        steps.append(rec)
+        prev = rec
+    return steps

@@ -20,7 +20,7 @@
  *                summary): non-contiguous, token-level attention sparsity,
  *                per-head soft voting, Selection Cache, dot-product kernel.
  * Where the pages leave a step open, the reading used is noted at the
- * function (R1..R10 in the design notes).
+ * function (readings R1..R19).
  *
  * Conventions shared by every function:
  *   - bf16 inputs are passed as raw uint16 bit patterns and widened exactly
@@ -239,6 +239,47 @@ int64_t oracle_select(const double *v, int64_t n, int64_t k, int64_t n_sink,
     }
     int64_t m = 0;
     for (int64_t i = 0; i < n; ++i)
+        if (chosen[i])
+            ids_out[m++] = (int32_t)i;
+    free(chosen);
+    return m;
+}
+
+/* Ids of a sequence that reuses its selection while its cache grows (a
+ * decode loop that appends the new token's K/V before each step; TS-README
+ * "Key Takeaways", Selection Cache; reading R19).  What is reused is the
+ * previous step's top-k part T_prev: the ids of the previous row that lie in
+ * that step's candidate range [s'_old, l0_old).  The sink and local windows
+ * are those of the current length n_new, and a kept id that is no longer a
+ * candidate, outside [s'_new, l0_new), is dropped:
+ *   ids = sort([0, s'_new) U (T_prev n [s'_new, l0_new)) U [l0_new, n_new)).
+ * With n_new == n_old this is the previous row itself (R8).
+ * prev_ids: the previous row, ascending, prev_count entries valid.
+ * ids_out must hold k + n_sink + n_local entries; entries past the returned
+ * count are set to -1.  Returns the count. */
+int64_t oracle_reuse_ids(const int32_t *prev_ids, int64_t prev_count, int64_t n_old, int64_t n_new,
+                         int64_t k, int64_t n_sink, int64_t n_local, int32_t *ids_out)
+{
+    int64_t cap = k + n_sink + n_local;
+    for (int64_t j = 0; j < cap; ++j)
+        ids_out[j] = -1;
+    if (n_new <= 0)
+        return 0;
+    int64_t s_old, l0_old, s_new, l0_new;
+    oracle_windows(n_old, n_sink, n_local, &s_old, &l0_old);
+    oracle_windows(n_new, n_sink, n_local, &s_new, &l0_new);
+    unsigned char *chosen = (unsigned char *)calloc((size_t)n_new, 1);
+    for (int64_t i = 0; i < s_new; ++i)
+        chosen[i] = 1;
+    for (int64_t i = l0_new; i < n_new; ++i)
+        chosen[i] = 1;
+    for (int64_t j = 0; j < prev_count; ++j) {
+        int64_t id = prev_ids[j];
+        if (id >= s_old && id < l0_old && id >= s_new && id < l0_new)
+            chosen[id] = 1;
+    }
+    int64_t m = 0;
+    for (int64_t i = 0; i < n_new && m < cap; ++i)
         if (chosen[i])
             ids_out[m++] = (int32_t)i;
     free(chosen);

@@ -313,4 +313,98 @@ def pin_ar1_reuse_rate():
     assert 0.80 < reuse < 0.95, reuse
 
 
+
+# ------------------------------------------------ decode loop with KV append (R19)
+
+def _rand_query(seed, h_q, d):
+    g = torch.Generator().manual_seed(seed)
+    return W.bf16_bits(torch.randn((h_q, d), generator=g).to(torch.bfloat16))
+
+
+def pin_reuse_hand_example():
+    """The hand-worked growth, shrink and unchanged-length cases."""
+    c = _golden()["reuse_with_growth"]
+    v = np.array(c["votes"], np.float64)
+    ids, m = oracle.select(v, c["k"], c["n_sink"], c["n_local"])
+    assert m == c["step0"]["count"] and ids[:m].tolist() == c["step0"]["ids"], (ids, m)
+    for r in c["reused"]:
+        got, gm = oracle.reuse_ids(ids, m, r["n_old"], r["n_new"], c["k"], c["n_sink"], c["n_local"])
+        assert gm == r["count"] and got[:gm].tolist() == r["ids"] and (got[gm:] == -1).all(), (r, got, gm)
+    t = c["tiny_then_grow"]
+    got, gm = oracle.reuse_ids(np.array(t["prev_ids"], np.int32), t["prev_count"], t["n_old"], t["n_new"], c["k"],
+                               c["n_sink"], c["n_local"])
+    assert gm == t["count"] and got[:gm].tolist() == t["ids"], (got, gm)
+
+
+def pin_reuse_unchanged_length_keeps_row():
+    """With the same length the reused row is exactly the previous row (R8)."""
+    rng = np.random.default_rng(777)
+    for _ in range(300):
+        n = int(rng.integers(0, 80))
+        k, s, l = int(rng.integers(0, 20)), int(rng.integers(0, 6)), int(rng.integers(0, 12))
+        ids, m = oracle.select(np.round(rng.random(n) * 8) / 8, k, s, l)
+        got, gm = oracle.reuse_ids(ids, m, n, n, k, s, l)
+        assert gm == m and np.array_equal(got, ids), (n, k, s, l)
+
+
+def pin_reuse_growth_properties():
+    """After growth from n0 to n1 >= n0: the windows of n1 are in the row, every
+    other id was selected at n0 (it is from the old top-k part, which rank
+    counting finds independently), the old top-k part is kept whole, and
+    growing in two steps gives the same row as growing in one."""
+    rng = np.random.default_rng(4242)
+    for _ in range(400):
+        n0 = int(rng.integers(0, 70))
+        n1 = n0 + int(rng.integers(0, 12))
+        n2 = n1 + int(rng.integers(0, 12))
+        k, s, l = int(rng.integers(0, 20)), int(rng.integers(0, 6)), int(rng.integers(0, 12))
+        v = np.round(rng.random(n0) * 8) / 8
+        ids, m = oracle.select(v, k, s, l)
+        got, gm = oracle.reuse_ids(ids, m, n0, n1, k, s, l)
+        row = got[:gm]
+        assert (got[gm:] == -1).all() and np.all(np.diff(row) > 0) and (gm == 0 or row[-1] < n1)
+        s1, l1 = min(s, n1), max(n1 - l, min(s, n1))
+        assert set(range(s1)) <= set(row.tolist()) and set(range(l1, n1)) <= set(row.tolist())
+        s0, l0 = min(s, n0), max(n0 - l, min(s, n0))
+        top_old = {int(i) for i in _brute_select(v, k, s, l) if s0 <= i < l0}
+        middle = {int(i) for i in row if s1 <= i < l1}
+        assert middle == top_old, (n0, n1, k, s, l)          # growth never pushes a kept id out
+        two, tm = oracle.reuse_ids(got, gm, n1, n2, k, s, l)
+        one, om = oracle.reuse_ids(ids, m, n0, n2, k, s, l)
+        assert tm == om and np.array_equal(two, one), (n0, n1, n2, k, s, l)
+
+
+def pin_decode_loop_slides_the_local_window():
+    """A decode loop that reuses at every step after the first keeps the first
+    step's top-k part, and its local window follows the growing cache: the
+    last n_local ids of step t are n_t - n_local .. n_t - 1."""
+    d, h_q, h_kv, n0, T = 16, 4, 2, 200, 6
+    k, v, _ = _rand_case(31, n0 + T, h_q, h_kv, d)
+    qs = np.stack([_rand_query(90 + t, h_q, d) for t in range(T)])
+    kt, s, l = 12, 3, 8
+    steps = oracle.decode_loop(k, v, n0, qs, kt, s, l, theta=0.9, reuse_override=[False] + [True] * (T - 1))
+    first = steps[0]
+    top0 = [int(i) for i in first["ids"][:first["count"]] if s <= i < n0 - l]
+    assert len(top0) == kt
+    for t, st in enumerate(steps):
+        row = st["ids"][:st["count"]].tolist()
+        assert st["n"] == n0 + t and st["count"] == kt + s + l
+        assert row[:s] == list(range(s)) and row[s:s + kt] == top0 and row[-l:] == list(range(n0 + t - l, n0 + t))
+
+
+def pin_decode_loop_without_reuse_is_a_fresh_step():
+    """Without reuse every step is the single-step oracle over the current
+    prefix of the cache: the loop appends before it attends."""
+    d, h_q, h_kv, n0, T = 16, 4, 2, 120, 4
+    k, v, _ = _rand_case(77, n0 + T, h_q, h_kv, d)
+    qs = np.stack([_rand_query(500 + t, h_q, d) for t in range(T)])
+    steps = oracle.decode_loop(k, v, n0, qs, 10, 2, 6, theta=2.0)
+    for t, st in enumerate(steps):
+        n = n0 + t
+        assert not st["reuse"]
+        ref = oracle.decode_step(k[:n], v[:n], np.array([0, n]), qs[t][None], 10, 2, 6)
+        assert st["count"] == ref.count[0] and np.array_equal(st["ids"], ref.ids[0])
+        assert np.array_equal(st["out"], ref.out[0])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

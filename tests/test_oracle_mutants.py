@@ -35,6 +35,12 @@ MUTANTS = {
     "cosine_strict": ("reuse = (c >= theta) ? 1 : 0;", "reuse = (c > theta) ? 1 : 0;"),
     "cosine_no_norm": ("return ab / (sqrt(aa) * sqrt(bb));", "return ab / sqrt(aa * aa);"),
     "qprev_not_updated": ("    memcpy(q_prev, q, (size_t)len * sizeof(uint16_t));\n", "\n"),
+    "reuse_windows_of_old_length": ("oracle_windows(n_new, n_sink, n_local, &s_new, &l0_new);",
+                                    "oracle_windows(n_old, n_sink, n_local, &s_new, &l0_new);"),
+    "reuse_keeps_old_local_window": ("if (id >= s_old && id < l0_old && id >= s_new && id < l0_new)",
+                                     "if (id >= s_old && id >= s_new && id < l0_new)"),
+    "reuse_drops_topk_part": ("if (id >= s_old && id < l0_old && id >= s_new && id < l0_new)\n            chosen[id] = 1;",
+                              "if (id < 0)\n            chosen[id] = 1;"),
 }
 
 
