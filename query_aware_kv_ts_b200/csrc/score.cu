@@ -11,8 +11,10 @@
 // Design (B200):
 //  * One CTA per SM, persistent.  The active sequences' tokens are cut into
 //    chunks of T = 128 / h_kv tokens, so that a chunk holds 128 K rows (h_kv
-//    heads x T tokens, one pipeline stage); CTA j takes the contiguous,
-//    balanced chunk range [j*C/grid, (j+1)*C/grid).
+//    heads x T tokens, one pipeline stage).  Several sequences: CTA j takes
+//    the contiguous, balanced chunk range [j*C/grid, (j+1)*C/grid); one
+//    sequence: the chunks are dealt round-robin (CTA j: j, j + grid, ...), so
+//    every SM reads from every part of the cache.
 //  * Warp 8 streams K with 3-D TMA boxes {64 channels, T tokens, h_kv heads}
 //    (128-byte swizzle, L2 evict-first) into a ring of stages guarded by
 //    mbarriers.  Before waiting for the previous kernel in the stream it
@@ -34,17 +36,16 @@
 //    columns with tcgen05.ld, frees the accumulator, scales, stores the
 //    logits (a warp writes 32 consecutive tokens of a head: coalesced) and
 //    keeps an online (max, sum exp) per head; when the CTA leaves a sequence
-//    each warp reduces these over its lanes and writes them as its own
-//    partial of each head (R per (CTA, sequence) segment), with no barrier;
-//    they are
-//    reduced over the threads of each head and written as one partial of
-//    head h at slot j + b (CTA j, sequence b).  The slot is unique: along the
-//    chunk order neither j nor b decreases and one of them grows at every new
+//    each warp reduces these over its lanes (integer max of order-preserving
+//    keys, a fixed shuffle tree: deterministic) and writes them, with no
+//    barrier, as its own partial of each head: entry r of slot j + b (CTA j,
+//    sequence b), R entries per slot.  The slot is unique: along the chunk
+//    order neither j nor b decreases and one of them grows at every new
 //    (CTA, sequence) segment.  No fences, atomics or waits on other CTAs;
 //    every wait on a barrier is bounded.
-//  * score_merge (one warp per sequence and head) folds the partials of
-//    CTAs j0..j1, the CTAs that cover the sequence, into L[b, h]: fp32 terms
-//    exp(m - M) <= 1 summed in float64.
+//  * score_merge (one warp per sequence and head) folds the partials of the
+//    CTAs that cover the sequence (j0..j1; every CTA with chunks for one
+//    sequence) into L[b, h]: fp32 terms exp(m - M) <= 1 summed in float64.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
