@@ -19,7 +19,6 @@ constexpr int kScoreMaxStages = 12;
 constexpr int kScoreAccBufs = 4;                // TMEM accumulators in flight
 constexpr size_t kScoreDynSmemBudget = 212 * 1024;   // + the kernel's ~13 KB of static shared memory
 constexpr int kVoteThreads = 256;
-constexpr int kVoteTokensPerBlock = kVoteThreads;   // one token per thread
 constexpr int kSelectThreads = 256;
 constexpr int kSelectTokensPerCta = 2048;     // candidates per selection range
 constexpr int kMaxSelectRanges = 2048;        // ranges per sequence: n <= 4M candidates
