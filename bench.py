@@ -492,6 +492,7 @@ def run_reference(a, d: Dist):
     cfg = W.CONFIGS[a.workload]
     li = W.layer_inputs(cfg, 0, "cpu")
     total = int(li.seq_offsets[-1])
+    lengths = np.diff(li.seq_offsets)
     run, tokens = oracle_layer_step_fn(cfg, li)
     scale = 1.0
     sample = "one whole %s layer-step (%d tokens) per step" % (cfg.name, tokens)
@@ -513,8 +514,9 @@ def run_reference(a, d: Dist):
            "ms_per_step": el / a.steps * 1000.0, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": a.workload, "batch": cfg.batch, "h_q": cfg.h_q, "h_kv": cfg.h_kv,
-                      "head_dim": cfg.head_dim, "n": cfg.n, "k": cfg.k, "n_sink": cfg.n_sink,
-                      "n_local": cfg.n_local},
+                      "head_dim": cfg.head_dim, "n": int(lengths.max()), "tokens_total": total,
+                      "layers": cfg.layers, "k": cfg.k, "n_sink": cfg.n_sink, "n_local": cfg.n_local,
+                      "selection_cache_theta": cfg.theta, "parallelism": "host, one thread (rank 0)"},
            "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
