@@ -58,6 +58,7 @@ CASES = {
     "integer_keys_many_ties": ([2000], 28, 4, 128, 200, 4, 64, {"dist": "int"}),
     "padded_strides": ([3000], 28, 4, 128, 256, 4, 64, {"strides": (4 * 128 * 2 + 64, 256)}),
     "peaked_scores": ([2500], 8, 2, 128, 64, 4, 32, {"scale": 1.0}),
+    "d64_hkv8_g2": ([1500, 77], 16, 8, 64, 100, 4, 32, {"planted": 8}),
     # more than 32 sequences (score pass A's general chunk-table path)
     "batch_40_qwen_heads": ([int(x) for x in np.random.default_rng(40).integers(1, 700, 40)], 28, 4, 128, 64, 4,
                             32, {}),
