@@ -66,6 +66,8 @@ def parse_args(argv=None):
         a.warmup = 3 if a.impl == "reference" else (10 if big else 50)
     if a.warmup < 3:
         raise SystemExit("at least 3 warm-up steps are required")
+    if a.layers is not None and not 1 <= a.layers <= W.CONFIGS[a.workload].layers:
+        raise SystemExit("--layers must be in [1, %d] for %s" % (W.CONFIGS[a.workload].layers, a.workload))
     return a
 
 
@@ -209,9 +211,7 @@ class Workload:
         self.ts = ts
         cfg = W.CONFIGS[name]
         if layers is not None:
-            if not 1 <= layers <= cfg.layers:
-                raise SystemExit("--layers must be in [1, %d] for %s" % (cfg.layers, name))
-            cfg = dataclasses.replace(cfg, layers=layers)
+            cfg = dataclasses.replace(cfg, layers=layers)   # range checked by parse_args
         self.cfg = cfg
         self.name = name
         self.device = device

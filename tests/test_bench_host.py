@@ -1,0 +1,99 @@
+"""Host logic of the benchmark that needs no GPU: argument checks, the clock
+sampler's accept / reject rule (against a fake NVML), the measured-peak and
+ncu-traffic records."""
+import hashlib
+import json
+import os
+import shutil
+import sys
+import time
+import types
+
+import pytest
+
+import bench
+
+
+def test_parse_args_defaults_and_checks():
+    a = bench.parse_args([])
+    assert a.workload == "qwen7b_32k" and a.impl == "ours" and a.warmup >= 3 and a.layers is None
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
+    assert bench.parse_args(["--workload", "qwen7b_1m", "--layers", "1"]).layers == 1
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--workload", "qwen7b_1m", "--layers", "29"])
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--layers", "0"])
+
+
+def test_aggregate_is_units_over_max_time():
+    assert bench.aggregate(100, 4, 2.0) == 200.0
+
+
+def _fake_nvml(mask, mhz, max_mhz):
+    nv = types.ModuleType("pynvml")
+    nv.NVML_CLOCK_SM = 1
+    nv.nvmlInit = lambda: None
+    nv.nvmlDeviceGetHandleByPciBusId = lambda bus: "gpu0"
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, which: max_mhz
+    nv.nvmlDeviceGetClockInfo = lambda h, which: mhz
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: mask
+    return nv
+
+
+@pytest.mark.parametrize("mask,mhz,rejected,reasons", [
+    (0x0, 1965, False, []),                                   # clean run
+    (0x4, 1300, False, ["sw_power_cap"]),                     # power cap: kept and noted
+    (0x8, 1965, True, ["hw_slowdown"]),
+    (0x40, 1965, True, ["hw_thermal_slowdown"]),
+    (0x20, 1965, True, ["sw_thermal_slowdown"]),
+    (0x0, 900, True, []),                                     # far below max with no reason: a clock lock
+])
+def test_clock_sampler_rule(monkeypatch, mask, mhz, rejected, reasons):
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml(mask, mhz, 1965))
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=1, pci_device_id=0)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda i: props)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.02)
+    s = clk.summary()
+    assert s["samples"] > 0 and s["sm_mhz"] == mhz and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == reasons and clk.rejected() == rejected
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    nv = types.ModuleType("pynvml")
+
+    def boom():
+        raise RuntimeError("no driver")
+    nv.nvmlInit = boom
+    monkeypatch.setitem(sys.modules, "pynvml", nv)
+    with bench.ClockSampler(0) as clk:
+        pass
+    assert clk.summary()["reasons"] == ["nvml unavailable"] and not clk.rejected()
+
+
+def test_measured_peak_record():
+    value, kind = bench.measured_hbm_peak()
+    path = os.path.join(bench.ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            assert kind == "measured" and value == float(json.load(f)["hbm_gbs"])
+    else:
+        assert (value, kind) == (bench.FALLBACK_HBM_GBS, "fallback")
+
+
+def test_traffic_record_follows_the_kernel_source(tmp_path):
+    src = os.path.join(bench.ROOT, "query_aware_kv_ts_b200", "csrc", "score.cu")
+    with open(os.path.join(bench.ROOT, "profiles", "score_pass_a_traffic.json")) as f:
+        rec = json.load(f)
+    with open(src, "rb") as f:
+        current = hashlib.sha256(f.read()).hexdigest() == rec["source_sha256"]
+    # the record counts only while the kernel source is the one it was taken on
+    want = rec["per_launch_bytes"]["qwen7b_32k"] if current else None
+    assert bench.profile_traffic(src, "qwen7b_32k") == want
+    assert bench.profile_traffic(src, "no_such_workload") is None
+    changed = tmp_path / "score.cu"
+    shutil.copy(src, changed)
+    with open(changed, "a") as f:
+        f.write("\n// changed\n")
+    assert bench.profile_traffic(str(changed), "qwen7b_32k") is None
