@@ -340,6 +340,49 @@ def cpu_baseline(wl: Workload, budget_s: float):
             "sample": "%d x %s, float64 C oracle, 1 thread, %.1f s" % (n, sample_desc, el)}
 
 
+def usable_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_all_cores(wl, budget_s: float, threads=None):
+    """The same oracle on every usable core: independent layer-steps on as many
+    threads (the oracle's C calls release the interpreter lock, so the threads
+    run in parallel); the oracle itself is unchanged."""
+    cfg = wl.cfg
+    li = wl.layers[0]
+    total = int(li.seq_offsets[-1])
+    run, tokens = oracle_layer_step_fn(cfg, li)
+    scale = 1.0
+    sample_desc = "whole %s layer-steps (%d tokens)" % (cfg.name, tokens)
+    t0 = time.perf_counter()
+    run()
+    if time.perf_counter() - t0 > budget_s / 4:
+        run, tokens = oracle_layer_step_fn(cfg, li, max_tokens=32768)
+        scale = tokens / total
+        sample_desc = "%d-token samples of sequence 0 of %s layer-steps, scaled by tokens" % (tokens, cfg.name)
+    n_threads = threads or usable_cores()
+    counts = [0] * n_threads
+    stop_at = time.perf_counter() + budget_s
+
+    def worker(i):
+        while time.perf_counter() < stop_at:
+            run()
+            counts[i] += 1
+    t0 = time.perf_counter()
+    pool = [threading.Thread(target=worker, args=(i,)) for i in range(n_threads)]
+    for t in pool:
+        t.start()
+    for t in pool:
+        t.join()
+    el = time.perf_counter() - t0
+    n = sum(counts)
+    return {"value": n * scale / el, "unit": "layer-steps/s", "cores": n_threads, "kind": "oracle",
+            "sample": "%d x %s, float64 C oracle, %d threads, %.1f s" % (n, sample_desc, n_threads, el)}
+
+
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
@@ -479,6 +522,7 @@ def run_ours(a, d: Dist):
         result["reuse_rate"] = reuse_rate
     if d.world == 1 and not a.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
+        result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, 4.0)
     del graphs, graphs_n, ga
     d.close()
     if d.rank == 0:

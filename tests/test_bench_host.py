@@ -97,3 +97,20 @@ def test_traffic_record_follows_the_kernel_source(tmp_path):
     with open(changed, "a") as f:
         f.write("\n// changed\n")
     assert bench.profile_traffic(str(changed), "qwen7b_32k") is None
+
+
+def test_all_core_oracle_baseline_runs_threads_in_parallel():
+    """The all-core CPU baseline runs the unchanged oracle on several threads;
+    with two threads it completes more layer-steps per second than with one
+    (the C calls release the interpreter lock)."""
+    import types as _t
+
+    import workloads as W
+    cfg = W.CONFIGS["tiny"]
+    wl = _t.SimpleNamespace(cfg=cfg, layers=[W.layer_inputs(cfg, 0, "cpu")])
+    one = bench.cpu_baseline_all_cores(wl, 1.0, threads=1)
+    two = bench.cpu_baseline_all_cores(wl, 1.0, threads=2)
+    assert one["cores"] == 1 and two["cores"] == 2 and one["kind"] == "oracle"
+    assert "2 threads" in two["sample"]
+    if bench.usable_cores() >= 2:
+        assert two["value"] > 1.3 * one["value"], (one, two)
