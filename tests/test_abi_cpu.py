@@ -113,3 +113,19 @@ def test_decode_step_kernels_rejects_bad_arguments(lib):
     assert lib.ts_decode_step_kernels(None, -1, 4, 8) == -1 and b"non-negative" in lib.ts_last_error()
     assert lib.ts_decode_step_kernels(None, 0, 0, 0) == -1
     assert lib.ts_decode_step_kernels(None, 16, 4, 8) == -1 and b"kv" in lib.ts_last_error()
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU path: the binding refuses host tensors before calling the library."""
+    import torch
+
+    import query_aware_kv_ts_b200 as ts
+    k = torch.zeros((64, 4, 64), dtype=torch.bfloat16)
+    kv = ts.KVCache(k, k.clone(), [0, 64], 8)
+    q = torch.zeros((1, 8, 64), dtype=torch.bfloat16)
+    votes = torch.zeros(64)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="GPU only"):
+        ts.ts_score(kv, q, None, votes, ws)
+    with pytest.raises(ValueError, match="GPU only"):
+        ts.ts_selcache(q, q.clone(), torch.zeros(1, dtype=torch.int32), True, 0.9)
