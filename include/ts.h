@@ -107,8 +107,10 @@ TS_API ts_status_t ts_workspace_init(void *ws, size_t ws_bytes, void *stream);
  * Cache: consecutive similar queries share one token selection).
  * For each sequence b, over the flattened h_q*head_dim query vector:
  *   cos_b    = <q_b, q_prev_b> / (|q_b| |q_prev_b|)     (float64 accumulation)
- *   reuse[b] = !first_step && |q_b| > 0 && |q_prev_b| > 0 && cos_b >= threshold
- * then q_prev_b <- q_b.
+ *              with cos_b = 0 when either vector is zero (no direction)
+ *   reuse[b] = !first_step && cos_b >= threshold
+ * then q_prev_b <- q_b.  (A zero query therefore reuses only when
+ * threshold <= 0.)
  *   q          device bf16 [batch, h_q, head_dim] contiguous
  *   q_prev     device bf16, same shape; caller-owned state, overwritten
  *   reuse      device int32 [batch], written (0/1)
@@ -197,8 +199,13 @@ TS_API ts_status_t ts_sparse_attn(const ts_kv_t *kv, const void *q, const int32_
  *     bytes, splits = ceil(ids_capacity / 64)) are rejected with
  *     TS_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on each device looks the array up (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream
- *     capture.
+ *     with that device current).  Under CUDA's lazy module loading (the
+ *     default) the 4 MiB are committed on a device only when the library's
+ *     code first loads there, at that first call or at the first call of any
+ *     other entry point.  A caller whose memory budget is fixed at start-up
+ *     should therefore make one call per device at start-up, before it takes
+ *     its budget and before any stream capture.  A device reset ends the
+ *     context the address belongs to; the next call looks it up again.
  *   - Every call shares the one array, which keeps the last call's
  *     contents: calls that can overlap on the GPU (on different streams, or
  *     from different threads) race with each other.  Nothing in it has to
@@ -238,7 +245,9 @@ TS_API int32_t ts_decode_step_kernels(const ts_kv_t *kv, int32_t k, int32_t n_si
  * Read and clear the device status word of a workspace (synchronises the
  * stream).  Returns TS_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave
  * up since the last read, TS_OK otherwise.  *site_out (may be NULL) receives
- * a code naming the wait that gave up.
+ * a code naming the wait that gave up.  After TS_ERR_DEVICE_TIMEOUT the
+ * results of every call since the last TS_OK read are void, and so are the
+ * workspace's contents: re-initialise it (ts_workspace_init) before reuse.
  */
 TS_API ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream);
 

@@ -10,6 +10,7 @@
 
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "ts_device.cuh"
 #include "ts_internal.h"
@@ -56,6 +57,53 @@ ts_status_t cuda_fail(cudaError_t e, const char *what)
     return TS_ERR_CUDA;
 }
 }  // namespace
+
+void *current_context()
+{
+    using GetCurrent = CUresult (*)(CUcontext *);
+    static std::once_flag once;
+    static GetCurrent fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrent>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS)
+        return nullptr;
+    return ctx;
+}
+
+cudaError_t ensure_dyn_smem(const void *kernel, int bytes)
+{
+    struct Done {
+        const void *kernel;
+        void *ctx;
+        int bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Done> done;
+    // (no context yet: the attribute is set on every call)
+    void *ctx = current_context();
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Done &d : done)
+        if (d.kernel == kernel && d.ctx == ctx && ctx != nullptr && d.bytes >= bytes)
+            return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return e;
+    if (ctx != nullptr) {
+        for (Done &d : done)
+            if (d.kernel == kernel && d.ctx == ctx) {
+                d.bytes = bytes;
+                return cudaSuccess;
+            }
+        done.push_back({kernel, ctx, bytes});
+    }
+    return cudaSuccess;
+}
 
 bool pdl_enabled()
 {

@@ -358,18 +358,11 @@ template <int D, int NB>
 cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
 {
     constexpr size_t smem = attn_smem_bytes<D, NB>();
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(attn_split<D, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        configured_dev = dev;
-    }
+    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void *>(attn_split<D, NB>), (int)smem);
+    if (e != cudaSuccess)
+        return e;
     dim3 grid((unsigned)p.attn_splits, (unsigned)p.Hkv, (unsigned)p.B);
-    cudaError_t e = launch_ex(attn_split<D, NB>, grid, dim3(kAttnThreads), smem, st, 1, a);
+    e = launch_ex(attn_split<D, NB>, grid, dim3(kAttnThreads), smem, st, 1, a);
     if (e != cudaSuccess)
         return e;
     return launch_ex(attn_merge<D>, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(kAttnThreads), 0, st, 1, a);
@@ -420,11 +413,15 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) uint8_t g_attn_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of the array for the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached together with the context it
+// belongs to: after a device reset the device has a new context, in which the
+// library's module (and the array) is loaded afresh, and the address is
+// looked up again.
 static uint8_t *noalloc_scratch_ptr(ts_status_t *status)
 {
     static std::mutex mu;
     static uint8_t *ptrs[64] = {nullptr};
+    static void *ctxs[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) {
@@ -432,8 +429,9 @@ static uint8_t *noalloc_scratch_ptr(ts_status_t *status)
         *status = TS_ERR_CUDA;
         return nullptr;
     }
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(mu);
-    if (ptrs[dev] == nullptr) {
+    if (ptrs[dev] == nullptr || ctxs[dev] != ctx || ctx == nullptr) {
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_attn_noalloc_scratch);
         if (e != cudaSuccess || ptr == nullptr) {
@@ -442,6 +440,7 @@ static uint8_t *noalloc_scratch_ptr(ts_status_t *status)
             return nullptr;
         }
         ptrs[dev] = static_cast<uint8_t *>(ptr);
+        ctxs[dev] = current_context();
     }
     *status = TS_OK;
     return ptrs[dev];

@@ -445,7 +445,12 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
                     const uint32_t par = ((it / NS) - 1) & 1;
                     if (!mbar_wait_bounded(&sh.empty[s], par, kSpinLimit)) {
                         report_timeout(a.ctrl, kSiteScoreEmpty);
-                        break;   // nothing issued after this: the MMA warp times out on full[] too
+                        // nothing is issued after this (the MMA warp times out
+                        // on full[] too); before leaving, wait (bounded) for the
+                        // tiles already in flight: the last NS issued stages
+                        for (uint32_t j = it > (uint32_t)NS ? it - NS : 0u; j < it; ++j)
+                            (void)mbar_wait_bounded(&sh.full[j % NS], (j / NS) & 1, kSpinLimit);
+                        break;
                     }
                 }
                 mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
@@ -520,8 +525,13 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
             if (lane == 0)
                 umma_commit(&sh.mma_done);
             __syncwarp();
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&sh.mma_done, done_par, kSpinLimit)) && lane == 0)
-                report_timeout(a.ctrl, kSiteScoreMma);
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&sh.mma_done, done_par, kSpinLimit))) {
+                if (lane == 0)
+                    report_timeout(a.ctrl, kSiteScoreMma);
+                // one more bounded wait before TMEM is released under MMAs
+                // that may still be running (the step's results are void)
+                (void)mbar_wait_bounded(&sh.mma_done, done_par, kSpinLimit);
+            }
         }
     } else {
         // ================= epilogue: warps 0-3, one TMEM lane each =========
@@ -677,16 +687,10 @@ cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, ScoreArgs arg
         cols <<= 1;
     args.tmem_cols = cols;
     const size_t dyn = (size_t)ns * p.stage_bytes + q_bytes + 1024;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(score_pass_a<D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(kScoreDynSmemBudget + 1024));
-        if (e != cudaSuccess)
-            return e;
-        configured_dev = dev;
-    }
+    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void *>(score_pass_a<D, GP>),
+                                    (int)(kScoreDynSmemBudget + 1024));
+    if (e != cudaSuccess)
+        return e;
     return launch_ex(score_pass_a<D, GP>, dim3((unsigned)p.score_grid), dim3(kScoreThreads), dyn, st, 1, kmap,
                      args);
 }

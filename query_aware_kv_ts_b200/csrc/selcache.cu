@@ -2,9 +2,10 @@
 // similar queries share one token selection; GrooveSquid summary: the
 // Selection Cache lowers the selection frequency).
 // One block per sequence: float64 cosine of the flattened h_q*d query against
-// the previous step's query, reuse = !first && cos >= threshold, then the
-// current query replaces the previous one.  Each thread overwrites exactly the
-// q_prev elements it read, so no barrier is needed between read and write.
+// the previous step's query (0 when either vector is zero), reuse = !first &&
+// cos >= threshold, then the current query replaces the previous one.  Each
+// thread overwrites exactly the q_prev elements it read, so no barrier is
+// needed between read and write.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 

@@ -94,6 +94,16 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p);
 
 void set_error(const char *fmt, ...);
 
+// The calling thread's current CUDA context (a driver handle), or nullptr when
+// none is current or the driver entry point is unavailable.  Per-device state
+// the library caches (kernel attributes, symbol addresses) is keyed by it, so
+// that a device reset, which ends the context, makes the cache look again.
+void *current_context();
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// context, once per (kernel, context); thread-safe.
+cudaError_t ensure_dyn_smem(const void *kernel, int bytes);
+
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step,
                             int B, int len, double theta, cudaStream_t st);
