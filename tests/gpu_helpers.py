@@ -13,6 +13,8 @@ Tolerances (TokenSelect decode-step parity contract):
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -115,34 +117,82 @@ def check_select_same_precision(v_gpu: np.ndarray, ids_gpu, count_gpu, k, n_sink
     assert np.array_equal(ids_gpu, want), "select differs from the oracle on identical votes"
 
 
-def check_step(case: Case, buf, k, n_sink, n_local, *, reuse=None, prev_ids=None, ref=None):
-    """Compare one GPU layer-step with the oracle, sequence by sequence.
+def host_results(buf) -> dict:
+    """Host copies of one layer-step's results (votes, ids, count, out, reuse,
+    cos), taken right after the step so the device buffers can be reused."""
+    return {n: getattr(buf, n).cpu().numpy().copy() for n in ("votes", "ids", "count", "out", "reuse", "cos")}
+
+
+def check_arrays(kb, vb, off, qb, res: dict, k, n_sink, n_local, *, scale=None, reuse=None, prev_ids=None):
+    """Compare one layer-step's host results with the oracle, sequence by
+    sequence.  kb, vb: uint16 [sum_n, h_kv, d]; off: int64 [B+1]; qb: uint16
+    [B, h_q, d]; res: host_results().  A sequence with reuse[b] set must have
+    kept prev_ids[b]; any other is scored and selected again by the oracle.
     Returns a dict of diagnostics (max vote error, set differences)."""
-    votes = buf.votes.cpu().numpy()
-    ids = buf.ids.cpu().numpy()
-    count = buf.count.cpu().numpy()
-    out = buf.out.cpu().numpy()
-    qb = W.bf16_bits(case.q)
+    votes, ids, count, out = res["votes"], res["ids"], res["count"], res["out"]
+    h_q = qb.shape[1]
     diag = {"max_vote_rel": 0.0, "set_diffs": 0, "max_out_err": 0.0}
-    for b in range(case.B):
-        lo, hi = case.seq(b)
+    for b in range(off.size - 1):
+        lo, hi = int(off[b]), int(off[b + 1])
         n = hi - lo
-        kb, vb = case.kb[lo:hi], case.vb[lo:hi]
+        kbb, vbb = kb[lo:hi], vb[lo:hi]
         if reuse is not None and reuse[b]:
             assert np.array_equal(ids[b], prev_ids[b]), "reused sequence changed its ids"
         else:
-            v_ref, _ = oracle.votes(kb, qb[b], case.oracle_scale())
-            rel = check_votes(votes[lo:hi], v_ref, case.h_q)
+            v_ref, _ = oracle.votes(kbb, qb[b], scale)
+            rel = check_votes(votes[lo:hi], v_ref, h_q)
             diag["max_vote_rel"] = max(diag["max_vote_rel"], rel)
             ids_ref, m_ref = oracle.select(v_ref, k, n_sink, n_local)
             diag["set_diffs"] += check_ids(ids[b], int(count[b]), ids_ref, m_ref, v_ref, n, k, n_sink, n_local)
             check_select_same_precision(votes[lo:hi], ids[b], int(count[b]), k, n_sink, n_local)
         m_b = int(count[b])
-        o_ref = oracle.sparse_attn(kb, vb, qb[b], ids[b], m_b, case.oracle_scale())
+        o_ref = oracle.sparse_attn(kbb, vbb, qb[b], ids[b], m_b, scale)
         err = float(np.abs(out[b] - o_ref).max()) if o_ref.size else 0.0
         assert err <= OUT_ATOL, "attention output off by %.3g (sequence %d)" % (err, b)
         diag["max_out_err"] = max(diag["max_out_err"], err)
     return diag
+
+
+def check_step(case: Case, buf, k, n_sink, n_local, *, reuse=None, prev_ids=None, ref=None):
+    """Compare one GPU layer-step with the oracle, sequence by sequence.
+    Returns a dict of diagnostics (max vote error, set differences)."""
+    return check_arrays(case.kb, case.vb, case.off, W.bf16_bits(case.q), host_results(buf), k, n_sink, n_local,
+                        scale=case.oracle_scale(), reuse=reuse, prev_ids=prev_ids)
+
+
+class OracleChecks:
+    """Oracle comparisons run on host threads while the GPU goes on (the
+    oracle's C calls release the interpreter lock).  At most `in_flight`
+    checks are queued at once, which bounds the host memory their inputs hold.
+    join() waits for all of them and re-raises the first failure."""
+
+    def __init__(self, in_flight: int | None = None):
+        import concurrent.futures as cf
+        import threading
+        try:
+            cores = len(os.sched_getaffinity(0))
+        except AttributeError:
+            cores = os.cpu_count() or 1
+        self.workers = max(1, cores)
+        self._pool = cf.ThreadPoolExecutor(max_workers=self.workers)
+        self._slots = threading.BoundedSemaphore(in_flight or 2 * self.workers)
+        self._futures = []
+
+    def submit(self, fn, *args, **kw):
+        self._slots.acquire()
+
+        def run():
+            try:
+                return fn(*args, **kw)
+            finally:
+                self._slots.release()
+        self._futures.append(self._pool.submit(run))
+
+    def join(self) -> list:
+        try:
+            return [f.result() for f in self._futures]
+        finally:
+            self._pool.shutdown(wait=True)
 
 
 def config_case(cfg: W.Config, layer=0, step=0, n_override=None, device="cuda"):

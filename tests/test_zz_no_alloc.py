@@ -64,3 +64,33 @@ def test_noalloc_rejects_oversize_shapes():
         m.ts_sparse_attn_noalloc(kv, q, ids, count, out)
     assert e.value.status == m.TS_ERR_UNSUPPORTED
     assert "4194304" in str(e.value)
+
+
+def _scratch_bytes(B, h_kv, G, d, cap):
+    # split-K partials: one (d + 4)-float row per (sequence, kv head, split, head)
+    return B * h_kv * -(-cap // 64) * G * (d + 4) * 4
+
+
+def test_noalloc_scratch_limit_boundary():
+    """Either side of the 4 MiB limit, through the C ABI: 2 sequences, one kv
+    head of 16 query heads, d = 128; an ids row of 15872 needs 248 splits
+    (4,190,208 bytes: accepted, and equal to the workspace attention), one more
+    id needs 249 (4,207,104 bytes: rejected before anything is launched)."""
+    m = H.ts()
+    limit = 4 << 20
+    assert _scratch_bytes(2, 1, 16, 128, 15872) <= limit < _scratch_bytes(2, 1, 16, 128, 15873)
+    case, buf = _case([20000, 16000], 16, 1, 128, 15872 - 4 - 64, 4, 64, seed=11)
+    assert buf.ids.shape == (2, 15872)
+    out = torch.full_like(buf.out, float("nan"))
+    m.ts_sparse_attn_noalloc(case.kv, case.q, buf.ids, buf.count, out)
+    torch.cuda.synchronize()
+    assert (out - buf.out).abs().max().item() <= H.OUT_ATOL
+    wide = torch.full((2, 15873), -1, dtype=torch.int32, device="cuda")
+    wide[:, :15872] = buf.ids
+    out2 = torch.full_like(buf.out, float("nan"))
+    with pytest.raises(m.TsError) as e:
+        m.ts_sparse_attn_noalloc(case.kv, case.q, wide, buf.count, out2)
+    assert e.value.status == m.TS_ERR_UNSUPPORTED
+    assert str(_scratch_bytes(2, 1, 16, 128, 15873)) in str(e.value)
+    torch.cuda.synchronize()
+    assert torch.isnan(out2).all(), "a rejected call must not launch"
