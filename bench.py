@@ -7,10 +7,19 @@ One step = one pass of the whole decode hot path over one batch of synthetic
 input, for every layer of the workload: selection-cache decision (ts_selcache),
 soft vote (ts_score), top-k + sink/local selection (ts_select) and attention
 over the selected tokens (ts_sparse_attn), all through the C ABI.  The default
-workload is the Qwen2-7B-shaped single layer (B=1, h_q=28, h_kv=4, d=128,
-n=32768, k=2048 + 4 sink + 512 local).  Every step is replayed from CUDA graphs;
+workload is the largest one that fits one GPU: the 1M-token decode step over
+all 28 layers of a Qwen2-7B-shaped model (B=1, h_q=28, h_kv=4, d=128,
+n=1048576 per layer, k=4096 + 4 sink + 1024 local, selection cache with cosine
+threshold 0.9 over 16 AR(1) queries).  Every step is replayed from CUDA graphs;
 inputs rotate over enough copies of the KV cache that each step reads data
-that is not in L2.
+that is not in L2 (at 1M tokens one step reads 28 GiB of K: no copies needed).
+
+Two rooflines are reported.  `roofline` is the dominant kernel, score pass A
+(the K scan), timed alone.  `step_roofline` is the whole step: the algorithmic
+bytes of the timed steps (K of every layer-step whose selection was computed
+afresh, plus the gathered K and V rows of every layer-step) over the timed
+region's duration; which layer-steps reused their selection is read back from
+a replay of exactly the timed sequence of steps.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 (the path has no cross-sequence exchange); the timed region is bracketed by
@@ -51,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", default="qwen7b_32k", choices=W.ORDER)
+    ap.add_argument("--workload", default="qwen7b_1m", choices=W.ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -293,6 +302,18 @@ def time_graphs(graphs, K, W_, inner=1, singles=None):
     return s.elapsed_time(e) / 1000.0, reps * inner + rest
 
 
+def replay_order(n_graphs, K, W_, inner, n_singles):
+    """Step indices that time_graphs(graphs, K, W_, inner, singles) runs, in
+    order: (warm-up steps, timed steps), for graphs of `inner` consecutive
+    steps (graph j: steps j*inner .. j*inner + inner - 1) and single-step
+    graphs (graph j: step j)."""
+    reps, rest = divmod(K, inner)
+    warm = [(i % n_graphs) * inner + r for i in range(max(1, -(-W_ // inner))) for r in range(inner)]
+    timed = [(i % n_graphs) * inner + r for i in range(reps) for r in range(inner)]
+    timed += [(reps * inner + i) % n_singles for i in range(rest)]
+    return warm, timed
+
+
 # ---------------------------------------------------------------------------
 # CPU baseline: the oracle, as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
@@ -407,9 +428,16 @@ def run_ours(a, d: Dist):
     graphs_n = wl.capture(wl.step, max(1, wl.period // inner), inner)
 
     # ---- main timed region: whole steps ----
+    # every layer starts from an empty selection-cache state (first step
+    # recomputes), as the record pass below does
+    for b in wl.bufs:
+        b.q_prev.zero_()
     d.barrier()
     torch.cuda.synchronize()
     for attempt in range(2):
+        if attempt:
+            for b in wl.bufs:
+                b.q_prev.zero_()
         with ClockSampler(d.local) as clk:
             el, steps_run = time_graphs(graphs_n, a.steps, a.warmup, inner, graphs)
         if not clk.rejected():
@@ -470,17 +498,31 @@ def run_ours(a, d: Dist):
     e2e_el = d.max(time.perf_counter() - t0)
     e2e_value = aggregate(K_e2e * cfg.layers, d.world, e2e_el)
 
-    # reuse rate over one pass of the query sequence (selection-cache workloads)
-    reuse_rate = None
-    if cfg.theta is not None:
-        flags = []
-        for b in wl.bufs:
-            b.q_prev.zero_()
-        for i in range(wl.T):
-            for layer in range(cfg.layers):
-                wl.layer_step(layer, i)
-                flags.append(wl.bufs[layer].reuse.clone())
-        reuse_rate = float(torch.stack(flags).float().mean().item())
+    # which layer-steps of the timed region reused their selection: replay the
+    # same sequence of steps from the same empty state with single-step graphs
+    # and read every layer's reuse flags after each timed step
+    warm_idx, timed_idx = replay_order(len(graphs_n), steps_run, a.warmup, inner, len(graphs))
+    assert len(timed_idx) == steps_run
+    flags = torch.zeros((steps_run, cfg.layers, cfg.batch), dtype=torch.int32, device=dev)
+    for b in wl.bufs:
+        b.q_prev.zero_()
+    for j in warm_idx:
+        graphs[j % len(graphs)].replay()
+    for t, j in enumerate(timed_idx):
+        graphs[j % len(graphs)].replay()
+        for layer in range(cfg.layers):
+            flags[t, layer].copy_(wl.bufs[layer].reuse)
+    torch.cuda.synchronize()
+    flags_np = flags.cpu().numpy().astype(bool)
+    reuse_rate = float(flags_np.mean()) if cfg.theta is not None else None
+    # algorithmic bytes of the timed steps: K of each (layer-step, sequence)
+    # scored afresh, gathered K and V rows of every one
+    row_bytes = cfg.h_kv * cfg.head_dim * 2
+    m_b = np.minimum(wl.lengths, cfg.k + cfg.n_sink + cfg.n_local)
+    k_part = int(((~flags_np) * (wl.lengths * row_bytes)[None, None, :]).sum())
+    gather_part = int(m_b.sum()) * row_bytes * 2 * cfg.layers * steps_run
+    step_alg_bytes = k_part + gather_part
+    step_hbm_gbs = step_alg_bytes / el_max / 1e9
 
     # every layer-step is one ts_decode_step call (the same shapes in every layer)
     kernels_per_layer_step = ts.ts_decode_step_kernels(wl.kvs[0][0], cfg.k, cfg.n_sink, cfg.n_local)
@@ -505,8 +547,14 @@ def run_ours(a, d: Dist):
                    "l2": "inputs larger than L2: %d rotating KV copies, %.0f MiB of K read per rotation"
                          % (wl.rotate, wl.rotate * wl.k_bytes * cfg.layers / 2**20),
                    "graphs": "C-ABI calls captured in CUDA graphs of %d consecutive steps" % inner},
-        "step_hbm_gbs": alg_bytes / (el_max / a.steps) / 1e9 if cfg.theta is None else None,
-        "step_alg_bytes": alg_bytes,
+        "step_hbm_gbs": step_hbm_gbs,
+        "step_alg_bytes": step_alg_bytes / steps_run,
+        "step_roofline": {"bound": "hbm", "scope": "whole decode step (all layers): K of the layer-steps "
+                          "scored afresh + gathered K/V rows of every layer-step, over the timed region",
+                          "achieved": step_hbm_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                          "frac": step_hbm_gbs / peak, "alg_bytes_per_step": step_alg_bytes / steps_run,
+                          "alg_bytes_no_reuse_per_step": alg_bytes,
+                          "k_scored_fraction": float((~flags_np).mean())},
         "roofline": {"bound": "hbm", "kernel": "score pass A (ts_score_logits)", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "alg_bytes_per_launch": wl.k_bytes,
@@ -515,7 +563,7 @@ def run_ours(a, d: Dist):
         "e2e": {"value": e2e_value, "unit": "layer-steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "pinned host query copied in, graph of the C-ABI calls replayed, fp32 output copied "
                        "out and synchronised, every step; host wall clock"},
-        "gpu_launches": a.steps * cfg.layers * kernels_per_layer_step,
+        "gpu_launches": steps_run * cfg.layers * kernels_per_layer_step,
         "clocks": clk.summary(),
     }
     if reuse_rate is not None:

@@ -16,7 +16,7 @@ import bench
 
 def test_parse_args_defaults_and_checks():
     a = bench.parse_args([])
-    assert a.workload == "qwen7b_32k" and a.impl == "ours" and a.warmup >= 3 and a.layers is None
+    assert a.workload == "qwen7b_1m" and a.impl == "ours" and a.warmup >= 3 and a.layers is None
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
     assert bench.parse_args(["--workload", "qwen7b_1m", "--layers", "1"]).layers == 1
@@ -24,6 +24,39 @@ def test_parse_args_defaults_and_checks():
         bench.parse_args(["--workload", "qwen7b_1m", "--layers", "29"])
     with pytest.raises(SystemExit):
         bench.parse_args(["--layers", "0"])
+
+
+class _FakeEvent:
+    def __init__(self, **kw):
+        pass
+
+    def record(self):
+        pass
+
+    def elapsed_time(self, other):
+        return 1.0
+
+
+@pytest.mark.parametrize("n_graphs,K,W_,inner,n_singles", [
+    (1, 20, 5, 1, 16), (16, 20, 5, 1, 16), (1, 50, 5, 16, 16), (2, 37, 50, 8, 16), (4, 3, 3, 4, 16)])
+def test_replay_order_matches_time_graphs(monkeypatch, n_graphs, K, W_, inner, n_singles):
+    """The record pass replays exactly the steps the timed region ran."""
+    ran = []
+
+    class G:
+        def __init__(self, steps):
+            self.steps = steps
+
+        def replay(self):
+            ran.extend(self.steps)
+    graphs = [G([j * inner + r for r in range(inner)]) for j in range(n_graphs)]
+    singles = [G([j]) for j in range(n_singles)]
+    monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda: None)
+    monkeypatch.setattr(bench.torch.cuda, "Event", _FakeEvent)
+    _, steps_run = bench.time_graphs(graphs, K, W_, inner, singles)
+    warm, timed = bench.replay_order(n_graphs, K, W_, inner, n_singles)
+    assert steps_run == K == len(timed)
+    assert ran == warm + timed
 
 
 def test_aggregate_is_units_over_max_time():
