@@ -194,10 +194,12 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic(kernel_src: str, workload: str):
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "score_pass_a_traffic.json")
+
+
+def profile_traffic(kernel_src: str, workload: str, path: str = TRAFFIC_RECORD):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
     or None when the kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "score_pass_a_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -448,32 +450,37 @@ def run_ours(a, d: Dist):
     value = aggregate(layer_steps, d.world, el_max)
     ms_per_step = el_max / steps_run * 1000.0
 
-    # ---- dominant kernel alone: score pass A (all sequences scored) ----
-    def pass_a(i):
-        for layer in range(cfg.layers):
-            ts.ts_score_logits(wl.kvs[layer][i % wl.rotate], wl.q[layer][i % wl.T], None, wl.bufs[layer].ws)
-    ga = wl.capture(pass_a, 1, wl.rotate)
+    # ---- dominant kernel alone: score pass A (ts_score_logits: the K scan,
+    #      every sequence scored) ----
     Ka = max(a.steps, 20)
-    el_a, ka_run = time_graphs(ga, Ka, a.warmup, wl.rotate)
-    per_launch_s = el_a / (ka_run * cfg.layers)
+
+    def one(fn):
+        g = wl.capture(fn, 1, wl.rotate)
+        el_k, k_run = time_graphs(g, Ka, a.warmup, wl.rotate)
+        return el_k / (k_run * cfg.layers)
+    per_launch_s = one(lambda i: [ts.ts_score_logits(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T], None,
+                                                     wl.bufs[l].ws) for l in range(cfg.layers)])
     peak, peak_kind = measured_hbm_peak()
     achieved = wl.k_bytes / per_launch_s / 1e9
     traffic = profile_traffic(os.path.join(ROOT, "query_aware_kv_ts_b200", "csrc", "score.cu"), a.workload)
 
-    # per-kernel breakdown (each kernel alone, same rotation)
-    def one(fn):
-        g = wl.capture(fn, 1, wl.rotate)
-        el_k, k_run = time_graphs(g, Ka, a.warmup, wl.rotate)
-        return el_k / (k_run * cfg.layers) * 1e6
+    # per-kernel breakdown (each kernel alone, same rotation), with the fused
+    # one-kernel scoring beside the two passes
     kernels = {"score_pass_a_us": per_launch_s * 1e6}
-    kernels["score_pass_b_us"] = one(lambda i: [ts.ts_score_vote(wl.kvs[l][i % wl.rotate], None, wl.bufs[l].votes,
-                                                                 wl.bufs[l].ws) for l in range(cfg.layers)])
-    kernels["select_us"] = one(lambda i: [ts.ts_select(wl.kvs[l][i % wl.rotate], wl.bufs[l].votes, cfg.k, cfg.n_sink,
-                                                       cfg.n_local, None, wl.bufs[l].ids, wl.bufs[l].count,
-                                                       wl.bufs[l].ws) for l in range(cfg.layers)])
-    kernels["sparse_attn_us"] = one(lambda i: [ts.ts_sparse_attn(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T],
-                                                                 wl.bufs[l].ids, wl.bufs[l].count, wl.bufs[l].out,
-                                                                 wl.bufs[l].ws) for l in range(cfg.layers)])
+    kernels["score_pass_b_us"] = 1e6 * one(
+        lambda i: [ts.ts_score_vote(wl.kvs[l][i % wl.rotate], None, wl.bufs[l].votes, wl.bufs[l].ws)
+                   for l in range(cfg.layers)])
+    kernels["score_fused_us"] = 1e6 * one(
+        lambda i: [ts.ts_score_fused(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T], None, wl.bufs[l].votes,
+                                     wl.bufs[l].ws) for l in range(cfg.layers)])
+    kernels["select_us"] = 1e6 * one(lambda i: [ts.ts_select(wl.kvs[l][i % wl.rotate], wl.bufs[l].votes, cfg.k,
+                                                             cfg.n_sink, cfg.n_local, None, wl.bufs[l].ids,
+                                                             wl.bufs[l].count, wl.bufs[l].ws)
+                                                for l in range(cfg.layers)])
+    kernels["sparse_attn_us"] = 1e6 * one(lambda i: [ts.ts_sparse_attn(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T],
+                                                                       wl.bufs[l].ids, wl.bufs[l].count,
+                                                                       wl.bufs[l].out, wl.bufs[l].ws)
+                                                     for l in range(cfg.layers)])
 
     # ---- end to end: pinned host query in, result out, every step ----
     q_host = [q.cpu().pin_memory() for q in wl.q]
@@ -524,8 +531,14 @@ def run_ours(a, d: Dist):
     step_alg_bytes = k_part + gather_part
     step_hbm_gbs = step_alg_bytes / el_max / 1e9
 
-    # every layer-step is one ts_decode_step call (the same shapes in every layer)
+    # every layer-step is one ts_decode_step call (the same shapes in every
+    # layer); replayed from a graph, a layer-step in which every sequence
+    # reuses its selection skips the scoring and selection kernels (the cosine
+    # test and the two attention kernels run)
     kernels_per_layer_step = ts.ts_decode_step_kernels(wl.kvs[0][0], cfg.k, cfg.n_sink, cfg.n_local)
+    skip_on = cfg.theta is not None and os.environ.get("TS_NO_REUSE_SKIP") != "1"
+    all_reused = flags_np.all(axis=2) if skip_on else np.zeros(flags_np.shape[:2], bool)
+    gpu_launches = int(np.where(all_reused, 3, kernels_per_layer_step).sum())
     alg_bytes = wl.k_rows_bytes() * cfg.layers
     result = {
         "metric": "decode layer-steps/s (score+select+sparse-attn); HBM GB/s vs roofline",
@@ -563,7 +576,7 @@ def run_ours(a, d: Dist):
         "e2e": {"value": e2e_value, "unit": "layer-steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "pinned host query copied in, graph of the C-ABI calls replayed, fp32 output copied "
                        "out and synchronised, every step; host wall clock"},
-        "gpu_launches": steps_run * cfg.layers * kernels_per_layer_step,
+        "gpu_launches": gpu_launches,
         "clocks": clk.summary(),
     }
     if reuse_rate is not None:
@@ -571,7 +584,7 @@ def run_ours(a, d: Dist):
     if d.world == 1 and not a.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, 4.0)
-    del graphs, graphs_n, ga
+    del graphs, graphs_n
     d.close()
     if d.rank == 0:
         print(json.dumps(result), flush=True)

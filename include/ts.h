@@ -152,6 +152,21 @@ TS_API ts_status_t ts_score_vote(const ts_kv_t *kv, const int32_t *reuse, float 
                                  void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The soft vote of ts_score (same definition, arguments, workspace and
+ * errors) from one cooperative kernel instead of two passes: the kv heads are
+ * scored a few at a time (as many as keep one pass's logits within 32 MB of
+ * L2), and each pass's normalisers and votes are taken while the next pass
+ * streams K, with the logit lines dropped from L2 once read.  The votes equal
+ * ts_score's up to rounding (a few 1e-7 relative: the normalisers are merged
+ * in another order).  The kernel needs every CTA of its grid resident (one
+ * per SM); it synchronises them with counters in the workspace's control
+ * block, which it returns to zero.  ts_score and ts_decode_step use the
+ * two-pass kernels, which are faster on B200 at every workload measured.
+ */
+TS_API ts_status_t ts_score_fused(const ts_kv_t *kv, const void *q, const int32_t *reuse, float *votes,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Token selection (TokenSelect README summary: a small number of critical KV
  * tokens take part in attention).  For every sequence b with reuse[b] == 0:
  *   sink  = [0, s')         s' = min(n_sink, n_b)
@@ -223,6 +238,13 @@ TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, cons
  * the selection's first-level vote histogram, which ts_select otherwise builds
  * in a kernel of its own (ts_decode_step_kernels gives the count).  Every
  * argument is checked before the first launch.
+ *   Under stream capture with the selection cache able to reuse (first_step
+ *   0, threshold <= 1), the scoring and selection kernels are captured into
+ *   the body of a conditional graph node that the cosine kernel switches
+ *   off when every sequence reuses: such a replayed step runs 3 kernels (the
+ *   cosine test and the two attention kernels).  The results are the same
+ *   either way.  The body is captured on a stream the library creates once
+ *   per context; TS_NO_REUSE_SKIP=1 in the environment turns this off.
  *   reuse      device int32 [batch], required: written by the selection cache
  *              and read by every later phase (sequences that reuse keep their
  *              previous ids and count; their votes are left as they were)

@@ -62,6 +62,7 @@ _SIGS = {
     "ts_score": (ctypes.c_int, [_KV, _P, _P, _P, _P, _SZ, _P]),
     "ts_score_logits": (ctypes.c_int, [_KV, _P, _P, _P, _SZ, _P]),
     "ts_score_vote": (ctypes.c_int, [_KV, _P, _P, _P, _SZ, _P]),
+    "ts_score_fused": (ctypes.c_int, [_KV, _P, _P, _P, _P, _SZ, _P]),
     "ts_select": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "ts_sparse_attn": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
     "ts_sparse_attn_noalloc": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P]),
@@ -166,6 +167,13 @@ def ts_score(kv: KVCache, q, reuse, votes, ws, stream=None):
 def ts_score_logits(kv: KVCache, q, reuse, ws, stream=None):
     _check(_lib.ts_score_logits(kv.ref(), _ptr(q), _ptr(reuse), _ptr(ws), ws.numel() * ws.element_size(),
                                 _stream(stream)))
+
+
+def ts_score_fused(kv: KVCache, q, reuse, votes, ws, stream=None):
+    """The same votes as ts_score from one cooperative kernel that scores a few
+    kv heads per pass and takes each pass's votes while its logits are in L2."""
+    _check(_lib.ts_score_fused(kv.ref(), _ptr(q), _ptr(reuse), _ptr(votes), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def ts_score_vote(kv: KVCache, reuse, votes, ws, stream=None):

@@ -105,6 +105,42 @@ cudaError_t ensure_dyn_smem(const void *kernel, int bytes)
     return cudaSuccess;
 }
 
+// Graph replays of ts_decode_step skip the scoring and selection kernels of
+// a step in which every sequence reuses its selection, unless the
+// environment sets TS_NO_REUSE_SKIP=1.
+static bool reuse_skip_enabled()
+{
+    static const bool on = [] {
+        const char *e = getenv("TS_NO_REUSE_SKIP");
+        return !(e != nullptr && e[0] == '1');
+    }();
+    return on;
+}
+
+// A non-blocking stream of the current context on which the body of a
+// conditional graph node is captured (the caller's stream is capturing the
+// enclosing graph).  Created at the first use in a context, kept for the
+// process's lifetime.
+static cudaError_t body_stream(cudaStream_t *out)
+{
+    static std::mutex mu;
+    static std::vector<std::pair<void *, cudaStream_t>> streams;
+    void *ctx = current_context();
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto &e : streams)
+        if (e.first == ctx && ctx != nullptr) {
+            *out = e.second;
+            return cudaSuccess;
+        }
+    cudaStream_t st = nullptr;
+    const cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+    if (e != cudaSuccess)
+        return e;
+    streams.push_back({ctx, st});
+    *out = st;
+    return cudaSuccess;
+}
+
 bool pdl_enabled()
 {
     static const bool on = [] {
@@ -231,6 +267,28 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
         p->score_partials_per_slot = 2 * qph;
     }
     p->ld_logits = (n_total + 3) / 4 * 4;
+    {
+        // fused scoring: HS kv heads per pass, the largest of 4, 2, 1 that
+        // divides h_kv and whose logits (HS * G * n_total * 4 bytes) fit the
+        // L2 share a pass may keep; GP rows per kv head in the staged queries
+        // (HS * GP >= 8 keeps every pass's first row on a 1024-byte atom)
+        int hs = 4;
+        while (hs > 1 && (kv->h_kv % hs != 0 || (double)hs * G * (double)n_total * 4.0 > (double)kFusedPassLogitsBytes))
+            hs >>= 1;
+        int gp = 4;
+        while (gp < G || hs * gp < 8)
+            gp <<= 1;
+        p->fused_hs = hs;
+        p->fused_gp = gp;
+        p->fused_t = kFusedRows / hs;
+        p->fused_n = hs * gp < 16 ? 16 : hs * gp;
+        int64_t fc = 0;
+        for (int b = 0; b < kv->batch; ++b)
+            fc += (off[b + 1] - off[b] + p->fused_t - 1) / p->fused_t;
+        p->fused_chunks = fc;
+        p->fused_grid = (int)(fc < grid_cap ? fc : grid_cap);
+        p->fused_ld = fc * p->fused_t;
+    }
     p->sel_ranges = (int)((n_max + kSelectTokensPerCta - 1) / kSelectTokensPerCta) + 1;
     p->capacity = capacity;
     if (capacity > kMaxCapacity) {
@@ -252,8 +310,13 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->off_L = o;
     o = align_up(o + sizeof(double) * p->B * p->Hq, 256);
     p->off_partials = o;
-    o = align_up(o + sizeof(float) * 2 * (size_t)(p->score_grid + p->B) * p->score_partials_per_slot * p->Hq,
-                 256);
+    {
+        // the two-phase pass A keeps R partials per (CTA, sequence) slot and
+        // head, the fused kernel one
+        const size_t two_phase = (size_t)(p->score_grid + p->B) * p->score_partials_per_slot;
+        const size_t fused = (size_t)(p->fused_grid + p->B);
+        o = align_up(o + sizeof(float) * 2 * (two_phase > fused ? two_phase : fused) * p->Hq, 256);
+    }
     p->off_sel_inb1 = o;
     o = align_up(o + sizeof(uint32_t) * (size_t)p->B * p->sel_ranges, 256);
     p->off_sel_bin = o;
@@ -269,7 +332,15 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->off_sel_hist = o;
     o = align_up(o + sizeof(uint32_t) * 4096 * (size_t)p->B, 256);
     p->off_logits = o;
-    o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(p->ld_logits > 0 ? p->ld_logits : 4), 256);
+    {
+        // two-phase rows of ld_logits tokens; fused rows of fused_ld (chunk-padded)
+        const int64_t ld = p->ld_logits > p->fused_ld ? p->ld_logits : p->fused_ld;
+        o = align_up(o + sizeof(float) * (size_t)p->Hq * (size_t)(ld > 0 ? ld : 4), 256);
+    }
+    // the fused scoring's running votes between passes, chunk-aligned like
+    // its logits (16-byte aligned lines for bulk copies)
+    p->off_vacc = o;
+    o = align_up(o + sizeof(float) * (size_t)(p->fused_ld > 0 ? p->fused_ld : 4), 256);
     p->off_sel_cand = o;
     o = align_up(o + 8 * nt1, 256);
     // last: the only part whose size depends on the selection capacity, so
@@ -298,7 +369,11 @@ static ts_status_t check_ws(const Plan &p, void *ws, size_t ws_bytes)
     return TS_OK;
 }
 
-static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *map)
+// K as a 3-D tensor (channels, tokens, kv heads) for TMA.  fused: boxes of
+// {64, T, HS} (the fused scoring kernel, HS kv heads of T = 128 / HS tokens
+// per stage); else {64, T, h_kv} (the two-phase pass A, every head of
+// T = 128 / h_kv tokens per stage).
+static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *map, bool fused = false)
 {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (enc == nullptr) {
@@ -308,7 +383,8 @@ static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *ma
     // dims (innermost first): channels, tokens, kv heads
     cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.n_total, (cuuint64_t)p.Hkv};
     cuuint64_t strides[2] = {(cuuint64_t)kv->stride_tok * 2, (cuuint64_t)kv->stride_head * 2};
-    cuuint32_t box[3] = {64u, (cuuint32_t)p.tile_tokens, (cuuint32_t)p.Hkv};
+    cuuint32_t box[3] = {64u, fused ? (cuuint32_t)p.fused_t : (cuuint32_t)p.tile_tokens,
+                         fused ? (cuuint32_t)p.fused_hs : (cuuint32_t)p.Hkv};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(kv->k), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -439,6 +515,32 @@ ts_status_t ts_score(const ts_kv_t *kv, const void *q, const int32_t *reuse, flo
     return ts_score_vote(kv, reuse, votes, ws, ws_bytes, stream);
 }
 
+ts_status_t ts_score_fused(const ts_kv_t *kv, const void *q, const int32_t *reuse, float *votes, void *ws,
+                           size_t ws_bytes, void *stream)
+{
+    Plan p;
+    ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
+    if (s != TS_OK)
+        return s;
+    if (votes == nullptr) {
+        set_error("votes is required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15u)) {
+        set_error("q is required and must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (p.n_total == 0)
+        return TS_OK;
+    CUtensorMap kmap;
+    s = encode_kmap(p, kv, &kmap, true);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_score_fused(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, votes,
+                                      static_cast<uint8_t *>(ws), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "fused scoring launch");
+}
+
 ts_status_t ts_select(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink, int32_t n_local,
                       const int32_t *reuse, int32_t *ids, int32_t *count, void *ws, size_t ws_bytes, void *stream)
 {
@@ -512,6 +614,68 @@ ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, const int32
     return launch_attn_noalloc(p, kv, q, ids, count, out, static_cast<cudaStream_t>(stream));
 }
 
+// ts_decode_step under stream capture with the selection cache able to
+// reuse: cosine test -> IF (condition) { scoring, selection } -> attention.  The condition is 1 at every launch of the graph; the cosine
+// kernel sets it to 0 when every sequence reuses, and the body then does not
+// run at all (its kernels would only have read the flags and returned).
+static ts_status_t decode_step_graph(const Plan &p, const CUtensorMap &kmap, const ts_kv_t *kv, const void *q,
+                                     void *q_prev, int32_t *reuse, double *cos_out, double threshold, int32_t k,
+                                     int32_t n_sink, int32_t n_local, float *votes, int32_t *ids, int32_t *count,
+                                     float *out, uint8_t *w, cudaStream_t st, cudaGraph_t graph)
+{
+    cudaGraphConditionalHandle handle;
+    cudaError_t e = cudaGraphConditionalHandleCreate(&handle, graph, 1u, cudaGraphCondAssignDefault);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: conditional handle");
+    SelcacheSkip skip;
+    skip.handle = handle;
+    skip.counters = reinterpret_cast<uint32_t *>(w + p.off_ctrl) + kCtrlSkipCounters;
+    skip.enabled = 1;
+    e = launch_selcache(q, q_prev, reuse, cos_out, 0, p.B, p.Hq * p.D, threshold, st, &skip);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: selection cache launch");
+    cudaStreamCaptureStatus cap;
+    const cudaGraphNode_t *deps = nullptr;
+    size_t ndeps = 0;
+    e = cudaStreamGetCaptureInfo(st, &cap, nullptr, &graph, &deps, &ndeps);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: capture dependencies");
+    cudaGraphNodeParams np = {};
+    np.type = cudaGraphNodeTypeConditional;
+    np.conditional.handle = handle;
+    np.conditional.type = cudaGraphCondTypeIf;
+    np.conditional.size = 1;
+    cudaGraphNode_t cond_node;
+    e = cudaGraphAddNode(&cond_node, graph, deps, ndeps, &np);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: conditional node");
+    cudaGraph_t body = np.conditional.phGraph_out[0];
+    cudaStream_t side;
+    e = body_stream(&side);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: body capture stream");
+    e = cudaStreamBeginCaptureToGraph(side, body, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: body capture");
+    const SelectWindow win = {k, n_sink, n_local};
+    cudaError_t le = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, side);
+    if (le == cudaSuccess)
+        le = launch_vote(p, kv->seq_offsets_dev, reuse, votes, w, side, &win);
+    if (le == cudaSuccess)
+        le = launch_select(p, kv->seq_offsets_dev, votes, k, n_sink, n_local, reuse, ids, count, w, side, true);
+    cudaGraph_t captured = nullptr;
+    e = cudaStreamEndCapture(side, &captured);
+    if (le != cudaSuccess)
+        return cuda_fail(le, "ts_decode_step: conditional body launch");
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: body capture end");
+    e = cudaStreamUpdateCaptureDependencies(st, &cond_node, 1, cudaStreamSetCaptureDependencies);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: capture dependencies");
+    e = launch_attn(p, kv, q, ids, count, out, w, st);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_decode_step: sparse attention launch");
+}
+
 ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32_t *reuse, double *cos_out,
                            int32_t first_step, double threshold, int32_t k, int32_t n_sink, int32_t n_local,
                            float *votes, int32_t *ids, int32_t *count, float *out, void *ws, size_t ws_bytes,
@@ -552,7 +716,18 @@ ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *w = static_cast<uint8_t *>(ws);
-    cudaError_t e = launch_selcache(q, q_prev, reuse, cos_out, first_step != 0, p.B, p.Hq * p.D, threshold, st);
+    // captured into a graph with the selection cache able to reuse: scoring
+    // and selection go into a conditional node the cosine kernel can switch off
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamGetCaptureInfo(st, &cap, nullptr, &graph, nullptr, nullptr);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ts_decode_step: capture query");
+    const bool can_reuse = first_step == 0 && threshold <= 1.0 + 1e-6;
+    if (cap == cudaStreamCaptureStatusActive && can_reuse && p.n_total > 0 && reuse_skip_enabled())
+        return decode_step_graph(p, kmap, kv, q, q_prev, reuse, cos_out, threshold, k, n_sink, n_local, votes, ids,
+                                 count, out, w, st, graph);
+    e = launch_selcache(q, q_prev, reuse, cos_out, first_step != 0, p.B, p.Hq * p.D, threshold, st);
     if (e != cudaSuccess)
         return cuda_fail(e, "ts_decode_step: selection cache launch");
     if (p.n_total > 0) {

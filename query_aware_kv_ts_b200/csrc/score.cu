@@ -46,13 +46,13 @@
 //  * score_merge (one warp per sequence and head) folds the partials of the
 //    CTAs that cover the sequence (j0..j1; every CTA with chunks for one
 //    sequence) into L[b, h]: fp32 terms exp(m - M) <= 1 summed in float64.
+#include "score_common.cuh"
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
 namespace ts {
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxPrefetchTiles = 6;
 constexpr int kProducerWarp = kScoreEpiWarps;       // 8
 constexpr int kMmaWarp = kScoreEpiWarps + 1;        // 9
@@ -89,16 +89,6 @@ struct __align__(16) ScoreShared {
     int32_t pf_start[32];     // all-active chunk table of the prefetch hints (B <= 32)
     int64_t pf_off[32];       // and the sequence offsets it was built from
 };
-
-__device__ __forceinline__ void online_push(float &m, float &z, float x)
-{
-    if (x > m) {
-        z = z * exp2f((m - x) * kLog2e) + 1.0f;
-        m = x;
-    } else {
-        z += exp2f((x - m) * kLog2e);
-    }
-}
 
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int32_t x, int32_t y, int32_t z)
 {
@@ -138,15 +128,6 @@ __device__ __forceinline__ void build_chunk_table(ScoreShared &sh, const int32_t
             sh.chunk_start[0] = 0;
     }
     __syncthreads();
-}
-
-// floor(j * total / grid) for j <= grid <= 256 and total < 2^31: a double
-// quotient is exact enough (a non-integer quotient is at least 1/grid away
-// from an integer, far above the rounding error) and much cheaper than a
-// 64-bit integer division.
-__device__ __forceinline__ int32_t chunk_split(uint32_t j, int32_t total, uint32_t grid)
-{
-    return (int32_t)floor((double)j * (double)total / (double)grid);
 }
 
 // B <= 32: lane b < B computes c0 = first chunk of sequence b and c1 = one past
@@ -213,18 +194,6 @@ __device__ __forceinline__ void stage_queries(uint8_t *qs, const __nv_bfloat16 *
             }
         }
     }
-}
-
-// Order-preserving map of a float to a signed integer (and back), for the
-// integer warp max reduction.
-__device__ __forceinline__ int32_t float_order_key(float x)
-{
-    const int32_t b = __float_as_int(x);
-    return b >= 0 ? b : (b ^ 0x7fffffff);
-}
-__device__ __forceinline__ float float_from_order_key(int32_t k)
-{
-    return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff));
 }
 
 // End of a (CTA, sequence) segment in the epilogue: reduce each head's

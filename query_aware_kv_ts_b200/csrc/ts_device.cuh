@@ -21,6 +21,8 @@ enum : uint32_t {
     kSiteAttnGather = 3,      // attention waiting for its gathered K/V rows
     kSiteScoreAcc = 4,        // score epilogue waiting for a TMEM accumulator
     kSiteScoreMma = 5,        // score MMA issuer waiting for a stage, a free accumulator or its own MMAs
+    kSiteFusedGrid = 6,       // fused scoring waiting for every CTA to finish a pass
+    kSiteFusedCta = 7,        // fused scoring: a warp waiting for the other vote workers of its CTA
     kSiteSelftest = 99,
 };
 
@@ -257,6 +259,9 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor cores).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// The same for global memory: generic-proxy writes this thread has observed
+// become visible to its later bulk asynchronous copies.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // Programmatic dependent launch: every kernel of the library first does the
 // set-up that reads nothing another kernel writes, then waits for the kernel
@@ -273,9 +278,14 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src)
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Named barrier over a subset of the block's warps.
+// Named barrier over a subset of the block's warps (whole warps call it).
+// bar.sync counts a warp as arrived when any of its threads executes it, so
+// the warp is reconverged first: lanes left behind in a divergent branch
+// (one lane polling a flag, say) would otherwise arrive a second time later
+// and release a later phase of the barrier early.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads)
 {
+    __syncwarp();
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 

@@ -18,6 +18,7 @@ constexpr int kScoreThreads = (kScoreEpiWarps + 2) * 32;   // + TMA producer war
 constexpr int kScoreMaxStages = 12;
 constexpr int kScoreAccBufs = 4;                // TMEM accumulators in flight
 constexpr size_t kScoreDynSmemBudget = 212 * 1024;   // + the kernel's ~13 KB of static shared memory
+constexpr size_t kFusedDynSmemBudget = 224 * 1024;   // + the fused kernel's ~2 KB of static shared memory
 constexpr int kVoteThreads = 256;
 constexpr int kSelectThreads = 256;
 constexpr int kSelectTokensPerCta = 2048;     // candidates per selection range
@@ -25,6 +26,8 @@ constexpr int kMaxSelectRanges = 2048;        // ranges per sequence: n <= 4M ca
 constexpr int kAttnThreads = 256;
 constexpr int kAttnRows = 64;         // selected rows per attention CTA (one split)
 constexpr int kMaxCapacity = 16384;   // k + sink + local
+constexpr int kFusedRows = 128;       // K rows per stage of the fused scoring kernel (HS heads x T tokens)
+constexpr size_t kFusedPassLogitsBytes = size_t(32) << 20;   // logits one fused-scoring pass may keep in L2
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -62,6 +65,38 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Cooperative launch (every CTA of the grid resident at once, as a kernel
+// with grid-wide barriers needs), with programmatic stream serialization
+// unless TS_NO_PDL=1.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Control-block words (the first 256 bytes of every workspace, zeroed by
+// ts_workspace_init): [0] status, [1] site; [8, 9] the reuse-skip counters of
+// the cosine kernel; [16, 16 + passes) the fused scoring kernel's per-pass
+// arrival counters, [24] its finished-CTA count.
+constexpr int kCtrlFusedBarrier = 16;
+
 // Everything derived from the cache shape that the kernels and the workspace
 // layout need.  Built identically by every entry point.
 struct Plan {
@@ -77,6 +112,14 @@ struct Plan {
     int score_grid;          // <= 256
     int score_partials_per_slot;   // R: epilogue warps of pass A that see one kv head
     int64_t ld_logits;       // logits row stride: n_total rounded up to 4
+    // fused scoring (HS kv heads of T = 128 / HS tokens per stage)
+    int fused_hs;            // kv heads per pass (4, 2 or 1; divides h_kv)
+    int fused_t;             // tokens per chunk
+    int fused_gp;            // staged query rows per kv head (4, 8 or 16)
+    int fused_n;             // MMA N: max(16, HS * GP)
+    int64_t fused_chunks;    // sum_b ceil(n_b / T)
+    int fused_grid;          // min(SMs, fused_chunks)
+    int64_t fused_ld;        // its logits row stride: fused_chunks * T
     // selection
     int sel_ranges;          // ranges of kSelectTokensPerCta candidates per sequence (grid x)
     // attention
@@ -84,7 +127,7 @@ struct Plan {
     int attn_splits;
     // workspace layout (byte offsets)
     size_t off_ctrl, off_chunk_table, off_L, off_partials, off_logits, off_sel_hist, off_sel_cand,
-        off_sel_inb1, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_attn_part,
+        off_sel_inb1, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_vacc, off_attn_part,
         total_bytes;
 };
 
@@ -105,8 +148,18 @@ void *current_context();
 cudaError_t ensure_dyn_smem(const void *kernel, int bytes);
 
 // Launchers (return cudaGetLastError() of the launch).
+// In a graph replay the cosine kernel can switch off the conditional node
+// that holds the scoring and selection kernels: the last of its blocks sets
+// the node's condition to 0 when every sequence reuses its selection.
+// counters: two words of the workspace control block (zero between steps).
+constexpr int kCtrlSkipCounters = 8;   // control-block words 8, 9
+struct SelcacheSkip {
+    cudaGraphConditionalHandle handle;
+    uint32_t *counters;
+    int enabled;
+};
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step,
-                            int B, int len, double theta, cudaStream_t st);
+                            int B, int len, double theta, cudaStream_t st, const SelcacheSkip *skip = nullptr);
 
 // seq_off_host: the host copy of the offsets (prefetch hints before the
 // dependency wait; the device copy decides the work).
@@ -121,6 +174,13 @@ struct SelectWindow {
 
 cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
                         cudaStream_t st, const SelectWindow *hist_window = nullptr);
+
+// Logits, normalisers and votes in one cooperative kernel, one kv-head group
+// at a time (kmap_head: boxes of {64 channels, 128 tokens, 1 head}); with a
+// window it also builds the selection's level-1 histogram.
+cudaError_t launch_score_fused(const Plan &p, const CUtensorMap &kmap_head, const void *q, const int64_t *seq_off,
+                               const int64_t *seq_off_host, const int32_t *reuse, float *votes, uint8_t *ws,
+                               cudaStream_t st, const SelectWindow *hist_window = nullptr);
 
 // hist_ready: the level-1 histogram was already built by the vote pass.
 cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *votes, int k, int n_sink,

@@ -4,16 +4,10 @@
 // reading the logits written by pass A (L2-resident for moderate n) and the
 // float64 log-normalisers L.
 //
-// Precision: s - L is formed exactly as t + d (two-sum of s and the float
-// high part of L, minus L's low part).  The base-2 exponent u = (t + d) log2(e)
-// is carried as an unevaluated pair too: u_hi = fl(t * log2e_hi) and
-//   u_lo = fma(t, log2e_hi, -u_hi) + t * log2e_lo + d * log2e_hi
-// (the product error recovered with one fma, as in Dekker's exact product,
-// with log2(e) split Cody-Waite style into a float head and tail), so that
-// exp(s - L) = 2^u_hi * (1 + u_lo ln 2) up to second order in |u_lo| < 2^-17.
-// The only rounding left is the hardware 2^x (a few 1e-8 relative) and the
-// sum over heads.  A plain fp32 s - L would lose up to half an ulp of |s - L|
-// (~1e-6 relative for |s - L| ~ 20), the width of the selection band.
+// Precision: each term is exp_exact_arg (score_common.cuh): s - L formed
+// exactly, the base-2 exponent carried as a head/tail pair, so the only
+// rounding left is the hardware 2^x (a few 1e-8 relative) and the sum over
+// heads.
 //
 // Work split: grid (groups / threads, B).  Long sequences: a thread takes 4
 // consecutive tokens aligned to 4 in the logits rows (row stride padded to 4),
@@ -28,6 +22,7 @@
 // selection's level-1 histogram of its candidates' votes (top 12 bits of the
 // fp32 pattern, the bins the selection starts from): a shared-memory
 // histogram per block, merged into the sequence's global one with atomics.
+#include "score_common.cuh"
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -48,21 +43,6 @@ struct VoteArgs {
 
 constexpr int kMaxHeadsVote = 256;
 constexpr int kHeadBatch = 8;
-constexpr float kLog2eHi = 1.44269502162933349609375f;   // float nearest log2(e)
-constexpr float kLog2eLo = 1.925963033500011e-08f;       // log2(e) - kLog2eHi
-constexpr float kLn2 = 0.693147180559945309f;
-
-__device__ __forceinline__ float exp_exact_arg(float s, float Lhi, float Llo)
-{
-    const float t = s - Lhi;                       // two-sum: t + e == s - Lhi
-    const float bp = t - s;
-    const float e = (s - (t - bp)) + (-Lhi - bp);
-    const float d = e - Llo;                       // s - L == t + d
-    const float u = t * kLog2eHi;
-    const float u_lo = fmaf(t, kLog2eHi, -u) + fmaf(t, kLog2eLo, d * kLog2eHi);
-    const float p = exp2f(u);
-    return fmaf(p, u_lo * kLn2, p);
-}
 
 // Blackwell's packed fp32 instructions: two lanes per instruction, each lane
 // rounded exactly as the scalar IEEE operation.  The low half is the first

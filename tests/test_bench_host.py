@@ -116,20 +116,23 @@ def test_measured_peak_record():
 
 
 def test_traffic_record_follows_the_kernel_source(tmp_path):
-    src = os.path.join(bench.ROOT, "query_aware_kv_ts_b200", "csrc", "score.cu")
-    with open(os.path.join(bench.ROOT, "profiles", "score_pass_a_traffic.json")) as f:
-        rec = json.load(f)
-    with open(src, "rb") as f:
-        current = hashlib.sha256(f.read()).hexdigest() == rec["source_sha256"]
+    src = tmp_path / "kernel.cu"
+    src.write_text("// a kernel\n")
+    rec = {"source_sha256": hashlib.sha256(src.read_bytes()).hexdigest(),
+           "per_launch_bytes": {"qwen7b_1m": 1234}}
+    path = tmp_path / "record.json"
+    path.write_text(json.dumps(rec))
     # the record counts only while the kernel source is the one it was taken on
-    want = rec["per_launch_bytes"]["qwen7b_32k"] if current else None
-    assert bench.profile_traffic(src, "qwen7b_32k") == want
-    assert bench.profile_traffic(src, "no_such_workload") is None
-    changed = tmp_path / "score.cu"
-    shutil.copy(src, changed)
-    with open(changed, "a") as f:
-        f.write("\n// changed\n")
-    assert bench.profile_traffic(str(changed), "qwen7b_32k") is None
+    assert bench.profile_traffic(str(src), "qwen7b_1m", str(path)) == 1234
+    assert bench.profile_traffic(str(src), "no_such_workload", str(path)) is None
+    assert bench.profile_traffic(str(src), "qwen7b_1m", str(tmp_path / "missing.json")) is None
+    with open(src, "a") as f:
+        f.write("// changed\n")
+    assert bench.profile_traffic(str(src), "qwen7b_1m", str(path)) is None
+    # the committed record, where there is one, names the dominant kernel's source
+    if os.path.exists(bench.TRAFFIC_RECORD):
+        with open(bench.TRAFFIC_RECORD) as f:
+            assert json.load(f)["source"].endswith("score.cu")
 
 
 def test_all_core_oracle_baseline_runs_threads_in_parallel():

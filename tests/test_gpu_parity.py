@@ -101,3 +101,52 @@ def test_planted_keys_selected():
     votes = buf.votes.cpu().numpy()
     top = np.argsort(-votes)[:40]
     assert set(top.tolist()) <= ids
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fused_score_matches_oracle_and_two_phase(name):
+    """ts_score_fused (logits, normalisers and votes in one kernel, a few kv
+    heads per pass) against the oracle's votes, and against ts_score (the
+    two-phase scoring) to within their two roundings; a second call on the
+    same workspace gives the same votes (the kernel's grid-barrier counters
+    return to zero)."""
+    lengths, h_q, h_kv, d, k, s, l, extra = CASES[name]
+    case = _case(lengths, h_q, h_kv, d, seed=zlib.crc32(name.encode()) % 10000, **extra)
+    m = H.ts()
+    buf = m.StepBuffers(case.kv, k, s, l)
+    m.ts_score(case.kv, case.q, None, buf.votes, buf.ws)
+    two = buf.votes.cpu().numpy().copy()
+    m.ts_score_fused(case.kv, case.q, None, buf.votes, buf.ws)
+    fused = buf.votes.cpu().numpy().copy()
+    m.ts_score_fused(case.kv, case.q, None, buf.votes, buf.ws)
+    assert np.array_equal(buf.votes.cpu().numpy().view(np.uint32), fused.view(np.uint32))
+    status, site = m.ts_get_device_status(buf.ws)
+    assert status == m.TS_OK, (status, site)
+    qb = W.bf16_bits(case.q)
+    for b in range(case.B):
+        lo, hi = case.seq(b)
+        if hi == lo:
+            continue
+        v_ref, _ = H.oracle.votes(case.kb[lo:hi], qb[b], case.oracle_scale())
+        H.check_votes(two[lo:hi], v_ref, h_q)
+        H.check_votes(fused[lo:hi], v_ref, h_q)
+        rel = np.abs(two[lo:hi].astype(np.float64) - fused[lo:hi]) / np.maximum(v_ref, 1e-30)
+        assert rel.max() < 1e-5, rel.max()
+
+
+@pytest.mark.parametrize("cfg_name", ["qwen7b_32k", "llama8b_b4", "ragged_b32", "qwen7b_1m"])
+def test_fused_score_full_size(cfg_name):
+    """ts_score_fused at the workloads' full sizes (one pass at 32K; two at
+    4 x 131072; one kv head per pass at 32 ragged sequences and at 1M tokens)
+    against the oracle's votes, sequence by sequence."""
+    cfg = W.CONFIGS[cfg_name]
+    case, _ = H.config_case(cfg)
+    m = H.ts()
+    buf = m.StepBuffers(case.kv, cfg.k, cfg.n_sink, cfg.n_local)
+    m.ts_score_fused(case.kv, case.q, None, buf.votes, buf.ws)
+    votes = buf.votes.cpu().numpy()
+    qb = W.bf16_bits(case.q)
+    for b in range(case.B):
+        lo, hi = case.seq(b)
+        v_ref, _ = H.oracle.votes(case.kb[lo:hi], qb[b], case.oracle_scale())
+        H.check_votes(votes[lo:hi], v_ref, cfg.h_q)
