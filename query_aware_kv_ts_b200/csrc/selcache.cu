@@ -6,6 +6,10 @@
 // cos >= threshold, then the current query replaces the previous one.  Each
 // thread overwrites exactly the q_prev elements it read, so no barrier is
 // needed between read and write.
+// Replayed from a CUDA graph, the kernel can also switch off the graph's
+// scoring and selection (a conditional node) for a step in which every
+// sequence reuses its selection: those kernels would only read the flags and
+// return.
 #include "ts_device.cuh"
 #include "ts_internal.h"
 
@@ -16,7 +20,7 @@ constexpr int kSelcacheThreads = 256;
 
 __global__ void __launch_bounds__(kSelcacheThreads)
 selcache_kernel(const uint32_t *__restrict__ q, uint32_t *__restrict__ q_prev, int32_t *reuse, double *cos_out, int first_step,
-                int len_pairs, double theta)
+                int len_pairs, double theta, const SelcacheSkip skip)
 {
     pdl_wait();
     pdl_launch_dependents();
@@ -86,17 +90,34 @@ selcache_kernel(const uint32_t *__restrict__ q, uint32_t *__restrict__ q_prev, i
         reuse[b] = r;
         if (cos_out)
             cos_out[b] = c;
+        if (skip.enabled) {
+            // the last block to finish has seen every sequence's decision:
+            // when all of them reuse, the graph's scoring and selection are
+            // switched off for this replay
+            atomicAdd(&skip.counters[0], (uint32_t)r);
+            __threadfence();
+            if (atomicAdd(&skip.counters[1], 1u) == gridDim.x - 1) {
+                __threadfence();
+                if (atomicAdd(&skip.counters[0], 0u) == gridDim.x)
+                    cudaGraphSetConditional(skip.handle, 0u);
+                atomicExch(&skip.counters[0], 0u);   // zero again for the next replay
+                atomicExch(&skip.counters[1], 0u);
+            }
+        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step, int B,
-                            int len, double theta, cudaStream_t st)
+                            int len, double theta, cudaStream_t st, const SelcacheSkip *skip)
 {
+    SelcacheSkip sk = {};
+    if (skip != nullptr)
+        sk = *skip;
     return launch_ex(selcache_kernel, dim3((unsigned)B), dim3(kSelcacheThreads), 0, st, 1,
                      static_cast<const uint32_t *>(q), static_cast<uint32_t *>(q_prev), reuse, cos_out, first_step,
-                     len / 2, theta);
+                     len / 2, theta, sk);
 }
 
 }  // namespace ts
