@@ -67,6 +67,10 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="run only the first N layers of the workload (a smaller case of the same kernels, "
                          "for profiler captures); the JSON line's config records it")
+    ap.add_argument("--eager-steps", type=int, default=None,
+                    help="profiler capture mode: after set-up, run this many decode steps of the workload as "
+                         "plain (not graph-replayed) C-ABI calls, along the workload's query sequence, and exit "
+                         "without timing or printing a result")
     a = ap.parse_args(argv)
     big = a.workload in ("llama8b_b4", "ragged_b32", "qwen7b_1m")
     if a.steps is None:
@@ -417,6 +421,12 @@ def run_ours(a, d: Dist):
     wl = Workload(a.workload, dev, a.layers)
     cfg = wl.cfg
     ts = wl.ts
+    if a.eager_steps is not None:
+        for i in range(a.eager_steps):
+            wl.step(i)
+        torch.cuda.synchronize()
+        d.close()
+        return
 
     # eager warm-up (also configures kernel attributes before capture)
     for i in range(2):
@@ -532,11 +542,11 @@ def run_ours(a, d: Dist):
     step_hbm_gbs = step_alg_bytes / el_max / 1e9
 
     # every layer-step is one ts_decode_step call (the same shapes in every
-    # layer); replayed from a graph, a layer-step in which every sequence
-    # reuses its selection skips the scoring and selection kernels (the cosine
-    # test and the two attention kernels run)
+    # layer); with TS_REUSE_SKIP=1 a graph-replayed layer-step in which every
+    # sequence reuses its selection skips the scoring and selection kernels
+    # (the cosine test and the two attention kernels run)
     kernels_per_layer_step = ts.ts_decode_step_kernels(wl.kvs[0][0], cfg.k, cfg.n_sink, cfg.n_local)
-    skip_on = cfg.theta is not None and os.environ.get("TS_NO_REUSE_SKIP") != "1"
+    skip_on = cfg.theta is not None and os.environ.get("TS_REUSE_SKIP") == "1"
     all_reused = flags_np.all(axis=2) if skip_on else np.zeros(flags_np.shape[:2], bool)
     gpu_launches = int(np.where(all_reused, 3, kernels_per_layer_step).sum())
     alg_bytes = wl.k_rows_bytes() * cfg.layers

@@ -238,13 +238,15 @@ TS_API ts_status_t ts_sparse_attn_noalloc(const ts_kv_t *kv, const void *q, cons
  * the selection's first-level vote histogram, which ts_select otherwise builds
  * in a kernel of its own (ts_decode_step_kernels gives the count).  Every
  * argument is checked before the first launch.
- *   Under stream capture with the selection cache able to reuse (first_step
- *   0, threshold <= 1), the scoring and selection kernels are captured into
- *   the body of a conditional graph node that the cosine kernel switches
- *   off when every sequence reuses: such a replayed step runs 3 kernels (the
- *   cosine test and the two attention kernels).  The results are the same
+ *   With TS_REUSE_SKIP=1 in the environment, a call under stream capture
+ *   with the selection cache able to reuse (first_step 0, threshold <= 1)
+ *   captures the scoring and selection kernels into the body of a
+ *   conditional graph node that the cosine kernel switches off when every
+ *   sequence reuses: such a replayed step runs 3 kernels (the cosine test
+ *   and the two attention kernels) instead of 9.  The results are the same
  *   either way.  The body is captured on a stream the library creates once
- *   per context; TS_NO_REUSE_SKIP=1 in the environment turns this off.
+ *   per context.  Off by default: the node's edges cannot use programmatic
+ *   launch, which on B200 costs more than the skipped kernels save.
  *   reuse      device int32 [batch], required: written by the selection cache
  *              and read by every later phase (sequences that reuse keep their
  *              previous ids and count; their votes are left as they were)

@@ -105,16 +105,16 @@ cudaError_t ensure_dyn_smem(const void *kernel, int bytes)
     return cudaSuccess;
 }
 
-// Graph replays of ts_decode_step skip the scoring and selection kernels of
-// a step in which every sequence reuses its selection, unless the
-// environment sets TS_NO_REUSE_SKIP=1.
+// Captured into a graph, ts_decode_step can put its scoring and selection
+// kernels in a conditional node that the cosine kernel switches off when
+// every sequence reuses its selection.  Off unless the environment sets
+// TS_REUSE_SKIP=1 (read at every call): measured on B200, the two edges a
+// conditional node forces to full serialisation (no programmatic launch
+// into or out of it) cost more than the early-exiting kernels it skips.
 static bool reuse_skip_enabled()
 {
-    static const bool on = [] {
-        const char *e = getenv("TS_NO_REUSE_SKIP");
-        return !(e != nullptr && e[0] == '1');
-    }();
-    return on;
+    const char *e = getenv("TS_REUSE_SKIP");
+    return e != nullptr && e[0] == '1';
 }
 
 // A non-blocking stream of the current context on which the body of a

@@ -1,6 +1,7 @@
-"""ts_decode_step captured into CUDA graphs with the selection cache on: the
-scoring and selection kernels sit in a conditional node that the cosine
-kernel switches off when every sequence of the step reuses its selection.
+"""ts_decode_step captured into CUDA graphs with the selection cache on and
+TS_REUSE_SKIP=1: the scoring and selection kernels sit in a conditional node
+that the cosine kernel switches off when every sequence of the step reuses
+its selection.
 Replaying the captured steps must give, at every step of an AR(1) query
 trajectory, exactly (bit for bit) what the eager one-call step gives, and the
 graph-replayed trajectory must follow the oracle."""
@@ -21,7 +22,8 @@ def _step(m, case, buf, cfg, t, stream=None):
 
 
 @pytest.mark.parametrize("cfg_name,n", [("llama8b_b4", 4096), ("qwen7b_1m", 16384), ("qwen7b_32k_theta", 32768)])
-def test_graph_replay_equals_eager_trajectory(cfg_name, n):
+def test_graph_replay_equals_eager_trajectory(cfg_name, n, monkeypatch):
+    monkeypatch.setenv("TS_REUSE_SKIP", "1")
     if cfg_name == "qwen7b_32k_theta":
         # the Qwen2-7B layer with the selection cache on and AR(1) queries
         import dataclasses
