@@ -74,6 +74,13 @@ typedef enum {
  *   stride_tok,        in elements; multiples of 8; stride_head >= head_dim,
  *   stride_head        stride_tok >= (h_kv-1)*stride_head + head_dim
  *   scale              softmax scale; 0 selects 1/sqrt(head_dim)
+ *   capacity           0, or (batch 1 only) the number of tokens the K and V
+ *                      buffers hold, >= the current length: the cache can
+ *                      then grow on the device (ts_append_kv).  Workspace
+ *                      sizes, launch shapes and the tensor map follow the
+ *                      capacity and every kernel takes the current length
+ *                      from seq_offsets_dev, so one workspace and one
+ *                      captured graph serve every length up to it.
  */
 typedef struct ts_kv {
     int32_t batch, h_q, h_kv, head_dim;
@@ -83,6 +90,7 @@ typedef struct ts_kv {
     const void *v;
     int64_t stride_tok, stride_head;
     float scale;
+    int64_t capacity;
 } ts_kv_t;
 
 /*
@@ -131,7 +139,8 @@ TS_API ts_status_t ts_selcache(const void *q, void *q_prev, int32_t *reuse, doub
  * skipped (their votes are left as they were).
  *   q          device bf16 [batch, h_q, head_dim] contiguous, 16-byte aligned
  *   reuse      device int32 [batch] or NULL (NULL: score every sequence)
- *   votes      device float32 [seq_offsets[batch]], written
+ *   votes      device float32 [seq_offsets[batch]] (a cache with a capacity:
+ *              [capacity]), written
  * The float32 votes carry a relative error of a few 1e-7.
  */
 TS_API ts_status_t ts_score(const ts_kv_t *kv, const void *q, const int32_t *reuse, float *votes,
@@ -258,6 +267,26 @@ TS_API ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev
                                   int32_t *count, float *out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Append one token to a growing cache (capacity mode, batch 1), entirely on
+ * the device: the token's K and V rows go to position n = seq_offsets_dev[1]
+ * and seq_offsets_dev[1] becomes n + 1, so a captured graph can append step
+ * after step.  With the selection cache on, a later step that reuses its
+ * selection keeps the previous top-k part and takes the sink and local
+ * windows of the new length (TokenSelect README, "Key Takeaways", Selection
+ * Cache).
+ *   kv            the cache, capacity > 0
+ *   seq_offsets   kv->seq_offsets_dev, writable
+ *   k_cache, v_cache   kv->k and kv->v, writable
+ *   k_new, v_new  device bf16 [h_kv][head_dim] each, contiguous, 16-byte aligned
+ *   ws            a workspace of this cache: appending to a full cache
+ *                 writes nothing and records the error in its status word
+ *                 (ts_get_device_status then returns TS_ERR_INVALID_ARG)
+ * The host copy kv->seq_offsets_host is not read here and not updated.
+ */
+TS_API ts_status_t ts_append_kv(const ts_kv_t *kv, int64_t *seq_offsets, void *k_cache, void *v_cache,
+                                const void *k_new, const void *v_new, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Number of kernels one ts_decode_step call on this cache launches (for
  * launch accounting and profiling), or -1 with ts_last_error set when the
  * cache description or the selection sizes are invalid.  Host only; touches
@@ -268,10 +297,11 @@ TS_API int32_t ts_decode_step_kernels(const ts_kv_t *kv, int32_t k, int32_t n_si
 /*
  * Read and clear the device status word of a workspace (synchronises the
  * stream).  Returns TS_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave
- * up since the last read, TS_OK otherwise.  *site_out (may be NULL) receives
- * a code naming the wait that gave up.  After TS_ERR_DEVICE_TIMEOUT the
- * results of every call since the last TS_OK read are void, and so are the
- * workspace's contents: re-initialise it (ts_workspace_init) before reuse.
+ * up since the last read, TS_ERR_INVALID_ARG when ts_append_kv found the
+ * cache full, TS_OK otherwise.  *site_out (may be NULL) receives a code
+ * naming the wait or the call.  After TS_ERR_DEVICE_TIMEOUT the results of
+ * every call since the last TS_OK read are void, and so are the workspace's
+ * contents: re-initialise it (ts_workspace_init) before reuse.
  */
 TS_API ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, void *stream);
 

@@ -46,6 +46,7 @@ class ts_kv_t(ctypes.Structure):
         ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64),
         ("scale", ctypes.c_float),
+        ("capacity", ctypes.c_int64),
     ]
 
 
@@ -69,6 +70,7 @@ _SIGS = {
     "ts_decode_step": (ctypes.c_int, [_KV, _P, _P, _P, _P, _I32, _F64, _I32, _I32, _I32, _P, _P, _P, _P, _P,
                                       _SZ, _P]),
     "ts_decode_step_kernels": (_I32, [_KV, _I32, _I32, _I32]),
+    "ts_append_kv": (ctypes.c_int, [_KV, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -113,7 +115,8 @@ class KVCache:
     tensor; a device copy is made once).  Keeps the ts_kv_t and the tensors it
     points at alive together."""
 
-    def __init__(self, k: torch.Tensor, v: torch.Tensor, seq_offsets, h_q: int, scale: float = 0.0):
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, seq_offsets, h_q: int, scale: float = 0.0,
+                 capacity: int = 0):
         if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
             raise TypeError("K and V must be bf16")
         if k.dim() != 3 or k.shape != v.shape or k.stride() != v.stride() or k.stride(2) != 1:
@@ -128,7 +131,9 @@ class KVCache:
         self.struct = ts_kv_t(self.batch, self.h_q, self.h_kv, self.head_dim,
                               self.seq_offsets_dev.data_ptr(),
                               off.ctypes.data_as(ctypes.c_void_p).value,
-                              k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), float(scale))
+                              k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), float(scale),
+                              int(capacity))
+        self.capacity = int(capacity)
 
     @property
     def n_total(self) -> int:
@@ -208,6 +213,15 @@ def ts_decode_step(kv: KVCache, q, q_prev, reuse, first_step: bool, threshold: f
                                _stream(stream)))
 
 
+def ts_append_kv(kv: KVCache, k_new, v_new, ws, stream=None):
+    """Append one token ([h_kv, d] K and V rows, bf16, on the device) to a
+    growing cache (KVCache(..., capacity=C), batch 1) on the device: rows at
+    position n = seq_offsets[1], then seq_offsets[1] = n + 1 (device copy
+    only; kv.seq_offsets_host is left as it was)."""
+    _check(_lib.ts_append_kv(kv.ref(), kv.seq_offsets_dev.data_ptr(), _ptr(kv.k), _ptr(kv.v), _ptr(k_new),
+                             _ptr(v_new), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def ts_decode_step_kernels(kv: KVCache, k: int, n_sink: int, n_local: int) -> int:
     """Kernels one ts_decode_step call on this cache launches."""
     n = _lib.ts_decode_step_kernels(kv.ref(), k, n_sink, n_local)
@@ -254,7 +268,7 @@ class StepBuffers:
         nbytes = ts_workspace_bytes(kv, k, n_sink, n_local)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         ts_workspace_init(self.ws)
-        self.votes = torch.zeros(max(kv.n_total, 1), dtype=torch.float32, device=dev)
+        self.votes = torch.zeros(max(kv.n_total, kv.capacity, 1), dtype=torch.float32, device=dev)
         self.ids = torch.full((kv.batch, self.capacity), -1, dtype=torch.int32, device=dev)
         self.count = torch.zeros(kv.batch, dtype=torch.int32, device=dev)
         self.out = torch.zeros((kv.batch, kv.h_q, kv.head_dim), dtype=torch.float32, device=dev)

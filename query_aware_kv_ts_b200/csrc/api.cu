@@ -225,7 +225,24 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
         }
         n_max = n > n_max ? n : n_max;
     }
-    const int64_t n_total = off[kv->batch];
+    int64_t n_total = off[kv->batch];
+    if (kv->capacity < 0) {
+        set_error("capacity must be >= 0");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (kv->capacity > 0) {
+        // a growing cache: sizes for its largest length, work from the device offsets
+        if (kv->batch != 1) {
+            set_error("a cache with a capacity must hold one sequence (batch %d)", kv->batch);
+            return TS_ERR_UNSUPPORTED;
+        }
+        if (kv->capacity < n_total) {
+            set_error("capacity %lld is below the current length %lld", (long long)kv->capacity,
+                      (long long)n_total);
+            return TS_ERR_INVALID_ARG;
+        }
+        n_total = n_max = kv->capacity;
+    }
     if (n_total >= (int64_t(1) << 31)) {
         set_error("total tokens %lld must be below 2^31", (long long)n_total);
         return TS_ERR_UNSUPPORTED;
@@ -254,7 +271,7 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->stage_bytes = kScoreRows * D * 2;
     int64_t chunks = 0;
     for (int b = 0; b < kv->batch; ++b) {
-        const int64_t n = off[b + 1] - off[b];
+        const int64_t n = kv->capacity > 0 ? n_total : off[b + 1] - off[b];
         chunks += (n + p->tile_tokens - 1) / p->tile_tokens;
     }
     p->max_chunks = chunks;
@@ -283,8 +300,10 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
         p->fused_t = kFusedRows / hs;
         p->fused_n = hs * gp < 16 ? 16 : hs * gp;
         int64_t fc = 0;
-        for (int b = 0; b < kv->batch; ++b)
-            fc += (off[b + 1] - off[b] + p->fused_t - 1) / p->fused_t;
+        for (int b = 0; b < kv->batch; ++b) {
+            const int64_t n = kv->capacity > 0 ? n_total : off[b + 1] - off[b];   // a growing cache: its capacity
+            fc += (n + p->fused_t - 1) / p->fused_t;
+        }
         p->fused_chunks = fc;
         p->fused_grid = (int)(fc < grid_cap ? fc : grid_cap);
         p->fused_ld = fc * p->fused_t;
@@ -329,6 +348,8 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     o = align_up(o + sizeof(uint64_t) * (size_t)p->B, 256);
     p->off_sel_mode = o;
     o = align_up(o + sizeof(int32_t) * (size_t)p->B, 256);
+    p->off_sel_prev_n = o;   // length + 1 at the previous selection (0: none yet)
+    o = align_up(o + sizeof(int64_t) * (size_t)p->B, 256);
     p->off_sel_hist = o;
     o = align_up(o + sizeof(uint32_t) * 4096 * (size_t)p->B, 256);
     p->off_logits = o;
@@ -780,11 +801,45 @@ ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *site_out, 
         return cuda_fail(e, "ts_get_device_status");
     if (site_out)
         *site_out = h[1];
+    if (h[0] == 2u) {
+        set_error("ts_append_kv found the cache full");
+        return TS_ERR_INVALID_ARG;
+    }
     if (h[0] != 0u) {
         set_error("a device-side wait gave up (site %u)", h[1]);
         return TS_ERR_DEVICE_TIMEOUT;
     }
     return TS_OK;
+}
+
+ts_status_t ts_append_kv(const ts_kv_t *kv, int64_t *seq_offsets, void *k_cache, void *v_cache, const void *k_new,
+                         const void *v_new, void *ws, size_t ws_bytes, void *stream)
+{
+    if (kv == nullptr || kv->capacity <= 0) {
+        set_error("ts_append_kv needs a cache with a capacity");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (seq_offsets != kv->seq_offsets_dev || k_cache != kv->k || v_cache != kv->v) {
+        set_error("seq_offsets, k_cache and v_cache must be the cache's own device arrays");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (k_new == nullptr || v_new == nullptr ||
+        ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)) {
+        set_error("k_new and v_new must be 16-byte aligned device rows");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (ws == nullptr || ws_bytes < 256) {
+        set_error("workspace is NULL or smaller than its control block");
+        return TS_ERR_WORKSPACE;
+    }
+    Plan p;
+    const ts_status_t s = make_plan(kv, -1, &p);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_append(seq_offsets, k_cache, v_cache, k_new, v_new, kv->stride_tok, kv->stride_head,
+                                  p.Hkv, p.D, kv->capacity, reinterpret_cast<uint32_t *>(ws),
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "ts_append_kv");
 }
 
 ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_limit, void *stream)

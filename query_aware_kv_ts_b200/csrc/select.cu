@@ -56,6 +56,7 @@ struct SelArgs {
     uint32_t *range_off;       // [B][rps] output offset of each range within the top-k part
     unsigned long long *thr;   // [B] threshold key T
     int32_t *mode;             // [B] 0: none, 1: keys >= T, 2: every candidate
+    int64_t *prev_n;           // [B] sequence length + 1 when its row was last written (0: never)
     int k, n_sink, n_local, cap, B, rps;
 };
 
@@ -484,6 +485,62 @@ sel_resolve(const SelArgs a)
 // ---------------------------------------------------------------------------
 // S4: ordered write of the selected ids; windows, count and padding
 // ---------------------------------------------------------------------------
+// A sequence that reuses its selection keeps its row unless its length
+// changed since the row was written (a cache that grows between decode
+// steps).  Then the row becomes: the sink window of the new length, the kept
+// top-k part (the old row's ids inside both the old and the new candidate
+// ranges), the local window of the new length, -1 padding; the count follows.
+// The old row is ascending, so the kept ids are one contiguous run of it; they
+// are staged in the sequence's candidate-list slots (unused in a reused step)
+// before the row is rewritten in place.  One block, all threads.
+__device__ void rewrite_reused_row(const SelArgs &a, int b, int64_t off, int64_t end)
+{
+    __shared__ uint32_t s_cnt[2];
+    const int64_t n_new = end - off;
+    const int64_t pn = __ldcg(&a.prev_n[b]);
+    if (pn == 0 || pn - 1 == n_new) {   // unknown or unchanged length: the row stays
+        if (threadIdx.x == 0)
+            a.prev_n[b] = n_new + 1;
+        return;
+    }
+    const Window wo = make_window(a, off, off + (pn - 1));
+    const Window wn = make_window(a, off, end);
+    int32_t *row = a.ids + (int64_t)b * a.cap;
+    const int m_old = max(0, min(__ldcg(a.count + b), a.cap));
+    const int64_t lo_id = max(wo.s_end, wn.s_end), hi_id = min(wo.l0, wn.l0);
+    if (threadIdx.x < 2)
+        s_cnt[threadIdx.x] = 0u;
+    __syncthreads();
+    uint32_t below_lo = 0, below_hi = 0;
+    for (int j = threadIdx.x; j < m_old; j += NT) {
+        const int32_t id = __ldcg(row + j);
+        below_lo += (id < lo_id) ? 1u : 0u;
+        below_hi += (id < hi_id) ? 1u : 0u;
+    }
+    atomicAdd(&s_cnt[0], below_lo);
+    atomicAdd(&s_cnt[1], below_hi);
+    __syncthreads();
+    const int j0 = (int)s_cnt[0];
+    const int nt = hi_id > lo_id ? min((int)s_cnt[1] - j0, a.k) : 0;   // at most the top-k part
+    uint32_t *stage = reinterpret_cast<uint32_t *>(a.cand + off);   // n_new >= nt slots of 8 bytes
+    for (int t = threadIdx.x; t < nt; t += NT)
+        stage[t] = (uint32_t)__ldcg(row + j0 + t);
+    __syncthreads();
+    const int64_t m_new = wn.s_end + nt + (wn.n - wn.l0);
+    for (int64_t i = threadIdx.x; i < wn.s_end; i += NT)
+        row[i] = (int32_t)i;
+    for (int t = threadIdx.x; t < nt; t += NT)
+        row[wn.s_end + t] = (int32_t)__ldcg(stage + t);
+    for (int64_t j = threadIdx.x; j < wn.n - wn.l0; j += NT)
+        row[wn.s_end + nt + j] = (int32_t)(wn.l0 + j);
+    for (int64_t j = m_new + threadIdx.x; j < a.cap; j += NT)
+        row[j] = -1;
+    if (threadIdx.x == 0) {
+        a.count[b] = (int32_t)m_new;
+        a.prev_n[b] = n_new + 1;
+    }
+}
+
 __global__ void __launch_bounds__(NT)
 sel_write(const SelArgs a)
 {
@@ -498,11 +555,16 @@ sel_write(const SelArgs a)
     const int md = __ldcg(&a.mode[b]);
     const unsigned long long T = __ldcg(&a.thr[b]);
     const uint32_t base = r < a.rps ? __ldcg(&a.range_off[(size_t)b * a.rps + r]) : 0u;
-    if (re != 0)
-        return;   // the previous ids stay
+    if (re != 0) {
+        if (r == 0)
+            rewrite_reused_row(a, b, off, end);   // the previous row, with the windows of a grown cache
+        return;
+    }
     const Window w = make_window(a, off, end);
     int32_t *idrow = a.ids + (int64_t)b * a.cap;
     if (r == 0) {
+        if (threadIdx.x == 0)
+            a.prev_n[b] = w.n + 1;
         const int64_t mcount = w.s_end + w.keff + (w.n - w.l0);
         for (int64_t i = threadIdx.x; i < w.s_end; i += NT)
             idrow[i] = (int32_t)i;
@@ -577,6 +639,7 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
     a.range_off = reinterpret_cast<uint32_t *>(ws + p.off_sel_range_off);
     a.thr = reinterpret_cast<unsigned long long *>(ws + p.off_sel_thr);
     a.mode = reinterpret_cast<int32_t *>(ws + p.off_sel_mode);
+    a.prev_n = reinterpret_cast<int64_t *>(ws + p.off_sel_prev_n);
     a.k = k;
     a.n_sink = n_sink;
     a.n_local = n_local;

@@ -127,7 +127,8 @@ struct Plan {
     int attn_splits;
     // workspace layout (byte offsets)
     size_t off_ctrl, off_chunk_table, off_L, off_partials, off_logits, off_sel_hist, off_sel_cand,
-        off_sel_inb1, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_vacc, off_attn_part,
+        off_sel_inb1, off_sel_bin, off_sel_above, off_sel_range_off, off_sel_thr, off_sel_mode, off_sel_prev_n,
+        off_vacc, off_attn_part,
         total_bytes;
 };
 
@@ -148,6 +149,11 @@ void *current_context();
 cudaError_t ensure_dyn_smem(const void *kernel, int bytes);
 
 // Launchers (return cudaGetLastError() of the launch).
+// One token appended at seq_offsets[1] (batch 1); ctrl[0] = 2 when full.
+cudaError_t launch_append(int64_t *seq_offsets, void *k_cache, void *v_cache, const void *k_new, const void *v_new,
+                          int64_t stride_tok, int64_t stride_head, int Hkv, int D, int64_t capacity, uint32_t *ctrl,
+                          cudaStream_t st);
+
 // In a graph replay the cosine kernel can switch off the conditional node
 // that holds the scoring and selection kernels: the last of its blocks sets
 // the node's condition to 0 when every sequence reuses its selection.

@@ -78,7 +78,8 @@ class _KV(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("seq_offsets_dev", ctypes.c_void_p),
                 ("seq_offsets_host", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
-                ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64), ("scale", ctypes.c_float)]
+                ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64), ("scale", ctypes.c_float),
+                ("capacity", ctypes.c_int64)]
 
 
 def test_decode_step_checks_everything_before_launching(lib):
@@ -129,3 +130,24 @@ def test_binding_refuses_host_tensors():
         ts.ts_score(kv, q, None, votes, ws)
     with pytest.raises(ValueError, match="GPU only"):
         ts.ts_selcache(q, q.clone(), torch.zeros(1, dtype=torch.int32), True, 0.9)
+
+
+def test_growing_cache_arguments_are_checked_on_the_host(lib):
+    """A cache with a capacity: one sequence only, capacity >= the current
+    length, and ts_append_kv refuses a cache without one; all decided on the
+    host before any device query."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    lib.ts_decode_step_kernels.restype = ctypes.c_int32
+    lib.ts_decode_step_kernels.argtypes = [ctypes.POINTER(_KV), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    off1 = (ctypes.c_int64 * 2)(0, 64)
+    off2 = (ctypes.c_int64 * 3)(0, 64, 128)
+    kv = _KV(1, 8, 4, 64, ctypes.addressof(off1), ctypes.addressof(off1), 16, 16, 256, 64, 0.0, -1)
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv), 16, 4, 8) == -1 and b">= 0" in lib.ts_last_error()
+    kv = _KV(2, 8, 4, 64, ctypes.addressof(off2), ctypes.addressof(off2), 16, 16, 256, 64, 0.0, 4096)
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv), 16, 4, 8) == -1 and b"one sequence" in lib.ts_last_error()
+    kv = _KV(1, 8, 4, 64, ctypes.addressof(off1), ctypes.addressof(off1), 16, 16, 256, 64, 0.0, 32)
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv), 16, 4, 8) == -1 and b"below" in lib.ts_last_error()
+    P = ctypes.c_void_p
+    lib.ts_append_kv.argtypes = [ctypes.POINTER(_KV), P, P, P, P, P, P, ctypes.c_size_t, P]
+    kv = _KV(1, 8, 4, 64, ctypes.addressof(off1), ctypes.addressof(off1), 16, 16, 256, 64, 0.0, 0)
+    assert lib.ts_append_kv(ctypes.byref(kv), None, None, None, None, None, None, 0, None) == 1
