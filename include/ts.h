@@ -184,7 +184,11 @@ TS_API ts_status_t ts_score_fused(const ts_kv_t *kv, const void *q, const int32_
  *           equal votes going to the lower token id
  *   ids[b, 0:count[b]] = sink U T U local in ascending order (sequence-local
  *   0-based ids), ids[b, count[b]:] = -1.
- * Sequences with reuse[b] != 0 keep their previous ids and count.
+ * Sequences with reuse[b] != 0 keep their previous ids and count, unless
+ * their length changed since those were written (a growing cache, see
+ * ts_append_kv): then the previous top-k part, the ids of the old row inside
+ * both the old and the new candidate ranges, is kept and the sink and local
+ * windows are those of the new length.
  *   votes      device float32 [seq_offsets[batch]] (non-negative, finite)
  *   ids        device int32 [batch, k + n_sink + n_local]
  *   count      device int32 [batch]
