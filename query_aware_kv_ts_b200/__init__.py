@@ -231,11 +231,13 @@ def ts_decode_step_kernels(kv: KVCache, k: int, n_sink: int, n_local: int) -> in
 
 
 def ts_get_device_status(ws, stream=None):
-    """Returns (status, site); status is TS_OK or TS_ERR_DEVICE_TIMEOUT."""
+    """Returns (status, site); status is TS_OK, TS_ERR_DEVICE_TIMEOUT (a bounded
+    device wait gave up) or TS_ERR_INVALID_ARG (ts_append_kv found the cache
+    full)."""
     site = ctypes.c_uint32(0)
     s = _lib.ts_get_device_status(_ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(site),
                                   _stream(stream))
-    if s not in (TS_OK, TS_ERR_DEVICE_TIMEOUT):
+    if s not in (TS_OK, TS_ERR_DEVICE_TIMEOUT, TS_ERR_INVALID_ARG):
         _check(s)
     return int(s), int(site.value)
 
