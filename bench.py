@@ -491,6 +491,16 @@ def run_ours(a, d: Dist):
                                                                        wl.bufs[l].ids, wl.bufs[l].count,
                                                                        wl.bufs[l].out, wl.bufs[l].ws)
                                                      for l in range(cfg.layers)])
+    # the same attention with its dot products on the CUDA cores (fp32 FMA)
+    # instead of the tensor cores, for the comparison
+    os.environ["TS_ATTN_CUDA_CORES"] = "1"
+    try:
+        kernels["sparse_attn_cuda_cores_us"] = 1e6 * one(
+            lambda i: [ts.ts_sparse_attn(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T], wl.bufs[l].ids,
+                                         wl.bufs[l].count, wl.bufs[l].out, wl.bufs[l].ws)
+                       for l in range(cfg.layers)])
+    finally:
+        del os.environ["TS_ATTN_CUDA_CORES"]
 
     # ---- end to end: pinned host query in, result out, every step ----
     q_host = [q.cpu().pin_memory() for q in wl.q]

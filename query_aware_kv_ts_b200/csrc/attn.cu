@@ -20,6 +20,8 @@
 // splits: a thread owns 4 output channels and every NG-th split, loads all of
 // them at once, and the NG split groups are combined through shared memory.
 // Each selected K/V row is read from HBM once for all G heads of its group.
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "ts_device.cuh"
@@ -46,10 +48,13 @@ struct AttnArgs {
     float scale_log2;   // scale * log2(e): logits in base-2 units
 };
 
-template <int D, int NB>
+// Dynamic shared memory of attn_split: K and V tiles, the logits, then the
+// tensor-core path's bf16 weight halves, or the CUDA-core path's fp32 queries.
+template <int D, int NB, bool TC>
 constexpr size_t attn_smem_bytes()
 {
-    return (size_t)2 * R * (D * 2 + 16) + (size_t)R * NB * 8 * 4 + (size_t)2 * NB * 8 * R * 2;
+    return (size_t)2 * R * (D * 2 + 16) + (size_t)R * NB * 8 * 4 +
+           (TC ? (size_t)2 * NB * 8 * R * 2 : (size_t)NB * 8 * D * 4);
 }
 
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x)
@@ -57,7 +62,11 @@ __device__ __forceinline__ uint16_t bf16_bits_rn(float x)
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-template <int D, int NB>
+// TC: logits and weighted sums on tensor cores (mma.sync, P split into a
+// bf16 head and remainder); otherwise on the CUDA cores in fp32 (one warp per
+// row for the logits, lanes splitting the channels; one thread per channel
+// pair and head for the weighted sums).
+template <int D, int NB, bool TC>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_split(const AttnArgs a)
 {
@@ -67,13 +76,13 @@ attn_split(const AttnArgs a)
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *sK = smem;
     uint8_t *sV = sK + R * RS;
-    float *sS = reinterpret_cast<float *>(sV + R * RS);          // [R][GM] logits (base 2)
-    uint16_t *sPh = reinterpret_cast<uint16_t *>(sS + R * GM);   // [GM][R] weights, bf16 high part
-    uint16_t *sPl = sPh + GM * R;                                 // [GM][R] bf16 remainder
-    __shared__ float s_m[GM], s_l[GM], s_M[GM], s_Linv[GM];
+    float *sS = reinterpret_cast<float *>(sV + R * RS);          // [R][GM] logits (base 2), then weights (CUDA cores)
+    uint16_t *sPh = reinterpret_cast<uint16_t *>(sS + R * GM);   // [GM][R] weights, bf16 high part (tensor cores)
+    uint16_t *sPl = sPh + GM * R;                                 // [GM][R] bf16 remainder (tensor cores)
+    float *sQ = sS + R * GM;                                      // [GM][D] fp32 queries (CUDA cores)
+    __shared__ float s_m[GM], s_l[GM];
     __shared__ int32_t s_id[R];
     __shared__ uint8_t s_valid[R];
-    __shared__ int s_last;
 
     pdl_wait();                 // ids and count come from the selection kernel
     pdl_launch_dependents();
@@ -123,27 +132,74 @@ attn_split(const AttnArgs a)
         }
     }
 
-    uint32_t bq[D / 16][NB][2];
+    uint32_t bq[TC ? D / 16 : 1][NB][2];
+    if constexpr (TC) {
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
+        for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            const int j = nb * 8 + r0;
-            if (j < G) {
-                const uint32_t *qp = reinterpret_cast<const uint32_t *>(
-                    a.q + ((int64_t)b * a.Hq + g * G + j) * D + ks * 16 + c0);
-                bq[ks][nb][0] = __ldg(qp);
-                bq[ks][nb][1] = __ldg(qp + 4);
-            } else {
-                bq[ks][nb][0] = 0u;
-                bq[ks][nb][1] = 0u;
+            for (int nb = 0; nb < NB; ++nb) {
+                const int j = nb * 8 + r0;
+                if (j < G) {
+                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(
+                        a.q + ((int64_t)b * a.Hq + g * G + j) * D + ks * 16 + c0);
+                    bq[ks][nb][0] = __ldg(qp);
+                    bq[ks][nb][1] = __ldg(qp + 4);
+                } else {
+                    bq[ks][nb][0] = 0u;
+                    bq[ks][nb][1] = 0u;
+                }
             }
+    } else {
+        // the G queries as fp32 in shared memory (rows j >= G stay unread)
+        for (int i = tid; i < G * D / 2; i += kAttnThreads) {
+            const int j = i / (D / 2), c = 2 * (i - j * (D / 2));
+            const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(a.q + ((int64_t)b * a.Hq + g * G + j) * D + c));
+            sQ[j * D + c] = bf16_lo(w);
+            sQ[j * D + c + 1] = bf16_hi(w);
         }
+    }
     cp_async_wait_all();
     __syncthreads();
 
     // ---- 2. logits S = Q K^T (base-2 units) ----------------------------------
-    const int nmb = (nrows + 15) / 16;
+    if constexpr (!TC) {
+        // one warp per row: lane l takes channels [l*D/32, (l+1)*D/32) of every
+        // head, then a butterfly sum leaves each head's dot product in every lane
+        constexpr int CPL = D / 32;
+        for (int r = warp; r < R; r += kAttnWarps) {
+            const bool rv = r < nrows && s_valid[r];
+            float kf[CPL];
+            if constexpr (CPL == 4) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(sK + r * RS + lane * 8);
+                kf[0] = bf16_lo(w.x);
+                kf[1] = bf16_hi(w.x);
+                kf[2] = bf16_lo(w.y);
+                kf[3] = bf16_hi(w.y);
+            } else {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(sK + r * RS + lane * 4);
+                kf[0] = bf16_lo(w);
+                kf[1] = bf16_hi(w);
+            }
+            float mine = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < GM; ++j) {
+                if (j < G) {
+                    float d = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i)
+                        d = fmaf(kf[i], sQ[j * D + lane * CPL + i], d);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        d += __shfl_xor_sync(0xffffffffu, d, o);
+                    if (lane == j)
+                        mine = d;
+                }
+            }
+            if (lane < GM)
+                sS[r * GM + lane] = (rv && lane < G) ? mine * a.scale_log2 : -INFINITY;
+        }
+    }
+    const int nmb = TC ? (nrows + 15) / 16 : 0;
     for (int mb = warp; mb < nmb; mb += kAttnWarps) {
         float acc[NB][4];
 #pragma unroll
@@ -195,9 +251,13 @@ attn_split(const AttnArgs a)
             const int r = lane + 32 * i;
             const float p = (mx == -INFINITY) ? 0.0f : exp2f(x[i] - mx);
             sum += p;
-            const uint16_t hb = bf16_bits_rn(p);
-            sPh[h * R + r] = hb;
-            sPl[h * R + r] = bf16_bits_rn(p - __uint_as_float((uint32_t)hb << 16));
+            if constexpr (TC) {
+                const uint16_t hb = bf16_bits_rn(p);
+                sPh[h * R + r] = hb;
+                sPl[h * R + r] = bf16_bits_rn(p - __uint_as_float((uint32_t)hb << 16));
+            } else {
+                sS[r * GM + h] = p;   // the weight replaces its logit (read above by this lane)
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
@@ -209,49 +269,81 @@ attn_split(const AttnArgs a)
     }
     __syncthreads();
 
-    // ---- 4. O^T = V^T P^T: warp w owns channels [16w, 16w + 16) --------------
-    float o[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[nb][e] = 0.0f;
-    if (warp < D / 16) {
-        const int cw = warp * 16;
-        const int nks = (nrows + 15) / 16;
-        for (int ks = 0; ks < nks; ++ks) {
-            const int rb = ks * 16;
-            const uint32_t addr = smem_u32(sV + (rb + (lane & 7) + ((lane >> 4) & 1) * 8) * RS) +
-                                  (uint32_t)((cw + ((lane >> 3) & 1) * 8) * 2);
-            uint32_t a0, a1, a2, a3;
-            ldmatrix_x4_trans(a0, a1, a2, a3, addr);
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int h = nb * 8 + r0;
-                const int rr = rb + c0;
-                const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr);
-                const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr + 8);
-                const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr);
-                const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr + 8);
-                mma_16816(o[nb], a0, a1, a2, a3, bh0, bh1);
-                mma_16816(o[nb], a0, a1, a2, a3, bl0, bl1);
-            }
-        }
-    }
-
-    // ---- 5. this split's partial ---------------------------------------------
     const int64_t GS = (int64_t)G * PS;
     float *mypart = a.part + (((int64_t)b * a.Hkv + g) * a.splits + sp) * GS;
-    if (warp < D / 16) {
+    if constexpr (!TC) {
+        // ---- 4'. O = P^T V on the CUDA cores: thread = (channel pair, heads
+        //          hg, hg + NH, ...); a warp shares its heads (weights broadcast)
+        constexpr int CP = D / 2;                    // channel pairs
+        constexpr int NH = kAttnThreads / CP;        // head groups
+        constexpr int HPT = (GM + NH - 1) / NH;      // heads per thread (at most)
+        const int cp = tid % CP, hg = tid / CP;
+        float o2[HPT][2];
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
+        for (int u = 0; u < HPT; ++u)
+            o2[u][0] = o2[u][1] = 0.0f;
+        for (int r = 0; r < nrows; ++r) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(sV + r * RS + cp * 4);
+            const float v0 = bf16_lo(w), v1 = bf16_hi(w);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int ch = warp * 16 + r0 + (e >= 2 ? 8 : 0);
-                const int h = nb * 8 + c0 + (e & 1);
-                if (h < G)
-                    mypart[h * PS + ch] = o[nb][e];
+            for (int u = 0; u < HPT; ++u) {
+                const int h = hg + u * NH;
+                if (h < G) {
+                    const float pw = sS[r * GM + h];
+                    o2[u][0] = fmaf(pw, v0, o2[u][0]);
+                    o2[u][1] = fmaf(pw, v1, o2[u][1]);
+                }
             }
+        }
+#pragma unroll
+        for (int u = 0; u < HPT; ++u) {
+            const int h = hg + u * NH;
+            if (h < G)
+                *reinterpret_cast<float2 *>(mypart + h * PS + 2 * cp) = make_float2(o2[u][0], o2[u][1]);
+        }
+    } else {
+        // ---- 4. O^T = V^T P^T: warp w owns channels [16w, 16w + 16) --------------
+        float o[NB][4];
+    #pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+    #pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[nb][e] = 0.0f;
+        if (warp < D / 16) {
+            const int cw = warp * 16;
+            const int nks = (nrows + 15) / 16;
+            for (int ks = 0; ks < nks; ++ks) {
+                const int rb = ks * 16;
+                const uint32_t addr = smem_u32(sV + (rb + (lane & 7) + ((lane >> 4) & 1) * 8) * RS) +
+                                      (uint32_t)((cw + ((lane >> 3) & 1) * 8) * 2);
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4_trans(a0, a1, a2, a3, addr);
+    #pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int h = nb * 8 + r0;
+                    const int rr = rb + c0;
+                    const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr);
+                    const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(sPh + h * R + rr + 8);
+                    const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr);
+                    const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(sPl + h * R + rr + 8);
+                    mma_16816(o[nb], a0, a1, a2, a3, bh0, bh1);
+                    mma_16816(o[nb], a0, a1, a2, a3, bl0, bl1);
+                }
+            }
+        }
+
+        // ---- 5. this split's partial ---------------------------------------------
+        if (warp < D / 16) {
+    #pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int ch = warp * 16 + r0 + (e >= 2 ? 8 : 0);
+                    const int h = nb * 8 + c0 + (e & 1);
+                    if (h < G)
+                        mypart[h * PS + ch] = o[nb][e];
+                }
+        }
     }
     if (tid < G) {
         mypart[tid * PS + D] = s_m[tid];
@@ -354,25 +446,39 @@ attn_merge(const AttnArgs a)
         make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
 }
 
-template <int D, int NB>
+template <int D, int NB, bool TC>
 cudaError_t launch_attn_t(const Plan &p, const AttnArgs &a, cudaStream_t st)
 {
-    constexpr size_t smem = attn_smem_bytes<D, NB>();
-    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void *>(attn_split<D, NB>), (int)smem);
+    constexpr size_t smem = attn_smem_bytes<D, NB, TC>();
+    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void *>(attn_split<D, NB, TC>), (int)smem);
     if (e != cudaSuccess)
         return e;
     dim3 grid((unsigned)p.attn_splits, (unsigned)p.Hkv, (unsigned)p.B);
-    e = launch_ex(attn_split<D, NB>, grid, dim3(kAttnThreads), smem, st, 1, a);
+    e = launch_ex(attn_split<D, NB, TC>, grid, dim3(kAttnThreads), smem, st, 1, a);
     if (e != cudaSuccess)
         return e;
     return launch_ex(attn_merge<D>, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(kAttnThreads), 0, st, 1, a);
 }
 
+// The logits and weighted sums run on the CUDA cores when the environment
+// sets TS_ATTN_CUDA_CORES=1 (read at every call; for comparing the two), on
+// the tensor cores otherwise.
+static bool attn_cuda_cores()
+{
+    const char *e = getenv("TS_ATTN_CUDA_CORES");
+    return e != nullptr && e[0] == '1';
+}
+
 cudaError_t launch_attn_any(const Plan &p, const AttnArgs &a, cudaStream_t st)
 {
+    if (attn_cuda_cores()) {
+        if (p.D == 128)
+            return p.G <= 8 ? launch_attn_t<128, 1, false>(p, a, st) : launch_attn_t<128, 2, false>(p, a, st);
+        return p.G <= 8 ? launch_attn_t<64, 1, false>(p, a, st) : launch_attn_t<64, 2, false>(p, a, st);
+    }
     if (p.D == 128)
-        return p.G <= 8 ? launch_attn_t<128, 1>(p, a, st) : launch_attn_t<128, 2>(p, a, st);
-    return p.G <= 8 ? launch_attn_t<64, 1>(p, a, st) : launch_attn_t<64, 2>(p, a, st);
+        return p.G <= 8 ? launch_attn_t<128, 1, true>(p, a, st) : launch_attn_t<128, 2, true>(p, a, st);
+    return p.G <= 8 ? launch_attn_t<64, 1, true>(p, a, st) : launch_attn_t<64, 2, true>(p, a, st);
 }
 
 AttnArgs make_args(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,

@@ -150,3 +150,18 @@ def test_fused_score_full_size(cfg_name):
         lo, hi = case.seq(b)
         v_ref, _ = H.oracle.votes(case.kb[lo:hi], qb[b], case.oracle_scale())
         H.check_votes(votes[lo:hi], v_ref, cfg.h_q)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_attention_on_cuda_cores(name, monkeypatch):
+    """The CUDA-core (fp32 FMA) variant of the sparse attention, selected with
+    TS_ATTN_CUDA_CORES=1, against the oracle's attention over the same ids."""
+    lengths, h_q, h_kv, d, k, s, l, extra = CASES[name]
+    case = _case(lengths, h_q, h_kv, d, seed=zlib.crc32(name.encode()) % 10000, **extra)
+    buf = H.run_step(case, k, s, l)
+    tc_out = buf.out.clone()
+    monkeypatch.setenv("TS_ATTN_CUDA_CORES", "1")
+    H.ts().ts_sparse_attn(case.kv, case.q, buf.ids, buf.count, buf.out, buf.ws)
+    torch.cuda.synchronize()
+    H.check_step(case, buf, k, s, l)
+    assert (buf.out - tc_out).abs().max().item() <= 2 * H.OUT_ATOL
