@@ -81,6 +81,23 @@ typedef enum {
  *                      capacity and every kernel takes the current length
  *                      from seq_offsets_dev, so one workspace and one
  *                      captured graph serve every length up to it.
+ *   page_size          0 (the layout above), or the tokens per page of a
+ *                      paged cache: then k and v are a pool of pool_pages
+ *                      pages of page_size token rows each (row r of the pool
+ *                      at k + r*stride_tok, same strides), and token i of
+ *                      sequence b sits in pool row
+ *                        page_table[b*page_table_stride + i/page_size]
+ *                          * page_size + i % page_size.
+ *                      seq_offsets still give the sequences' lengths and lay
+ *                      out the votes; ids stay sequence-local.  Supported:
+ *                      page_size a power of two, at least 128/h_kv (so that
+ *                      one scoring stage of 128/h_kv tokens lies in one page)
+ *                      and at most 4096; capacity 0.
+ *   page_table_dev     device int32 [batch * page_table_stride], the block
+ *                      table; entries of pages a sequence uses must be in
+ *                      [0, pool_pages) (the kernels skip others)
+ *   page_table_stride  entries per sequence, >= the pages of the longest
+ *   pool_pages         pages in the pool
  */
 typedef struct ts_kv {
     int32_t batch, h_q, h_kv, head_dim;
@@ -91,6 +108,9 @@ typedef struct ts_kv {
     int64_t stride_tok, stride_head;
     float scale;
     int64_t capacity;
+    int32_t page_size, page_table_stride;
+    int64_t pool_pages;
+    const int32_t *page_table_dev;
 } ts_kv_t;
 
 /*

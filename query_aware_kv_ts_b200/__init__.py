@@ -47,6 +47,9 @@ class ts_kv_t(ctypes.Structure):
         ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64),
         ("scale", ctypes.c_float),
         ("capacity", ctypes.c_int64),
+        ("page_size", ctypes.c_int32), ("page_table_stride", ctypes.c_int32),
+        ("pool_pages", ctypes.c_int64),
+        ("page_table_dev", ctypes.c_void_p),
     ]
 
 
@@ -113,10 +116,13 @@ class KVCache:
     k, v: bf16 CUDA tensors [sum_n, h_kv, d] (channel stride 1; token and head
     strides are read from the tensor); seq_offsets: int64 [B+1] (host array or
     tensor; a device copy is made once).  Keeps the ts_kv_t and the tensors it
-    points at alive together."""
+    points at alive together.
+
+    Paged cache: page_table (int32 [B, stride] on the device, the block table)
+    and page_size; k and v are then the pool, [pool_pages * page_size, h_kv, d]."""
 
     def __init__(self, k: torch.Tensor, v: torch.Tensor, seq_offsets, h_q: int, scale: float = 0.0,
-                 capacity: int = 0):
+                 capacity: int = 0, page_table: torch.Tensor | None = None, page_size: int = 0):
         if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
             raise TypeError("K and V must be bf16")
         if k.dim() != 3 or k.shape != v.shape or k.stride() != v.stride() or k.stride(2) != 1:
@@ -128,11 +134,20 @@ class KVCache:
         self.seq_offsets_dev = torch.from_numpy(off).to(k.device)
         self.batch = off.size - 1
         self.h_q, self.h_kv, self.head_dim = int(h_q), int(k.shape[1]), int(k.shape[2])
+        stride, pool_pages, table_ptr = 0, 0, None
+        if page_table is not None:
+            if page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_contiguous():
+                raise ValueError("page_table must be a contiguous int32 [batch, stride] tensor")
+            if page_size <= 0 or k.shape[0] % page_size:
+                raise ValueError("page_size must divide the pool's rows")
+            stride, pool_pages, table_ptr = page_table.shape[1], k.shape[0] // page_size, page_table.data_ptr()
+        self.page_table = page_table
         self.struct = ts_kv_t(self.batch, self.h_q, self.h_kv, self.head_dim,
                               self.seq_offsets_dev.data_ptr(),
                               off.ctypes.data_as(ctypes.c_void_p).value,
                               k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), float(scale),
-                              int(capacity))
+                              int(capacity), int(page_size if page_table is not None else 0), int(stride),
+                              int(pool_pages), table_ptr)
         self.capacity = int(capacity)
 
     @property

@@ -247,6 +247,41 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
         set_error("total tokens %lld must be below 2^31", (long long)n_total);
         return TS_ERR_UNSUPPORTED;
     }
+    // a paged cache: k and v are a pool of pages, a block table maps pages
+    p->paged = kv->page_size != 0;
+    p->kv_rows = n_total;
+    if (p->paged) {
+        const int64_t ps = kv->page_size;
+        if (ps < 0 || (ps & (ps - 1)) != 0 || ps > 4096 || ps < kScoreRows / kv->h_kv) {
+            set_error("page_size %lld must be a power of two in [128/h_kv = %d, 4096]", (long long)ps,
+                      kScoreRows / kv->h_kv);
+            return TS_ERR_UNSUPPORTED;
+        }
+        if (kv->capacity != 0) {
+            set_error("a paged cache cannot also have a capacity");
+            return TS_ERR_UNSUPPORTED;
+        }
+        if (kv->page_table_dev == nullptr || kv->pool_pages < 1 || kv->page_table_stride < 1) {
+            set_error("a paged cache needs page_table_dev, pool_pages >= 1 and page_table_stride >= 1");
+            return TS_ERR_INVALID_ARG;
+        }
+        if ((n_max + ps - 1) / ps > kv->page_table_stride) {
+            set_error("page_table_stride %d is below the %lld pages of the longest sequence", kv->page_table_stride,
+                      (long long)((n_max + ps - 1) / ps));
+            return TS_ERR_INVALID_ARG;
+        }
+        if (kv->pool_pages * ps >= (int64_t(1) << 31)) {
+            set_error("the pool's %lld rows must be below 2^31", (long long)(kv->pool_pages * ps));
+            return TS_ERR_UNSUPPORTED;
+        }
+        p->kv_rows = kv->pool_pages * ps;
+        int shift = 0;
+        while ((int64_t(1) << shift) < ps)
+            ++shift;
+        p->page_shift = shift;
+    } else {
+        p->page_shift = 0;
+    }
     if (n_max > (int64_t)kMaxSelectRanges * kSelectTokensPerCta) {
         set_error("sequence length %lld exceeds the supported maximum %lld", (long long)n_max,
                   (long long)kMaxSelectRanges * kSelectTokensPerCta);
@@ -402,7 +437,7 @@ static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *ma
         return TS_ERR_CUDA;
     }
     // dims (innermost first): channels, tokens, kv heads
-    cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.n_total, (cuuint64_t)p.Hkv};
+    cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.kv_rows, (cuuint64_t)p.Hkv};
     cuuint64_t strides[2] = {(cuuint64_t)kv->stride_tok * 2, (cuuint64_t)kv->stride_head * 2};
     cuuint32_t box[3] = {64u, fused ? (cuuint32_t)p.fused_t : (cuuint32_t)p.tile_tokens,
                          fused ? (cuuint32_t)p.fused_hs : (cuuint32_t)p.Hkv};
@@ -501,7 +536,7 @@ ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reu
     if (s != TS_OK)
         return s;
     cudaError_t e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, static_cast<uint8_t *>(ws),
-                                 static_cast<cudaStream_t>(stream));
+                                 static_cast<cudaStream_t>(stream), kv->page_table_dev, kv->page_table_stride);
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass A launch");
 }
 
@@ -543,6 +578,10 @@ ts_status_t ts_score_fused(const ts_kv_t *kv, const void *q, const int32_t *reus
     ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
     if (s != TS_OK)
         return s;
+    if (p.paged) {
+        set_error("ts_score_fused takes packed caches only (use ts_score for a paged cache)");
+        return TS_ERR_UNSUPPORTED;
+    }
     if (votes == nullptr) {
         set_error("votes is required");
         return TS_ERR_INVALID_ARG;
@@ -679,7 +718,8 @@ static ts_status_t decode_step_graph(const Plan &p, const CUtensorMap &kmap, con
     if (e != cudaSuccess)
         return cuda_fail(e, "ts_decode_step: body capture");
     const SelectWindow win = {k, n_sink, n_local};
-    cudaError_t le = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, side);
+    cudaError_t le = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, side,
+                                  kv->page_table_dev, kv->page_table_stride);
     if (le == cudaSuccess)
         le = launch_vote(p, kv->seq_offsets_dev, reuse, votes, w, side, &win);
     if (le == cudaSuccess)
@@ -752,7 +792,8 @@ ts_status_t ts_decode_step(const ts_kv_t *kv, const void *q, void *q_prev, int32
     if (e != cudaSuccess)
         return cuda_fail(e, "ts_decode_step: selection cache launch");
     if (p.n_total > 0) {
-        e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, st);
+        e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, w, st, kv->page_table_dev,
+                         kv->page_table_stride);
         if (e != cudaSuccess)
             return cuda_fail(e, "ts_decode_step: score pass A launch");
         const SelectWindow win = {k, n_sink, n_local};

@@ -46,6 +46,11 @@ struct AttnArgs {
     float *part;        // [B][Hkv][splits][G][D + 4]: D weighted-V sums, then (max, sum)
     int B, Hq, Hkv, G, splits;
     float scale_log2;   // scale * log2(e): logits in base-2 units
+    // paged cache (page_table != null): token i of sequence b is pool row
+    // page_table[b * pt_stride + (i >> page_shift)] << page_shift | (i & (page - 1))
+    const int32_t *page_table;
+    int pt_stride, page_shift;
+    int64_t pool_pages;
 };
 
 // Dynamic shared memory of attn_split: K and V tiles, the logits, then the
@@ -82,6 +87,7 @@ attn_split(const AttnArgs a)
     float *sQ = sS + R * GM;                                      // [GM][D] fp32 queries (CUDA cores)
     __shared__ float s_m[GM], s_l[GM];
     __shared__ int32_t s_id[R];
+    __shared__ int32_t s_row[R];   // the id's K / V row (its pool row in a paged cache)
     __shared__ uint8_t s_valid[R];
 
     pdl_wait();                 // ids and count come from the selection kernel
@@ -111,7 +117,17 @@ attn_split(const AttnArgs a)
             if (id < 0 || (int64_t)id >= n_b)
                 id = -1;                            // ids outside the sequence are ignored
         }
+        int32_t row = (int32_t)(off + id);
+        if (id >= 0 && a.page_table != nullptr) {
+            // one more round trip in a paged cache: the id's page
+            const int32_t pg = __ldcg(a.page_table + (int64_t)b * a.pt_stride + (id >> a.page_shift));
+            if (pg >= 0 && pg < a.pool_pages)
+                row = (pg << a.page_shift) | (id & ((1 << a.page_shift) - 1));
+            else
+                id = -1;                            // a page outside the pool: left out
+        }
         s_id[tid] = id;
+        s_row[tid] = row;
         s_valid[tid] = id >= 0 ? 1 : 0;
     }
     __syncthreads();
@@ -124,7 +140,7 @@ attn_split(const AttnArgs a)
             uint8_t *dst = (isV ? sV : sK) + r * RS + chunk * 16;
             const int32_t id = s_id[r];
             if (id >= 0) {
-                const __nv_bfloat16 *src = (isV ? a.v : a.k) + (off + id) * a.st + (int64_t)g * a.sh;
+                const __nv_bfloat16 *src = (isV ? a.v : a.k) + (int64_t)s_row[r] * a.st + (int64_t)g * a.sh;
                 cp_async_16(dst, reinterpret_cast<const uint8_t *>(src) + chunk * 16);
             } else if (isV) {
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);   // P is 0 there; V must be finite
@@ -502,6 +518,10 @@ AttnArgs make_args(const Plan &p, const ts_kv_t *kv, const void *q, const int32_
     a.G = p.G;
     a.splits = p.attn_splits;
     a.scale_log2 = p.scale * kLog2e;
+    a.page_table = p.paged ? kv->page_table_dev : nullptr;
+    a.pt_stride = p.paged ? kv->page_table_stride : 0;
+    a.page_shift = p.page_shift;
+    a.pool_pages = p.paged ? p.kv_rows >> p.page_shift : 0;
     return a;
 }
 

@@ -75,6 +75,12 @@ struct ScoreArgs {
     int64_t pf_off[33];       // B <= 32: the host copy of the offsets, for the prefetch hints only
     uint32_t tmem_cols;       // TMEM columns allocated (power of 2 >= 4 * N)
     float scale;
+    // paged cache (page_table != null): token i of sequence b is pool row
+    // page_table[b * pt_stride + (i >> page_shift)] << page_shift | (i & (page - 1))
+    const int32_t *page_table;
+    int pt_stride;
+    int page_shift;
+    int64_t pool_pages;
 };
 
 struct __align__(16) ScoreShared {
@@ -269,7 +275,11 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
     //      computed as if every sequence were active (a wrong guess costs
     //      nothing but bandwidth; the data itself is read after the wait) -----
     const int npf = NS < kMaxPrefetchTiles ? NS : kMaxPrefetchTiles;
-    if (B <= 32) {
+    if (a.page_table != nullptr) {
+        // a paged cache: no host copy of the block table, so no early hints
+        if (warp == kProducerWarp && lane == 0)
+            tma_prefetch_desc(&kmap);
+    } else if (B <= 32) {
         if (warp == kProducerWarp) {
             if (lane == 0)
                 tma_prefetch_desc(&kmap);
@@ -402,13 +412,37 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
     const int half_bytes = kScoreRows * 128;   // one 64-channel box
 
     if (warp == kProducerWarp) {
-        // ================= TMA producer: one elected lane ==================
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_first();
-            uint32_t it = 0;
-            for (int32_t v = v_begin; v < v_end; v += v_step, ++it) {
-                const int b = upper_seq(sh.chunk_start, B, v);
-                const int64_t t0 = sh.off[b] + (int64_t)(v - sh.chunk_start[b]) * T;
+        // ================= TMA producer ====================================
+        // The whole warp walks the chunks: every 32 chunks its lanes look up
+        // the K row where each chunk starts (one round trip for the block
+        // table of a paged cache), and lane 0 issues the loads.
+        const uint64_t pol = l2_policy_evict_first();
+        uint32_t it = 0;
+        int32_t my_row = 0;
+        bool stop = false;
+        for (int32_t v = v_begin; v < v_end && !stop; v += v_step, ++it) {
+            if ((it & 31u) == 0) {
+                const int32_t vl = v + (int32_t)lane * v_step;
+                my_row = 0;
+                if (vl < v_end) {
+                    const int bl = upper_seq(sh.chunk_start, B, vl);
+                    const int64_t i0 = (int64_t)(vl - sh.chunk_start[bl]) * T;   // first token of the chunk in its sequence
+                    if (a.page_table == nullptr) {
+                        my_row = (int32_t)(sh.off[bl] + i0);
+                    } else {
+                        // a chunk lies in one page (page size >= T, both powers of two);
+                        // an entry outside the pool reads out of bounds: zero keys
+                        const int32_t pg = __ldcg(a.page_table + (int64_t)bl * a.pt_stride + (i0 >> a.page_shift));
+                        const int64_t r = (pg >= 0 && pg < a.pool_pages)
+                                              ? ((int64_t)pg << a.page_shift) + (i0 & ((1 << a.page_shift) - 1))
+                                              : (a.pool_pages << a.page_shift);
+                        my_row = (int32_t)r;
+                    }
+                }
+            }
+            const int32_t row = __shfl_sync(0xffffffffu, my_row, (int)(it & 31u));
+            bool ok = true;
+            if (lane == 0) {
                 const int s = it % NS;
                 if (it >= (uint32_t)NS) {
                     const uint32_t par = ((it / NS) - 1) & 1;
@@ -419,15 +453,18 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
                         // tiles already in flight: the last NS issued stages
                         for (uint32_t j = it > (uint32_t)NS ? it - NS : 0u; j < it; ++j)
                             (void)mbar_wait_bounded(&sh.full[j % NS], (j / NS) & 1, kSpinLimit);
-                        break;
+                        ok = false;
                     }
                 }
-                mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
+                if (ok) {
+                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
 #pragma unroll
-                for (int x = 0; x < D / 64; ++x)
-                    tma_load_3d(stages + (size_t)s * a.stage_bytes + x * half_bytes, &kmap, &sh.full[s], x * 64,
-                                (int32_t)t0, 0, pol);
+                    for (int x = 0; x < D / 64; ++x)
+                        tma_load_3d(stages + (size_t)s * a.stage_bytes + x * half_bytes, &kmap, &sh.full[s], x * 64,
+                                    row, 0, pol);
+                }
             }
+            stop = !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
         }
         return;   // takes no part in the final barrier
     }
@@ -667,7 +704,8 @@ cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, ScoreArgs arg
 }  // namespace
 
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
-                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st)
+                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st,
+                         const int32_t *page_table, int page_table_stride)
 {
     ScoreArgs a;
     for (int b = 0; b <= 32; ++b)
@@ -689,6 +727,10 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.T = p.tile_tokens;
     a.stage_bytes = p.stage_bytes;
     a.scale = p.scale;
+    a.page_table = p.paged ? page_table : nullptr;
+    a.pt_stride = p.paged ? page_table_stride : 0;
+    a.page_shift = p.page_shift;
+    a.pool_pages = p.paged ? p.kv_rows >> p.page_shift : 0;
     cudaError_t e;
     // GP: columns per kv head in the MMA's N (the smallest of 4, 8, 16 that
     // holds the group); a small N keeps the query tile small and leaves

@@ -103,6 +103,9 @@ struct Plan {
     int B, Hq, Hkv, G, D;
     int64_t n_total;         // seq_offsets[B]
     int64_t n_max;           // longest sequence
+    bool paged;              // k, v are a pool of pages (block table in kv->page_table_dev)
+    int page_shift;          // log2(page_size) when paged
+    int64_t kv_rows;         // token rows of k and v: n_total, the capacity, or the pool's rows
     float scale;
     int sms;
     // score pass A
@@ -169,8 +172,10 @@ cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double 
 
 // seq_off_host: the host copy of the offsets (prefetch hints before the
 // dependency wait; the device copy decides the work).
+// page_table, page_table_stride: the block table of a paged cache (p.paged).
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
-                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st);
+                         const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st,
+                         const int32_t *page_table = nullptr, int page_table_stride = 0);
 
 // Selection parameters, for the vote pass that also builds the selection's
 // level-1 histogram.
