@@ -90,12 +90,14 @@ typedef enum {
  *                          * page_size + i % page_size.
  *                      seq_offsets still give the sequences' lengths and lay
  *                      out the votes; ids stay sequence-local.  Supported:
- *                      page_size a power of two, at least 128/h_kv (so that
- *                      one scoring stage of 128/h_kv tokens lies in one page)
- *                      and at most 4096; capacity 0.
+ *                      page_size a power of two in [8, 4096] (a scoring stage
+ *                      of 128/h_kv tokens that spans several pages is loaded
+ *                      one page and kv head at a time); capacity 0.
  *   page_table_dev     device int32 [batch * page_table_stride], the block
  *                      table; entries of pages a sequence uses must be in
- *                      [0, pool_pages) (the kernels skip others)
+ *                      [0, pool_pages): a page outside it reads as zero keys
+ *                      in the scoring and is left out of the attention (no
+ *                      access outside the pool; the results are not defined)
  *   page_table_stride  entries per sequence, >= the pages of the longest
  *   pool_pages         pages in the pool
  */

@@ -252,9 +252,8 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->kv_rows = n_total;
     if (p->paged) {
         const int64_t ps = kv->page_size;
-        if (ps < 0 || (ps & (ps - 1)) != 0 || ps > 4096 || ps < kScoreRows / kv->h_kv) {
-            set_error("page_size %lld must be a power of two in [128/h_kv = %d, 4096]", (long long)ps,
-                      kScoreRows / kv->h_kv);
+        if (ps < 8 || (ps & (ps - 1)) != 0 || ps > 4096) {
+            set_error("page_size %lld must be a power of two in [8, 4096]", (long long)ps);
             return TS_ERR_UNSUPPORTED;
         }
         if (kv->capacity != 0) {
@@ -303,6 +302,11 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     p->scale = kv->scale != 0.0f ? kv->scale : (float)(1.0 / sqrt((double)D));
     p->sms = sms;
     p->tile_tokens = kScoreRows / kv->h_kv;          // one stage = 128 K rows (h_kv heads x T tokens)
+    // pages shorter than a stage's T tokens: one TMA box {64, page, h_kv} per
+    // page (the stage's rows then go page by page), or for 8-token pages one
+    // box {64, 8, 1} per page and kv head (rows head by head as usual)
+    p->box_tokens = (p->paged && (1 << p->page_shift) < p->tile_tokens) ? (1 << p->page_shift) : p->tile_tokens;
+    p->box_heads = (p->box_tokens < p->tile_tokens && p->box_tokens < 16) ? 1 : kv->h_kv;
     p->stage_bytes = kScoreRows * D * 2;
     int64_t chunks = 0;
     for (int b = 0; b < kv->batch; ++b) {
@@ -313,10 +317,13 @@ ts_status_t make_plan(const ts_kv_t *kv, int capacity, Plan *p)
     const int grid_cap = sms < 256 ? sms : 256;
     p->score_grid = (int)(chunks < grid_cap ? chunks : grid_cap);
     {
-        // two stage parities x the lane quarters (32 rows each) one kv head's
-        // T = 128 / h_kv rows span
-        const int qph = p->tile_tokens > 32 ? p->tile_tokens / 32 : 1;
-        p->score_partials_per_slot = 2 * qph;
+        // two stage parities x the pieces of up to 32 tokens (one lane
+        // quarter's rows of one kv head) that a chunk of T = 128 / h_kv
+        // tokens of a head is cut into: blocks of EBT tokens of a head, EBT
+        // = T, or the page size when a paged stage goes page by page
+        const int ebt = p->box_heads > 1 ? p->box_tokens : p->tile_tokens;
+        const int span = ebt < 32 ? ebt : 32;
+        p->score_partials_per_slot = 2 * (p->tile_tokens / span);
     }
     p->ld_logits = (n_total + 3) / 4 * 4;
     {
@@ -428,7 +435,9 @@ static ts_status_t check_ws(const Plan &p, void *ws, size_t ws_bytes)
 // K as a 3-D tensor (channels, tokens, kv heads) for TMA.  fused: boxes of
 // {64, T, HS} (the fused scoring kernel, HS kv heads of T = 128 / HS tokens
 // per stage); else {64, T, h_kv} (the two-phase pass A, every head of
-// T = 128 / h_kv tokens per stage).
+// T = 128 / h_kv tokens per stage), or for a paged cache whose pages are
+// shorter than T {64, page, h_kv} (one box per page) or, for 8-token pages,
+// {64, 8, 1} (one box per page and kv head).
 static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *map, bool fused = false)
 {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -439,8 +448,8 @@ static ts_status_t encode_kmap(const Plan &p, const ts_kv_t *kv, CUtensorMap *ma
     // dims (innermost first): channels, tokens, kv heads
     cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.kv_rows, (cuuint64_t)p.Hkv};
     cuuint64_t strides[2] = {(cuuint64_t)kv->stride_tok * 2, (cuuint64_t)kv->stride_head * 2};
-    cuuint32_t box[3] = {64u, fused ? (cuuint32_t)p.fused_t : (cuuint32_t)p.tile_tokens,
-                         fused ? (cuuint32_t)p.fused_hs : (cuuint32_t)p.Hkv};
+    cuuint32_t box[3] = {64u, fused ? (cuuint32_t)p.fused_t : (cuuint32_t)p.box_tokens,
+                         fused ? (cuuint32_t)p.fused_hs : (cuuint32_t)p.box_heads};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(kv->k), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

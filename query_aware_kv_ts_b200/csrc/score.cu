@@ -81,6 +81,8 @@ struct ScoreArgs {
     int pt_stride;
     int page_shift;
     int64_t pool_pages;
+    int box_tokens;           // BT: tokens of one TMA box: T, or the page size when pages are shorter than T
+    int box_heads;            // kv heads of one TMA box: h_kv, or 1 (one box per page and kv head)
 };
 
 struct __align__(16) ScoreShared {
@@ -211,11 +213,9 @@ __device__ __forceinline__ void stage_queries(uint8_t *qs, const __nv_bfloat16 *
 // them.  No barrier: the warps of the CTA never wait for each other here.
 // (m, z) are consumed: on return they hold the warp's (max, sum) per head.
 template <int GP>
-__device__ __forceinline__ void score_flush(float (&m)[GP], float (&z)[GP], int G, int T, int span, int lane,
-                                            int warp, int g, float2 *partials, int64_t stride, int64_t slot_base)
+__device__ __forceinline__ void score_flush(float (&m)[GP], float (&z)[GP], int G, int span, int lane, int slot,
+                                            int g, float2 *partials, int64_t stride, int64_t slot_base)
 {
-    const int quarter = warp & 3, hs = warp >> 2;
-    const int qph = T > 32 ? T / 32 : 1;   // lane quarters per head
     const uint32_t grp = span == 32 ? 0xffffffffu : (lane < 16 ? 0x0000ffffu : 0xffff0000u);
 #pragma unroll
     for (int j = 0; j < GP; ++j) {
@@ -231,11 +231,10 @@ __device__ __forceinline__ void score_flush(float (&m)[GP], float (&z)[GP], int 
                 z[j] += __shfl_xor_sync(0xffffffffu, z[j], o);
         }
     if ((lane % span) == 0) {
-        const int r = hs * qph + (quarter % qph);
 #pragma unroll
         for (int j = 0; j < GP; ++j)
             if (j < G)
-                partials[(int64_t)(g * G + j) * stride + slot_base + r] = make_float2(m[j], z[j]);
+                partials[(int64_t)(g * G + j) * stride + slot_base + slot] = make_float2(m[j], z[j]);
     }
 }
 
@@ -413,37 +412,50 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
 
     if (warp == kProducerWarp) {
         // ================= TMA producer ====================================
-        // The whole warp walks the chunks: every 32 chunks its lanes look up
-        // the K row where each chunk starts (one round trip for the block
-        // table of a paged cache), and lane 0 issues the loads.
+        // The whole warp walks the chunks.  A warp-wide lookup finds the K
+        // row of every page of the next 32 / npp chunks, one page per lane
+        // (the block table of a paged cache costs one round trip per
+        // lookup), and lane 0 issues the loads.  npp = 1 unless a paged
+        // cache's pages are shorter than a chunk; then each page of the chunk
+        // arrives as one box {64, page, h_kv} (the epilogue reads the rows
+        // page by page), or, for 8-token pages, as one box {64, 8, 1} per kv
+        // head placed where the chunk's single box {64, T, h_kv} would have
+        // put those rows.
         const uint64_t pol = l2_policy_evict_first();
+        const int BT = a.box_tokens;                     // tokens of one box
+        const int npp = T / BT;                          // boxes along the tokens of a chunk (power of 2, <= 16)
+        const int cpb = 32 / npp;                        // chunks per lookup
+        const int64_t oob_row = a.pool_pages << a.page_shift;   // past the pool: reads zeros
         uint32_t it = 0;
         int32_t my_row = 0;
         bool stop = false;
         for (int32_t v = v_begin; v < v_end && !stop; v += v_step, ++it) {
-            if ((it & 31u) == 0) {
-                const int32_t vl = v + (int32_t)lane * v_step;
+            const int jb = (int)(it % (uint32_t)cpb);
+            if (jb == 0) {
+                const int32_t vl = v + (lane / npp) * v_step;
+                const int p = lane % npp;
                 my_row = 0;
                 if (vl < v_end) {
                     const int bl = upper_seq(sh.chunk_start, B, vl);
-                    const int64_t i0 = (int64_t)(vl - sh.chunk_start[bl]) * T;   // first token of the chunk in its sequence
+                    // first token of this lane's box in its sequence
+                    const int64_t i0 = (int64_t)(vl - sh.chunk_start[bl]) * T + (int64_t)p * BT;
                     if (a.page_table == nullptr) {
                         my_row = (int32_t)(sh.off[bl] + i0);
+                    } else if (i0 >= sh.off[bl + 1] - sh.off[bl]) {
+                        my_row = (int32_t)oob_row;       // a page past the sequence's end: never looked up
                     } else {
-                        // a chunk lies in one page (page size >= T, both powers of two);
-                        // an entry outside the pool reads out of bounds: zero keys
+                        // a box lies in one page (BT = min(T, page), both powers of two); an
+                        // entry outside the pool reads past the pool's rows: zero keys
                         const int32_t pg = __ldcg(a.page_table + (int64_t)bl * a.pt_stride + (i0 >> a.page_shift));
-                        const int64_t r = (pg >= 0 && pg < a.pool_pages)
-                                              ? ((int64_t)pg << a.page_shift) + (i0 & ((1 << a.page_shift) - 1))
-                                              : (a.pool_pages << a.page_shift);
-                        my_row = (int32_t)r;
+                        my_row = (pg >= 0 && pg < a.pool_pages)
+                                     ? (int32_t)(((int64_t)pg << a.page_shift) + (i0 & ((1 << a.page_shift) - 1)))
+                                     : (int32_t)oob_row;
                     }
                 }
             }
-            const int32_t row = __shfl_sync(0xffffffffu, my_row, (int)(it & 31u));
+            const int s = it % NS;
             bool ok = true;
             if (lane == 0) {
-                const int s = it % NS;
                 if (it >= (uint32_t)NS) {
                     const uint32_t par = ((it / NS) - 1) & 1;
                     if (!mbar_wait_bounded(&sh.empty[s], par, kSpinLimit)) {
@@ -456,15 +468,30 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
                         ok = false;
                     }
                 }
-                if (ok) {
+                if (ok)
                     mbar_arrive_expect_tx(&sh.full[s], (uint32_t)a.stage_bytes);
-#pragma unroll
-                    for (int x = 0; x < D / 64; ++x)
-                        tma_load_3d(stages + (size_t)s * a.stage_bytes + x * half_bytes, &kmap, &sh.full[s], x * 64,
-                                    row, 0, pol);
-                }
             }
             stop = !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
+            if (stop)
+                break;
+            uint8_t *dst = stages + (size_t)s * a.stage_bytes;
+            for (int p = 0; p < npp; ++p) {
+                const int32_t row = __shfl_sync(0xffffffffu, my_row, jb * npp + p);
+                if (lane == 0) {
+                    if (a.box_heads == a.Hkv) {
+#pragma unroll
+                        for (int x = 0; x < D / 64; ++x)
+                            tma_load_3d(dst + x * half_bytes + p * a.Hkv * BT * 128, &kmap, &sh.full[s], x * 64, row,
+                                        0, pol);
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < D / 64; ++x)
+                            for (int g = 0; g < a.Hkv; ++g)
+                                tma_load_3d(dst + x * half_bytes + (g * T + p * BT) * 128, &kmap, &sh.full[s],
+                                            x * 64, row, g, pol);
+                    }
+                }
+            }
         }
         return;   // takes no part in the final barrier
     }
@@ -542,10 +569,22 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
     } else {
         // ================= epilogue: warps 0-3, one TMEM lane each =========
         const int quarter = warp & 3, hs = warp >> 2;
+        // Row r of a stage holds kv head g, token t of the chunk.  The rows
+        // come in blocks of EBT tokens of one head, the h_kv blocks of a
+        // page side by side, then the next page: EBT = T (one block per
+        // head) unless a paged cache's pages are shorter than T and were
+        // loaded as one box of every kv head per page.
+        const int EBT = a.box_heads > 1 ? a.box_tokens : T;
+        const int PB = a.Hkv * EBT;                // rows of one page of blocks
         const int r = quarter * 32 + lane;         // accumulator row
-        const int g = r / T, t = r - g * T;        // kv head, token within the chunk
-        const int g_lo = (quarter * 32) / T;       // first kv head of this warp's rows
-        const int span = T < 32 ? T : 32;          // lanes of this warp with the same head
+        const int g = (r % PB) / EBT;              // kv head
+        const int t = (r / PB) * EBT + r % EBT;    // token within the chunk
+        const int g_lo = ((quarter * 32) % PB) / EBT;   // first kv head of this warp's rows
+        const int span = EBT < 32 ? EBT : 32;      // lanes of this warp with the same head
+        // this warp's partial slot for head g: the two stage parities x the
+        // span-token pieces of the chunk (the piece of this warp's first row
+        // of head g)
+        const int slot = hs * (T / span) + ((r - lane % span) / PB * EBT + (r - lane % span) % EBT) / span;
         const int G = a.G;
         const float scale = a.scale;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -555,7 +594,7 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
         uint32_t it = 0;
 
         auto flush_segment = [&]() {
-            score_flush<GP>(m, z, G, T, span, lane, warp, g, a.partials, (int64_t)a.S * a.R,
+            score_flush<GP>(m, z, G, span, lane, slot, g, a.partials, (int64_t)a.S * a.R,
                             ((int64_t)blockIdx.x + cur_b) * a.R);
         };
 
@@ -584,8 +623,8 @@ score_pass_a(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ S
             uint32_t raw[GP], raw2[GP];
             const uint32_t taddr = lane_base + (uint32_t)(buf * N + g_lo * GP);
             tmem_ld_32x32b<GP>(taddr, raw);
-            if (T < 32)
-                tmem_ld_32x32b<GP>(taddr + GP, raw2);   // h_kv = 8: two heads per lane quarter
+            if (span < 32)
+                tmem_ld_32x32b<GP>(taddr + GP, raw2);   // two heads per lane quarter
             tmem_wait_ld();
             tmem_fence_before();
             __syncwarp();
@@ -731,6 +770,8 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
     a.pt_stride = p.paged ? page_table_stride : 0;
     a.page_shift = p.page_shift;
     a.pool_pages = p.paged ? p.kv_rows >> p.page_shift : 0;
+    a.box_tokens = p.box_tokens;
+    a.box_heads = p.box_heads;
     cudaError_t e;
     // GP: columns per kv head in the MMA's N (the smallest of 4, 8, 16 that
     // holds the group); a small N keeps the query tile small and leaves

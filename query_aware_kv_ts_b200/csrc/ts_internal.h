@@ -110,6 +110,8 @@ struct Plan {
     int sms;
     // score pass A
     int tile_tokens;         // T: tokens per pipeline stage
+    int box_tokens;          // tokens of one TMA box of K: T, or a shorter page of a paged cache
+    int box_heads;           // kv heads of one TMA box of K: h_kv, or 1 for 8-token pages shorter than T
     int stage_bytes;
     int64_t max_chunks;      // sum_b ceil(n_b / T)
     int score_grid;          // <= 256

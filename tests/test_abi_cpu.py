@@ -79,7 +79,9 @@ class _KV(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("seq_offsets_dev", ctypes.c_void_p),
                 ("seq_offsets_host", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("stride_tok", ctypes.c_int64), ("stride_head", ctypes.c_int64), ("scale", ctypes.c_float),
-                ("capacity", ctypes.c_int64)]
+                ("capacity", ctypes.c_int64), ("page_size", ctypes.c_int32),
+                ("page_table_stride", ctypes.c_int32), ("pool_pages", ctypes.c_int64),
+                ("page_table_dev", ctypes.c_void_p)]
 
 
 def test_decode_step_checks_everything_before_launching(lib):
@@ -151,3 +153,31 @@ def test_growing_cache_arguments_are_checked_on_the_host(lib):
     lib.ts_append_kv.argtypes = [ctypes.POINTER(_KV), P, P, P, P, P, P, ctypes.c_size_t, P]
     kv = _KV(1, 8, 4, 64, ctypes.addressof(off1), ctypes.addressof(off1), 16, 16, 256, 64, 0.0, 0)
     assert lib.ts_append_kv(ctypes.byref(kv), None, None, None, None, None, None, 0, None) == 1
+
+
+def test_paged_cache_arguments_are_checked_on_the_host(lib):
+    """A paged cache: page size a power of two in [8, 4096], no capacity, a
+    block table with a row per sequence wide enough for the longest one, and
+    a pool below 2^31 rows; all decided on the host before any device query."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    lib.ts_decode_step_kernels.restype = ctypes.c_int32
+    lib.ts_decode_step_kernels.argtypes = [ctypes.POINTER(_KV), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    off = (ctypes.c_int64 * 3)(0, 100, 130)
+    table = (ctypes.c_int32 * 64)()
+
+    def kv(page, stride, pool, capacity=0, tab=ctypes.addressof(table)):
+        return _KV(2, 8, 4, 64, ctypes.addressof(off), ctypes.addressof(off), 16, 16, 256, 64, 0.0, capacity,
+                   page, stride, pool, tab)
+
+    for page in (4, 24, 8192):
+        assert lib.ts_decode_step_kernels(ctypes.byref(kv(page, 32, 64)), 16, 4, 8) == -1
+        assert b"page_size" in lib.ts_last_error()
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv(16, 32, 64, capacity=200)), 16, 4, 8) == -1
+    assert b"capacity" in lib.ts_last_error()
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv(16, 32, 64, tab=None)), 16, 4, 8) == -1
+    assert b"page_table_dev" in lib.ts_last_error()
+    # the longest sequence (100 tokens) needs 7 pages of 16
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv(16, 6, 64)), 16, 4, 8) == -1
+    assert b"page_table_stride" in lib.ts_last_error()
+    assert lib.ts_decode_step_kernels(ctypes.byref(kv(4096, 1, 1 << 19)), 16, 4, 8) == -1
+    assert b"2^31" in lib.ts_last_error()
