@@ -12,8 +12,9 @@ held in ``numpy.uint16`` arrays.
 
 Sources: the TokenSelect GitHub README ("Key Takeaways": per-head Q.K
 criticality, per-head soft voting, Selection Cache) and the GrooveSquid summary
-of the TokenSelect paper.  Readings of the open points (R1..R10) are listed at
-each function in ``ts_oracle.c``.
+of the TokenSelect paper; for the page-level comparator (``quest_*``), the
+Bohrium page for Quest (arXiv 2406.10774), Abstract and "Method Overview".
+Readings of the open points are listed at each function in ``ts_oracle.c``.
 """
 from __future__ import annotations
 
@@ -67,6 +68,14 @@ def _declare(lib):
     lib.oracle_sparse_attn.restype = None
     lib.oracle_dense_attn.argtypes = [P, P, i64, i32, i32, i64, i64, P, i32, f64, P]
     lib.oracle_dense_attn.restype = None
+    lib.oracle_quest_pages.argtypes = [i64, i64]
+    lib.oracle_quest_pages.restype = i64
+    lib.oracle_quest_meta.argtypes = [P, i64, i32, i32, i64, i64, i64, P, P]
+    lib.oracle_quest_meta.restype = None
+    lib.oracle_quest_scores.argtypes = [P, P, i64, i32, i32, P, i32, f64, P]
+    lib.oracle_quest_scores.restype = None
+    lib.oracle_quest_select.argtypes = [P, i64, i64, i64, i64, i64, P]
+    lib.oracle_quest_select.restype = i64
     return lib
 
 
@@ -339,3 +348,63 @@ def decode_loop(k, v, n0: int, qs, k_top: int, n_sink: int, n_local: int, theta:
         steps.append(rec)
         prev = rec
     return steps
+
+
+# ---------------------------------------------------------------------------
+# Page-level comparator (Quest's min/max page bounds)
+# ---------------------------------------------------------------------------
+
+def quest_pages(n: int, page_size: int) -> int:
+    """Pages of a sequence of n tokens: ceil(n / page_size)."""
+    return int(lib().oracle_quest_pages(int(n), int(page_size)))
+
+
+def quest_meta(k, page_size: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per-page element-wise (min, max) of one sequence's keys, bf16 bits
+    [pages, h_kv, d] each."""
+    k, st, sh = _kv_view(k)
+    n, h_kv, d = k.shape
+    pages = quest_pages(n, page_size)
+    kmin = np.empty((pages, h_kv, d), np.uint16)
+    kmax = np.empty((pages, h_kv, d), np.uint16)
+    lib().oracle_quest_meta(_ptr(k), n, h_kv, d, st, sh, int(page_size), _ptr(kmin), _ptr(kmax))
+    return kmin, kmax
+
+
+def quest_scores(kmin, kmax, q, scale: float | None = None) -> np.ndarray:
+    """Page scores (float64 [pages]): the per-head upper bounds of the scaled
+    logit over each page's min/max box, summed over the query heads."""
+    kmin = np.ascontiguousarray(_u16(kmin))
+    kmax = np.ascontiguousarray(_u16(kmax))
+    q = np.ascontiguousarray(_u16(q))
+    pages, h_kv, d = kmin.shape
+    h_q = q.shape[0]
+    if h_q % h_kv:
+        raise ValueError("h_q must be a multiple of h_kv")
+    out = np.empty(pages, np.float64)
+    lib().oracle_quest_scores(_ptr(kmin), _ptr(kmax), pages, h_kv, d, _ptr(q), h_q,
+                              default_scale(d) if scale is None else float(scale), _ptr(out))
+    return out
+
+
+def quest_select(scores, n: int, page_size: int, k: int, n_sink: int, n_local: int) -> tuple[np.ndarray, int]:
+    """Ascending ids (padded with -1 to k+s+l) and their count: the sink and
+    local windows plus the candidate tokens of the top floor(k / page_size)
+    candidate pages."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    assert scores.size == quest_pages(n, page_size)
+    ids = np.empty(k + n_sink + n_local, np.int32)
+    m = lib().oracle_quest_select(_ptr(scores), int(n), int(page_size), int(k), int(n_sink), int(n_local),
+                                  _ptr(ids))
+    return ids, int(m)
+
+
+def quest_step(k, v, q, page_size: int, k_top: int, n_sink: int, n_local: int,
+               scale: float | None = None):
+    """One sequence's page-level step: metadata, page scores, selection and
+    attention over the selected tokens.  Returns (scores, ids, count, out)."""
+    kmin, kmax = quest_meta(k, page_size)
+    sc = quest_scores(kmin, kmax, q, scale)
+    ids, m = quest_select(sc, k.shape[0], page_size, k_top, n_sink, n_local)
+    out = sparse_attn(k, v, q, ids, m, scale)
+    return sc, ids, m, out

@@ -19,8 +19,15 @@
  *   [TS-SUMMARY] GrooveSquid summary of the same paper (medium-difficulty
  *                summary): non-contiguous, token-level attention sparsity,
  *                per-head soft voting, Selection Cache, dot-product kernel.
+ *   [QUEST]      Bohrium page for "Quest: Query-Aware Sparsity for Efficient
+ *                Long-Context LLM Inference" (arXiv 2406.10774), Abstract and
+ *                "Method Overview" (4): each KV cache page keeps the minimal
+ *                and maximal key values; a page's criticality is estimated
+ *                from the element-wise products of the query with them; the
+ *                Top-K critical pages are loaded for attention.  Used here
+ *                only for the page-level comparator at the end of the file.
  * Where the pages leave a step open, the reading used is noted at the
- * function (readings R1..R19).
+ * function (readings R1..R19, R21..R23).
  *
  * Conventions shared by every function:
  *   - bf16 inputs are passed as raw uint16 bit patterns and widened exactly
@@ -366,4 +373,139 @@ void oracle_dense_attn(const uint16_t *k, const uint16_t *v, int64_t n,
         }
     }
     free(w);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Page-level comparator: Quest's min/max page bounds  [QUEST]              */
+/* ------------------------------------------------------------------------ */
+
+/* Pages of one sequence (reading R21): page j holds the sequence's tokens
+ * [j*P, min((j+1)*P, n)); there are ceil(n / P) of them, the last one
+ * possibly short. */
+int64_t oracle_quest_pages(int64_t n, int64_t P)
+{
+    return n <= 0 ? 0 : (n + P - 1) / P;
+}
+
+/* Per-page element-wise minimum and maximum of the keys, per kv head and
+ * channel [QUEST, Abstract: "keeps track of the minimal and maximal Key
+ * values in KV cache pages"].  Outputs are bf16 bit patterns laid out
+ * [page][kv head][channel]; the extremes of bf16 values are bf16 values.
+ * On equal values (+0 and -0) the earlier token's bits are kept. */
+void oracle_quest_meta(const uint16_t *k, int64_t n, int32_t h_kv, int32_t d,
+                       int64_t stride_tok, int64_t stride_head, int64_t P,
+                       uint16_t *kmin_out, uint16_t *kmax_out)
+{
+    int64_t pages = oracle_quest_pages(n, P);
+    for (int64_t j = 0; j < pages; ++j) {
+        int64_t t0 = j * P;
+        int64_t t1 = t0 + P < n ? t0 + P : n;
+        for (int32_t g = 0; g < h_kv; ++g) {
+            for (int32_t c = 0; c < d; ++c) {
+                uint16_t lo = k[t0 * stride_tok + (int64_t)g * stride_head + c];
+                uint16_t hi = lo;
+                for (int64_t t = t0 + 1; t < t1; ++t) {
+                    uint16_t x = k[t * stride_tok + (int64_t)g * stride_head + c];
+                    if (widen_bf16(x) < widen_bf16(lo))
+                        lo = x;
+                    if (widen_bf16(x) > widen_bf16(hi))
+                        hi = x;
+                }
+                int64_t o = (j * h_kv + g) * (int64_t)d + c;
+                kmin_out[o] = lo;
+                kmax_out[o] = hi;
+            }
+        }
+    }
+}
+
+/* Page criticality [QUEST, Method Overview (4)]: for query head h with kv
+ * head g(h) (R1), the largest value q_h . k can take over the box
+ * [kmin, kmax] of the page,
+ *   U_h(j) = scale * sum_c max(q_h[c] * kmin[j][g][c], q_h[c] * kmax[j][g][c]),
+ * an upper bound of the scaled logit of every key in the page.  One selection
+ * serves all heads of a sequence, so the page's score is the sum of the
+ * per-head bounds over the h_q query heads (reading R22):
+ *   score[j] = sum_h U_h(j). */
+void oracle_quest_scores(const uint16_t *kmin, const uint16_t *kmax, int64_t pages,
+                         int32_t h_kv, int32_t d, const uint16_t *q, int32_t h_q,
+                         double scale, double *score_out)
+{
+    int32_t group = h_q / h_kv;
+    for (int64_t j = 0; j < pages; ++j) {
+        double total = 0.0;
+        for (int32_t h = 0; h < h_q; ++h) {
+            int32_t g = h / group;
+            const uint16_t *qh = q + (int64_t)h * d;
+            const uint16_t *mn = kmin + (j * h_kv + g) * (int64_t)d;
+            const uint16_t *mx = kmax + (j * h_kv + g) * (int64_t)d;
+            double u = 0.0;
+            for (int32_t c = 0; c < d; ++c) {
+                double a = widen_bf16(qh[c]) * widen_bf16(mn[c]);
+                double b = widen_bf16(qh[c]) * widen_bf16(mx[c]);
+                u += a > b ? a : b;
+            }
+            total += scale * u;
+        }
+        score_out[j] = total;
+    }
+}
+
+/* Page selection with the token windows of R4 (reading R23): a page is a
+ * candidate when it holds at least one candidate token, i.e. when
+ * [max(j*P, s'), min((j+1)*P, l0)) is not empty.  The Top-K pages are the
+ * first min(floor(k / P), #candidates) candidate pages in (score desc, page
+ * asc) order [QUEST, Abstract: "only loading the Top-K critical KV cache
+ * pages"]; their candidate tokens join the sink and local windows:
+ *   ids = sort([0, s') U (tokens of the chosen pages n [s', l0)) U [l0, n)),
+ * at most s' + k + (n - l0) ids.  ids_out must hold k + n_sink + n_local
+ * entries; entries past the returned count are set to -1. */
+int64_t oracle_quest_select(const double *score, int64_t n, int64_t P, int64_t k,
+                            int64_t n_sink, int64_t n_local, int32_t *ids_out)
+{
+    int64_t cap = k + n_sink + n_local;
+    for (int64_t j = 0; j < cap; ++j)
+        ids_out[j] = -1;
+    if (n <= 0)
+        return 0;
+
+    int64_t s_end, l_begin;
+    oracle_windows(n, n_sink, n_local, &s_end, &l_begin);
+    unsigned char *chosen = (unsigned char *)calloc((size_t)n, 1);
+    for (int64_t i = 0; i < s_end; ++i)
+        chosen[i] = 1;
+    for (int64_t i = l_begin; i < n; ++i)
+        chosen[i] = 1;
+
+    int64_t pages = oracle_quest_pages(n, P);
+    vote_entry *e = (vote_entry *)malloc((size_t)(pages > 0 ? pages : 1) * sizeof(vote_entry));
+    int64_t nc = 0;
+    for (int64_t j = 0; j < pages; ++j) {
+        int64_t lo = j * P > s_end ? j * P : s_end;
+        int64_t hi = (j + 1) * P < l_begin ? (j + 1) * P : l_begin;
+        if (lo < hi) {
+            e[nc].v = score[j];
+            e[nc].i = j;
+            ++nc;
+        }
+    }
+    int64_t kp = k / P;
+    int64_t take = kp < nc ? kp : nc;
+    if (take > 0) {
+        qsort(e, (size_t)nc, sizeof(vote_entry), vote_entry_cmp);
+        for (int64_t x = 0; x < take; ++x) {
+            int64_t j = e[x].i;
+            int64_t lo = j * P > s_end ? j * P : s_end;
+            int64_t hi = (j + 1) * P < l_begin ? (j + 1) * P : l_begin;
+            for (int64_t i = lo; i < hi; ++i)
+                chosen[i] = 1;
+        }
+    }
+    free(e);
+    int64_t m = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (chosen[i])
+            ids_out[m++] = (int32_t)i;
+    free(chosen);
+    return m;
 }

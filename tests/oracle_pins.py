@@ -407,4 +407,150 @@ def pin_decode_loop_without_reuse_is_a_fresh_step():
         assert np.array_equal(st["out"], ref.out[0])
 
 
+# ------------------------------------------- page-level comparator (Quest)
+# Bohrium page for Quest (arXiv 2406.10774), Abstract and "Method Overview"
+# (4): per-page min/max keys, a query-dependent upper-bound criticality per
+# page, the Top-K pages loaded for attention.
+
+
+def pin_quest_hand_example():
+    c = _golden()["quest_pages"]
+    kb = _bits(c["keys"]).reshape(len(c["keys"]), 1, 4)
+    qb = _bits(c["q"])
+    kmin, kmax = oracle.quest_meta(kb, c["page_size"])
+    assert np.array_equal(kmin.reshape(-1, 4), _bits(c["kmin"])), kmin
+    assert np.array_equal(kmax.reshape(-1, 4), _bits(c["kmax"])), kmax
+    sc = oracle.quest_scores(kmin, kmax, qb)
+    assert np.array_equal(sc, _frac(c["scores"])), sc
+    for case in c["select"]:
+        ids, m = oracle.quest_select(sc, len(c["keys"]), c["page_size"], case["k"], c["n_sink"], c["n_local"])
+        assert m == case["count"] and ids[:m].tolist() == case["ids"], (ids, m)
+
+
+def _pages_np(kf, P):
+    """[pages] list of float64 [tokens, h_kv, d] slices (numpy slicing only)."""
+    n = kf.shape[0]
+    return [kf[j * P:min((j + 1) * P, n)] for j in range(-(-n // P))]
+
+
+def pin_quest_meta_is_the_page_box():
+    """Every key of a page lies in [kmin, kmax] and each bound is the value of
+    some key of that page (the extremes over exactly the page's tokens, the
+    short last page included); against numpy's min / max of the slices."""
+    for seed, n, h_kv, d, P in [(1, 100, 2, 64, 16), (2, 33, 4, 128, 8), (3, 7, 1, 64, 4), (4, 64, 2, 64, 64),
+                                (5, 5, 2, 64, 128)]:
+        kb, _, _ = _rand_case(seed, n, 2 * h_kv, h_kv, d)
+        kmin, kmax = oracle.quest_meta(kb, P)
+        kf = kb.astype(np.uint32) << 16
+        kf = kf.view(np.float32).astype(np.float64)
+        pages = _pages_np(kf, P)
+        assert kmin.shape == (len(pages), h_kv, d)
+        for j, pg in enumerate(pages):
+            lo = (kmin[j].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            hi = (kmax[j].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            assert np.array_equal(lo, pg.min(axis=0)), (seed, j)
+            assert np.array_equal(hi, pg.max(axis=0)), (seed, j)
+
+
+def pin_quest_one_token_pages_are_summed_logits():
+    """Pages of one token: the box is the key itself, so the page score is the
+    exact sum over query heads of the scaled dot products with that key."""
+    for seed, n, h_q, h_kv, d in [(11, 50, 8, 2, 64), (12, 20, 28, 4, 128), (13, 9, 4, 4, 64)]:
+        kb, _, qb = _rand_case(seed, n, h_q, h_kv, d)
+        kmin, kmax = oracle.quest_meta(kb, 1)
+        sc = oracle.quest_scores(kmin, kmax, qb)
+        kf = (kb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        qf = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        G = h_q // h_kv
+        want = np.zeros(n)
+        for h in range(h_q):
+            want += (kf[:, h // G, :] @ qf[h]) / math.sqrt(d)
+        assert np.allclose(sc, want, rtol=1e-12, atol=1e-12), (seed, np.abs(sc - want).max())
+
+
+def pin_quest_score_bounds_every_key():
+    """The page score bounds the head-summed scaled logit of every key of the
+    page, and is reached when the page's keys include the corner of the box
+    that each query head prefers (a page of one key per channel sign pattern
+    is not needed: a page of identical keys reaches it)."""
+    for seed, n, h_q, h_kv, d, P in [(21, 200, 8, 2, 64, 16), (22, 97, 28, 4, 128, 32), (23, 40, 4, 1, 64, 8)]:
+        kb, _, qb = _rand_case(seed, n, h_q, h_kv, d)
+        kmin, kmax = oracle.quest_meta(kb, P)
+        sc = oracle.quest_scores(kmin, kmax, qb)
+        kf = (kb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        qf = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        G = h_q // h_kv
+        summed = np.zeros(n)
+        for h in range(h_q):
+            summed += (kf[:, h // G, :] @ qf[h]) / math.sqrt(d)
+        for j in range(sc.size):
+            tok = summed[j * P:(j + 1) * P]
+            assert (tok <= sc[j] + 1e-9 * (1 + abs(sc[j]))).all(), (seed, j)
+        # identical keys in a page: the box is a point and the bound is exact
+        kb2 = np.repeat(kb[::P], P, axis=0)[:n]
+        sc2 = oracle.quest_scores(*oracle.quest_meta(kb2, P), qb)
+        kf2 = (kb2.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        s2 = np.zeros(n)
+        for h in range(h_q):
+            s2 += (kf2[:, h // G, :] @ qf[h]) / math.sqrt(d)
+        assert np.allclose(sc2, s2[::P], rtol=1e-12, atol=1e-12), seed
+
+
+def _brute_quest_select(sc, n, P, k, s, l):
+    """Rank counting over candidate pages: page j is chosen iff fewer than
+    floor(k / P) candidate pages precede it in (score desc, page asc) order."""
+    s_end = min(s, n)
+    l0 = max(n - l, s_end)
+    chosen = np.zeros(n, bool)
+    chosen[:s_end] = True
+    chosen[l0:] = True
+    pages = np.arange(-(-n // P)) if n > 0 else np.arange(0)
+    cand = np.array([j for j in pages if max(j * P, s_end) < min((j + 1) * P, l0)], np.int64)
+    kp = k // P
+    if cand.size and kp > 0:
+        v = sc[cand]
+        before = (v[None, :] > v[:, None]) | ((v[None, :] == v[:, None]) & (cand[None, :] < cand[:, None]))
+        for j in cand[before.sum(axis=1) < kp]:
+            chosen[max(j * P, s_end):min((j + 1) * P, l0)] = True
+    return np.nonzero(chosen)[0].astype(np.int32)
+
+
+def pin_quest_select_brute_force(seeds=600):
+    rng = np.random.default_rng(2406)
+    for _ in range(seeds):
+        n = int(rng.integers(0, 90))
+        P = int(rng.choice([1, 2, 4, 8, 16]))
+        k = int(rng.integers(0, 40))
+        s = int(rng.integers(0, 9))
+        l = int(rng.integers(0, 20))
+        sc = np.round(rng.standard_normal(-(-n // P)) * rng.choice([2, 8, 1 << 20])) / 4.0   # ties
+        ids, m = oracle.quest_select(sc, n, P, k, s, l)
+        want = _brute_quest_select(sc, n, P, k, s, l)
+        assert m == want.size and np.array_equal(ids[:m], want), (n, P, k, s, l)
+        assert (ids[m:] == -1).all() and m <= min(n, k + s + l)
+
+
+def pin_quest_one_token_pages_select_like_tokens():
+    """With one-token pages the page selection is the token-level top-k of the
+    same scores."""
+    rng = np.random.default_rng(7)
+    for n, k, s, l in [(300, 40, 4, 32), (50, 100, 2, 2), (64, 0, 4, 8)]:
+        sc = rng.standard_normal(n)
+        a = oracle.quest_select(sc, n, 1, k, s, l)
+        b = oracle.select(sc, k, s, l)
+        assert a[1] == b[1] and np.array_equal(a[0], b[0])
+
+
+def pin_quest_planted_pages_selected():
+    """Keys planted along the query dominate their pages' bounds: the pages
+    holding them are chosen."""
+    cfg = W.CONFIGS["tiny"]
+    li = W.layer_inputs(cfg)
+    kb, qb = W.bf16_bits(li.k), W.bf16_bits(li.q[0, 0])
+    P = 16
+    sc = oracle.quest_scores(*oracle.quest_meta(kb, P), qb)
+    ids, m = oracle.quest_select(sc, kb.shape[0], P, cfg.k, cfg.n_sink, cfg.n_local)
+    assert set(li.planted[0].tolist()) <= set(ids[:m].tolist())
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -41,6 +41,20 @@ MUTANTS = {
                                      "if (id >= s_old && id >= s_new && id < l0_new)"),
     "reuse_drops_topk_part": ("if (id >= s_old && id < l0_old && id >= s_new && id < l0_new)\n            chosen[id] = 1;",
                               "if (id < 0)\n            chosen[id] = 1;"),
+    # page-level comparator
+    "quest_meta_skips_last_token": ("for (int64_t t = t0 + 1; t < t1; ++t) {", "for (int64_t t = t0 + 1; t < t1 - 1; ++t) {"),
+    "quest_meta_page_off_by_one": ("int64_t t1 = t0 + P < n ? t0 + P : n;", "int64_t t1 = t0 + P + 1 < n ? t0 + P + 1 : n;"),
+    "quest_bound_takes_smaller_product": ("u += a > b ? a : b;", "u += a < b ? a : b;"),
+    "quest_bound_max_key_only": ("u += a > b ? a : b;", "u += b;"),
+    "quest_scores_drop_scale": ("total += scale * u;", "total += u;"),
+    "quest_scores_gqa_modulo": ("int32_t g = h / group;\n            const uint16_t *qh = q + (int64_t)h * d;\n            const uint16_t *mn",
+                                "int32_t g = h % h_kv;\n            const uint16_t *qh = q + (int64_t)h * d;\n            const uint16_t *mn"),
+    "quest_scores_max_over_heads": ("            total += scale * u;", "            total = total > scale * u ? total : scale * u;"),
+    "quest_budget_rounds_up": ("int64_t kp = k / P;", "int64_t kp = (k + P - 1) / P;"),
+    "quest_candidates_ignore_windows": ("        int64_t lo = j * P > s_end ? j * P : s_end;\n        int64_t hi = (j + 1) * P < l_begin ? (j + 1) * P : l_begin;\n        if (lo < hi) {",
+                                        "        int64_t lo = j * P;\n        int64_t hi = (j + 1) * P;\n        if (lo < hi) {"),
+    "quest_drops_pages_overlapping_the_sink": ("        if (lo < hi) {\n            e[nc].v = score[j];",
+                                               "        if (lo < hi && j * P >= s_end) {\n            e[nc].v = score[j];"),
 }
 
 
@@ -62,6 +76,8 @@ def test_mutant_is_caught(name, clean_source, tmp_path):
     with oracle.using_library(str(so)):
         for pin in oracle_pins.ALL_PINS:
             if pin is oracle_pins.pin_select_brute_force:
+                args = (150,)
+            elif pin is oracle_pins.pin_quest_select_brute_force:
                 args = (150,)
             else:
                 args = ()
