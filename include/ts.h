@@ -339,6 +339,74 @@ TS_API ts_status_t ts_get_device_status(void *ws, size_t ws_bytes, uint32_t *sit
  */
 TS_API ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_limit, void *stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Page-level comparator after Quest (Bohrium page for "Quest: Query-Aware
+ * Sparsity for Efficient Long-Context LLM Inference", arXiv 2406.10774:
+ * Abstract; Method Overview, item 4).  Each page of P consecutive tokens of a
+ * sequence keeps the element-wise minimum and maximum of its keys; a query
+ * bounds every key of the page from above with them; the Top-K pages by that
+ * bound are attended.  The selection has the same form as ts_select's (one
+ * ascending id row per sequence with the sink and local windows), so
+ * ts_sparse_attn attends over it unchanged.
+ *
+ * Pages: page j of sequence b holds its tokens [j*P, min((j+1)*P, n_b)), the
+ * last one possibly short; P is a power of two in [1, 4096].  The metadata
+ * and the scores have ts_quest_rows() rows; page j of sequence b is row
+ * (seq_offsets[b] / P) + b + j (at most one unused row per sequence; rows
+ * not holding a page are never written or read).  A cache with a capacity
+ * is laid out for the capacity; a paged KV cache (page_size != 0) is read
+ * through its block table, its page size independent of P.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Rows of the page metadata and scores of this cache for page size P,
+ * floor(n_total / P) + batch (n_total: the capacity of a growing cache), or
+ * -1 with ts_last_error set when kv or P is invalid.  Host only. */
+TS_API int64_t ts_quest_rows(const ts_kv_t *kv, int32_t page_size);
+
+/*
+ * Page metadata [Quest, Abstract: the minimal and maximal key values of each
+ * page]: kmin[row][g][c] and kmax[row][g][c] = the minimum and maximum over
+ * the page's tokens of K[token][g][c].
+ *   kmin, kmax   device bf16 [ts_quest_rows][h_kv][head_dim] each, 16-byte
+ *                aligned (caller-owned); only the rows of pages are written
+ * Reads K once; a growing cache's metadata is recomputed by calling again.
+ */
+TS_API ts_status_t ts_quest_metadata(const ts_kv_t *kv, int32_t page_size, void *kmin, void *kmax, void *stream);
+
+/*
+ * Page scores [Quest, Method Overview (4)]: with scale as in ts_score and
+ * kv head g(h) = h / (h_q / h_kv),
+ *   score[row of page j] = sum_h scale * sum_c max(q[h][c] * kmin[j][g(h)][c],
+ *                                                  q[h][c] * kmax[j][g(h)][c]),
+ * the per-head upper bound of the scaled logit over the page's min/max box,
+ * summed over the query heads (one selection serves all heads).  fp32,
+ * computed as one dot product per page of [kmax | kmin] with the query's
+ * head-summed positive and negative parts.
+ *   q            device bf16 [batch][h_q][head_dim], contiguous, 16-byte aligned
+ *   kmin, kmax   from ts_quest_metadata
+ *   scores       device fp32 [ts_quest_rows] (caller-owned); only the rows of
+ *                pages are written
+ */
+TS_API ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page_size, const void *kmin,
+                                  const void *kmax, float *scores, void *stream);
+
+/*
+ * Page selection with the token windows of ts_select: sink [0, s'),
+ * s' = min(n_sink, n); local [l0, n), l0 = max(n - n_local, s'); a page is a
+ * candidate when it holds a token of [s', l0).  The Top-K pages are the first
+ * min(floor(k / P), candidates) candidate pages by (score descending, page
+ * ascending) [Quest, Abstract: only the Top-K critical pages are loaded];
+ *   ids[b] = ascending [0, s') U (tokens of the chosen pages in [s', l0)) U [l0, n),
+ * count[b] = their number (at most s' + k + (n - l0)); ids[b][count..) = -1.
+ *   scores      from ts_quest_score
+ *   ids         device int32 [batch][k + n_sink + n_local]; count int32 [batch]
+ * One CTA per sequence (a radix select over the pages' scores); no workspace.
+ */
+TS_API ts_status_t ts_quest_select(const ts_kv_t *kv, const float *scores, int32_t page_size, int32_t k,
+                                   int32_t n_sink, int32_t n_local, int32_t *ids, int32_t *count, void *stream);
+
 TS_API const char *ts_status_string(ts_status_t status);
 
 /* Human-readable description of the calling thread's last error ("" if none). */

@@ -76,6 +76,10 @@ _SIGS = {
     "ts_append_kv": (ctypes.c_int, [_KV, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
+    "ts_quest_rows": (ctypes.c_int64, [_KV, _I32]),
+    "ts_quest_metadata": (ctypes.c_int, [_KV, _I32, _P, _P, _P]),
+    "ts_quest_score": (ctypes.c_int, [_KV, _P, _I32, _P, _P, _P, _P]),
+    "ts_quest_select": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ts_last_error": (ctypes.c_char_p, []),
 }
@@ -262,6 +266,29 @@ def ts_selftest_expire_wait(ws, spin_limit: int, stream=None):
                                         _stream(stream)))
 
 
+def ts_quest_rows(kv: KVCache, page_size: int) -> int:
+    """Rows of the page metadata and scores: floor(n_total / P) + batch."""
+    n = _lib.ts_quest_rows(kv.ref(), int(page_size))
+    if n < 0:
+        raise TsError(TS_ERR_INVALID_ARG, ts_last_error())
+    return int(n)
+
+
+def ts_quest_metadata(kv: KVCache, page_size: int, kmin, kmax, stream=None):
+    _check(_lib.ts_quest_metadata(kv.ref(), int(page_size), _ptr(kmin), _ptr(kmax), _stream(stream)))
+
+
+def ts_quest_score(kv: KVCache, q, page_size: int, kmin, kmax, scores, stream=None):
+    _check(_lib.ts_quest_score(kv.ref(), _ptr(q), int(page_size), _ptr(kmin), _ptr(kmax), _ptr(scores),
+                               _stream(stream)))
+
+
+def ts_quest_select(kv: KVCache, scores, page_size: int, k: int, n_sink: int, n_local: int, ids, count,
+                    stream=None):
+    _check(_lib.ts_quest_select(kv.ref(), _ptr(scores), int(page_size), int(k), int(n_sink), int(n_local),
+                                _ptr(ids), _ptr(count), _stream(stream)))
+
+
 def ts_status_string(status: int) -> str:
     return _status_name(status)
 
@@ -309,5 +336,29 @@ def decode_step(kv: KVCache, q, buf: StepBuffers, *, theta=None, first_step=True
         reuse = buf.reuse
     ts_score(kv, q, reuse, buf.votes, buf.ws, stream)
     ts_select(kv, buf.votes, buf.k, buf.n_sink, buf.n_local, reuse, buf.ids, buf.count, buf.ws, stream)
+    ts_sparse_attn(kv, q, buf.ids, buf.count, buf.out, buf.ws, stream)
+    return buf.out
+
+
+class QuestBuffers:
+    """Device buffers of the page-level comparator for one cache and page
+    size: the page metadata (kmin, kmax) and the page scores."""
+
+    def __init__(self, kv: KVCache, page_size: int):
+        rows = ts_quest_rows(kv, page_size)
+        dev = kv.k.device
+        self.page_size = int(page_size)
+        self.rows = rows
+        self.kmin = torch.empty((rows, kv.h_kv, kv.head_dim), dtype=torch.bfloat16, device=dev)
+        self.kmax = torch.empty((rows, kv.h_kv, kv.head_dim), dtype=torch.bfloat16, device=dev)
+        self.scores = torch.empty(rows, dtype=torch.float32, device=dev)
+
+
+def quest_step(kv: KVCache, q, qbuf: QuestBuffers, buf: StepBuffers, stream=None):
+    """Page scores -> page selection -> sparse attention, in stream order
+    (the metadata is computed beforehand with ts_quest_metadata); the ids,
+    count and output land in buf like decode_step's."""
+    ts_quest_score(kv, q, qbuf.page_size, qbuf.kmin, qbuf.kmax, qbuf.scores, stream)
+    ts_quest_select(kv, qbuf.scores, qbuf.page_size, buf.k, buf.n_sink, buf.n_local, buf.ids, buf.count, stream)
     ts_sparse_attn(kv, q, buf.ids, buf.count, buf.out, buf.ws, stream)
     return buf.out

@@ -906,6 +906,79 @@ ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_lim
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "selftest launch");
 }
 
+// ---------------------------------------------------------------------------
+// Page-level comparator
+// ---------------------------------------------------------------------------
+
+static ts_status_t quest_prologue(const ts_kv_t *kv, int32_t page_size, int capacity, Plan *p)
+{
+    if (page_size < 1 || page_size > 4096 || (page_size & (page_size - 1)) != 0) {
+        set_error("page_size %d must be a power of two in [1, 4096]", page_size);
+        return TS_ERR_INVALID_ARG;
+    }
+    return make_plan(kv, capacity, p);
+}
+
+int64_t ts_quest_rows(const ts_kv_t *kv, int32_t page_size)
+{
+    Plan p;
+    if (quest_prologue(kv, page_size, 1, &p) != TS_OK)
+        return -1;
+    return quest_rows(p, page_size);
+}
+
+ts_status_t ts_quest_metadata(const ts_kv_t *kv, int32_t page_size, void *kmin, void *kmax, void *stream)
+{
+    Plan p;
+    ts_status_t s = quest_prologue(kv, page_size, 1, &p);
+    if (s != TS_OK)
+        return s;
+    if (kmin == nullptr || kmax == nullptr ||
+        ((reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) & 15u)) {
+        set_error("kmin and kmax are required and must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_quest_meta(p, kv, page_size, kmin, kmax, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "quest metadata launch");
+}
+
+ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page_size, const void *kmin, const void *kmax,
+                           float *scores, void *stream)
+{
+    Plan p;
+    ts_status_t s = quest_prologue(kv, page_size, 1, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || kmin == nullptr || kmax == nullptr || scores == nullptr ||
+        ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) &
+         15u)) {
+        set_error("q, kmin, kmax and scores are required; q, kmin and kmax 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_quest_score(p, kv, q, page_size, kmin, kmax, scores, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "quest score launch");
+}
+
+ts_status_t ts_quest_select(const ts_kv_t *kv, const float *scores, int32_t page_size, int32_t k, int32_t n_sink,
+                            int32_t n_local, int32_t *ids, int32_t *count, void *stream)
+{
+    if (k < 0 || n_sink < 0 || n_local < 0) {
+        set_error("k, n_sink and n_local must be >= 0");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = quest_prologue(kv, page_size, k + n_sink + n_local, &p);
+    if (s != TS_OK)
+        return s;
+    if (scores == nullptr || ids == nullptr || count == nullptr) {
+        set_error("scores, ids and count are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_quest_select(p, kv, scores, page_size, k, n_sink, n_local, ids, count,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "quest select launch");
+}
+
 const char *ts_status_string(ts_status_t status)
 {
     switch (status) {

@@ -1,0 +1,507 @@
+// Page-level comparator after Quest (Bohrium page for "Quest: Query-Aware
+// Sparsity for Efficient Long-Context LLM Inference", arXiv 2406.10774:
+// Abstract; Method Overview, item 4): each page of P tokens keeps the
+// element-wise minimum and maximum of its keys; a query bounds every key of
+// the page from above through those two vectors; the Top-K pages by that
+// bound are attended.  Here one selection serves all heads of a sequence,
+// so a page's score is the per-head bound summed over the query heads, and
+// the chosen pages' tokens join the sink and local windows of the
+// token-level selection, in the same id rows that ts_sparse_attn reads.
+//
+// Layout: page j of sequence b (tokens [j*P, min((j+1)*P, n_b))) has row
+// (seq_offsets[b] >> log2 P) + b + j of the metadata and of the scores;
+// every kernel finds it from the offsets alone (no prefix sum), at the cost
+// of at most one unused row per sequence.
+//
+// All three kernels move little data per unit of work and are HBM- or
+// latency-bound, so they run on the CUDA cores: the metadata pass reads K
+// once (one warp per page, 16-byte loads, bf16x2 min / max); the score pass
+// reads the metadata once and folds the sum over heads into one dot product
+// per page (below); the selection is one CTA per sequence doing a radix
+// select over the pages' order keys.
+#include <cuda_bf16.h>
+
+#include "score_common.cuh"
+#include "ts_device.cuh"
+#include "ts_internal.h"
+
+namespace ts {
+
+namespace {
+
+constexpr int kQuestWarps = 8;              // pages handled together by one CTA of the metadata / score passes
+constexpr int kQuestSelThreads = 1024;      // one CTA per sequence
+constexpr int kQuestSelBins = 2048;         // radix digits of 11, 11 and 10 bits
+
+struct QuestKV {
+    const __nv_bfloat16 *k;
+    const int64_t *seq_off;      // device offsets [B+1]
+    int64_t st, sh;              // token and head strides (elements)
+    const int32_t *page_table;   // paged KV cache: block table [B][pt_stride], else null
+    int pt_stride, kv_page_shift;
+    int64_t pool_pages;
+    int Hkv, D;
+    int P_shift;                 // log2 of the comparator's page size
+};
+
+// K row of token i of sequence b, or -1 when a paged cache's entry lies
+// outside the pool.
+__device__ __forceinline__ int64_t token_row(const QuestKV &a, int b, int64_t off0, int64_t i)
+{
+    if (a.page_table == nullptr)
+        return off0 + i;
+    const int32_t pg = __ldg(a.page_table + (int64_t)b * a.pt_stride + (i >> a.kv_page_shift));
+    if (pg < 0 || pg >= a.pool_pages)
+        return -1;
+    return ((int64_t)pg << a.kv_page_shift) + (i & ((int64_t(1) << a.kv_page_shift) - 1));
+}
+
+__device__ __forceinline__ uint4 bf16x8_min(uint4 x, uint4 y)
+{
+    uint4 r;
+    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&x);
+    const __nv_bfloat162 *c = reinterpret_cast<const __nv_bfloat162 *>(&y);
+    __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(&r);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        o[e] = __hmin2(a[e], c[e]);
+    return r;
+}
+
+__device__ __forceinline__ uint4 bf16x8_max(uint4 x, uint4 y)
+{
+    uint4 r;
+    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&x);
+    const __nv_bfloat162 *c = reinterpret_cast<const __nv_bfloat162 *>(&y);
+    __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(&r);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        o[e] = __hmax2(a[e], c[e]);
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// Page metadata: one warp per page.  Lane l owns the 16-byte chunks l,
+// l + 32, ... (CH of them) of the h_kv * d channels of a token row; the
+// warp's lanes look up the rows of 32 tokens at a time and walk them, U
+// tokens' loads in flight.
+// ---------------------------------------------------------------------------
+template <int CH>
+__global__ void __launch_bounds__(kQuestWarps * 32)
+quest_meta(const QuestKV a, __nv_bfloat16 *kmin, __nv_bfloat16 *kmax)
+{
+    constexpr int U = 8 / CH;
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t off0 = a.seq_off[b];
+    const int64_t n = a.seq_off[b + 1] - off0;
+    const int64_t j = (int64_t)blockIdx.x * kQuestWarps + warp;   // page of the sequence
+    const int64_t t0 = j << a.P_shift;
+    if (t0 >= n)
+        return;
+    const int64_t t1 = min(t0 + (int64_t(1) << a.P_shift), n);
+    const int E8 = (a.Hkv * a.D) >> 3;                             // 16-byte chunks per token row
+    int64_t coff[CH];
+    bool cval[CH];
+    uint4 lo[CH], hi[CH];
+#pragma unroll
+    for (int x = 0; x < CH; ++x) {
+        const int q = lane + 32 * x;
+        cval[x] = q < E8;
+        const int e = (q << 3) % (a.Hkv * a.D);
+        coff[x] = (int64_t)(e / a.D) * a.sh + (e % a.D);
+        lo[x] = make_uint4(0x7f807f80u, 0x7f807f80u, 0x7f807f80u, 0x7f807f80u);   // +inf
+        hi[x] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);   // -inf
+    }
+    for (int64_t tb = t0; tb < t1; tb += 32) {
+        const int cnt = (int)min((int64_t)32, t1 - tb);
+        const int64_t my_row = lane < cnt ? token_row(a, b, off0, tb + lane) : -1;
+        for (int i = 0; i < cnt; i += U) {
+            uint4 v[U][CH];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t row = __shfl_sync(0xffffffffu, my_row, (i + u) & 31);
+                ok[u] = i + u < cnt && row >= 0;
+#pragma unroll
+                for (int x = 0; x < CH; ++x)
+                    if (ok[u] && cval[x])
+                        v[u][x] = __ldcs(reinterpret_cast<const uint4 *>(a.k + row * a.st + coff[x]));
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int x = 0; x < CH; ++x)
+                    if (ok[u] && cval[x]) {
+                        lo[x] = bf16x8_min(lo[x], v[u][x]);
+                        hi[x] = bf16x8_max(hi[x], v[u][x]);
+                    }
+        }
+    }
+    const int64_t out = (((a.seq_off[b] >> a.P_shift) + b + j) * (int64_t)(a.Hkv * a.D));
+#pragma unroll
+    for (int x = 0; x < CH; ++x)
+        if (cval[x]) {
+            const int q = lane + 32 * x;
+            *reinterpret_cast<uint4 *>(kmin + out + q * 8) = lo[x];
+            *reinterpret_cast<uint4 *>(kmax + out + q * 8) = hi[x];
+        }
+}
+
+// ---------------------------------------------------------------------------
+// Page scores.  For query head h of kv head g the bound of the page is
+//   scale * sum_c max(q_h[c] kmin[g][c], q_h[c] kmax[g][c])
+//     = scale * sum_c (max(q_h[c], 0) kmax[g][c] + min(q_h[c], 0) kmin[g][c]),
+// so the sum over the G heads of group g is one dot product of the page's
+// [kmax | kmin] row with the sequence's weights
+//   A[g][c] = scale * sum_h max(q_h[c], 0),  Bw[g][c] = scale * sum_h min(q_h[c], 0)
+// (fp32), which each lane keeps for its own channels.  One warp per U pages
+// (U pages' loads in flight), a shuffle sum per page.
+// ---------------------------------------------------------------------------
+template <int CH>
+__global__ void __launch_bounds__(kQuestWarps * 32)
+quest_score(const int64_t *seq_off, const __nv_bfloat16 *q, const __nv_bfloat16 *kmin, const __nv_bfloat16 *kmax,
+            float *scores, int Hq, int Hkv, int D, int P_shift, float scale)
+{
+    constexpr int U = 4 / CH > 0 ? 4 / CH : 1;
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t off0 = seq_off[b];
+    const int64_t n = seq_off[b + 1] - off0;
+    const int64_t pages = (n + (int64_t(1) << P_shift) - 1) >> P_shift;
+    const int64_t j0 = ((int64_t)blockIdx.x * kQuestWarps + warp) * U;
+    if (j0 >= pages)
+        return;
+    const int E = Hkv * D, E8 = E >> 3, G = Hq / Hkv;
+    float wA[CH][8], wB[CH][8];
+#pragma unroll
+    for (int x = 0; x < CH; ++x) {
+        const int qc = lane + 32 * x;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            wA[x][e] = wB[x][e] = 0.0f;
+        if (qc < E8) {
+            const int g = (qc * 8) / D, c = (qc * 8) % D;
+            for (int jh = 0; jh < G; ++jh) {
+                const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(q + ((int64_t)b * Hq + g * G + jh) * D + c));
+                const __nv_bfloat16 *qe = reinterpret_cast<const __nv_bfloat16 *>(&qv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float f = __bfloat162float(qe[e]);
+                    wA[x][e] += fmaxf(f, 0.0f);
+                    wB[x][e] += fminf(f, 0.0f);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                wA[x][e] *= scale;
+                wB[x][e] *= scale;
+            }
+        }
+    }
+    const int64_t row0 = (off0 >> P_shift) + b;
+    uint4 mn[U][CH], mx[U][CH];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int x = 0; x < CH; ++x) {
+            const int qc = lane + 32 * x;
+            if (j0 + u < pages && qc < E8) {
+                const int64_t o = (row0 + j0 + u) * E + qc * 8;
+                mn[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmin + o));
+                mx[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmax + o));
+            }
+        }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int x = 0; x < CH; ++x) {
+            const int qc = lane + 32 * x;
+            if (j0 + u < pages && qc < E8) {
+                const __nv_bfloat16 *lo = reinterpret_cast<const __nv_bfloat16 *>(&mn[u][x]);
+                const __nv_bfloat16 *hi = reinterpret_cast<const __nv_bfloat16 *>(&mx[u][x]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    acc = fmaf(wA[x][e], __bfloat162float(hi[e]), acc);
+                    acc = fmaf(wB[x][e], __bfloat162float(lo[e]), acc);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0 && j0 + u < pages)
+            scores[row0 + j0 + u] = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Page selection: one CTA per sequence.
+// ---------------------------------------------------------------------------
+
+// Exclusive prefix sum of one value per thread over the CTA (thread order);
+// returns the thread's prefix and leaves the total in *total.
+__device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o)
+            x += y;
+    }
+    if (lane == 31)
+        warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < nw ? warp_sums[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o)
+                s += y;
+        }
+        warp_sums[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    const uint32_t before = (warp > 0 ? warp_sums[warp - 1] : 0u) + x - v;
+    *total = warp_sums[nw - 1];
+    __syncthreads();           // warp_sums is reused by the next scan
+    return before;
+}
+
+// Ascending unsigned key of a score: larger score, larger key.
+__device__ __forceinline__ uint32_t score_key(float s)
+{
+    return (uint32_t)float_order_key(s) ^ 0x80000000u;
+}
+
+__global__ void __launch_bounds__(kQuestSelThreads)
+quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, int n_sink, int n_local, int cap,
+             int32_t *ids, int32_t *count)
+{
+    __shared__ uint32_t hist[kQuestSelBins];
+    __shared__ uint32_t warp_sums[32];
+    __shared__ uint32_t s_digit, s_above;
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int64_t off0 = seq_off[b];
+    const int64_t n = seq_off[b + 1] - off0;
+    const float *sc = scores + (off0 >> P_shift) + b;   // page j's score at sc[j]
+    int32_t *row = ids + (int64_t)b * cap;
+    const int64_t P = int64_t(1) << P_shift;
+    const int64_t s_end = n_sink < n ? n_sink : n;
+    const int64_t l0 = n - n_local > s_end ? n - n_local : s_end;
+    // candidate pages [jlo, jlo + nc): those with a token in [s_end, l0)
+    const int64_t jlo = s_end >> P_shift;
+    const int64_t nc = s_end < l0 ? ((l0 + P - 1) >> P_shift) - jlo : 0;
+    const int64_t kp = (int64_t)k >> P_shift;
+    const int64_t take = kp < nc ? kp : nc;
+
+    // threshold key T and the count of pages above it: every page with a key
+    // above T is chosen, then the first `need` pages (in page order) with key T
+    uint32_t T = 0u, need = 0u;
+    bool all = take == nc;              // every candidate (or none: nc == 0)
+    if (!all && take > 0) {
+        uint32_t prefix = 0u, pmask = 0u, above = 0u;
+        const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+        for (int pass = 0; pass < 3; ++pass) {
+            const int sh = shifts[pass], w = widths[pass];
+            const uint32_t dmask = (1u << w) - 1u;
+            for (int i = tid; i < kQuestSelBins; i += blockDim.x)
+                hist[i] = 0u;
+            __syncthreads();
+            for (int64_t c = tid; c < nc; c += blockDim.x) {
+                const uint32_t key = score_key(sc[jlo + c]);
+                if ((key & pmask) == prefix)
+                    atomicAdd(&hist[(key >> sh) & dmask], 1u);
+            }
+            __syncthreads();
+            // digits in descending order, two per thread: thread t holds
+            // digits (top - 2t, top - 2t - 1) of the 2^w used bins
+            const int top = (int)dmask;
+            const int d1 = top - 2 * tid, d2 = d1 - 1;
+            const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
+            uint32_t tot;
+            const uint32_t before = above + cta_exclusive_scan(h1 + h2, warp_sums, &tot);
+            if (d1 >= 0 && before < (uint32_t)take && before + h1 >= (uint32_t)take) {
+                s_digit = (uint32_t)d1;
+                s_above = before;
+            } else if (d2 >= 0 && before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
+                s_digit = (uint32_t)d2;
+                s_above = before + h1;
+            }
+            __syncthreads();
+            prefix |= s_digit << sh;
+            pmask |= dmask << sh;
+            above = s_above;
+            __syncthreads();
+        }
+        T = prefix;
+        need = (uint32_t)take - above;
+    }
+
+    // ordered passes: thread t owns candidate pages [t*R, (t+1)*R)
+    const int64_t R = (nc + blockDim.x - 1) / blockDim.x;
+    const int64_t c0 = (int64_t)tid * R, c1 = c0 + R < nc ? c0 + R : nc;
+    uint32_t eq = 0u;
+    if (!all && take > 0)
+        for (int64_t c = c0; c < c1; ++c)
+            eq += score_key(sc[jlo + c]) == T ? 1u : 0u;
+    uint32_t unused;
+    uint32_t eq_rank = cta_exclusive_scan(eq, warp_sums, &unused);
+    // tokens of the chosen pages in this thread's range
+    auto chosen = [&](int64_t c, uint32_t &rank) -> bool {
+        if (all)
+            return true;
+        if (take == 0)
+            return false;
+        const uint32_t key = score_key(sc[jlo + c]);
+        if (key > T)
+            return true;
+        if (key == T)
+            return rank++ < need;
+        return false;
+    };
+    auto cand_tokens = [&](int64_t c) -> int64_t {
+        const int64_t j = jlo + c;
+        const int64_t lo = (j << P_shift) > s_end ? (j << P_shift) : s_end;
+        const int64_t hi = ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0;
+        return hi - lo;
+    };
+    uint32_t ntok = 0u;
+    {
+        uint32_t rank = eq_rank;
+        for (int64_t c = c0; c < c1; ++c)
+            if (chosen(c, rank))
+                ntok += (uint32_t)cand_tokens(c);
+    }
+    uint32_t total_tok;
+    uint32_t pos = (uint32_t)s_end + cta_exclusive_scan(ntok, warp_sums, &total_tok);
+    {
+        uint32_t rank = eq_rank;
+        for (int64_t c = c0; c < c1; ++c)
+            if (chosen(c, rank)) {
+                const int64_t j = jlo + c;
+                const int64_t lo = (j << P_shift) > s_end ? (j << P_shift) : s_end;
+                const int64_t hi = ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0;
+                for (int64_t i = lo; i < hi; ++i)
+                    row[pos++] = (int32_t)i;
+            }
+    }
+    // the windows, the count and the padding
+    const int64_t m = s_end + total_tok + (n - l0);
+    for (int64_t i = tid; i < s_end; i += blockDim.x)
+        row[i] = (int32_t)i;
+    for (int64_t i = l0 + tid; i < n; i += blockDim.x)
+        row[s_end + total_tok + (i - l0)] = (int32_t)i;
+    for (int64_t i = m + tid; i < cap; i += blockDim.x)
+        row[i] = -1;
+    if (tid == 0)
+        count[b] = (int32_t)m;
+}
+
+int log2_exact(int x)
+{
+    int s = 0;
+    while ((1 << s) < x)
+        ++s;
+    return s;
+}
+
+QuestKV make_quest_kv(const Plan &p, const ts_kv_t *kv, int page_size)
+{
+    QuestKV a;
+    a.k = static_cast<const __nv_bfloat16 *>(kv->k);
+    a.seq_off = kv->seq_offsets_dev;
+    a.st = kv->stride_tok;
+    a.sh = kv->stride_head;
+    a.page_table = p.paged ? kv->page_table_dev : nullptr;
+    a.pt_stride = p.paged ? kv->page_table_stride : 0;
+    a.kv_page_shift = p.page_shift;
+    a.pool_pages = p.paged ? p.kv_rows >> p.page_shift : 0;
+    a.Hkv = p.Hkv;
+    a.D = p.D;
+    a.P_shift = log2_exact(page_size);
+    return a;
+}
+
+// 16-byte chunks of a token row per lane: 1, 2 or 4 (h_kv * d in 64 .. 1024)
+int chunks_per_lane(const Plan &p)
+{
+    const int e8 = p.Hkv * p.D / 8;
+    return e8 <= 32 ? 1 : (e8 <= 64 ? 2 : 4);
+}
+
+}  // namespace
+
+int64_t quest_rows(const Plan &p, int page_size)
+{
+    // sum over b of ceil(n_b / P) <= floor(n_total / P) + B (n_total: the
+    // capacity of a growing cache)
+    return p.n_total / page_size + p.B;
+}
+
+cudaError_t launch_quest_meta(const Plan &p, const ts_kv_t *kv, int page_size, void *kmin, void *kmax,
+                              cudaStream_t st)
+{
+    const QuestKV a = make_quest_kv(p, kv, page_size);
+    const int64_t max_pages = (p.n_max + page_size - 1) / page_size;
+    const dim3 grid((unsigned)((max_pages + kQuestWarps - 1) / kQuestWarps), (unsigned)p.B);
+    if (max_pages == 0)
+        return cudaSuccess;
+    __nv_bfloat16 *lo = static_cast<__nv_bfloat16 *>(kmin), *hi = static_cast<__nv_bfloat16 *>(kmax);
+    switch (chunks_per_lane(p)) {
+    case 1:
+        quest_meta<1><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        break;
+    case 2:
+        quest_meta<2><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        break;
+    default:
+        quest_meta<4><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quest_score(const Plan &p, const ts_kv_t *kv, const void *q, int page_size, const void *kmin,
+                               const void *kmax, float *scores, cudaStream_t st)
+{
+    const int ch = chunks_per_lane(p);
+    const int u = 4 / ch > 0 ? 4 / ch : 1;
+    const int64_t max_pages = (p.n_max + page_size - 1) / page_size;
+    if (max_pages == 0)
+        return cudaSuccess;
+    const int64_t per_cta = (int64_t)kQuestWarps * u;
+    const dim3 grid((unsigned)((max_pages + per_cta - 1) / per_cta), (unsigned)p.B);
+    const __nv_bfloat16 *qq = static_cast<const __nv_bfloat16 *>(q);
+    const __nv_bfloat16 *lo = static_cast<const __nv_bfloat16 *>(kmin), *hi = static_cast<const __nv_bfloat16 *>(kmax);
+    const int ps = log2_exact(page_size);
+    switch (ch) {
+    case 1:
+        quest_score<1><<<grid, kQuestWarps * 32, 0, st>>>(kv->seq_offsets_dev, qq, lo, hi, scores, p.Hq, p.Hkv, p.D,
+                                                         ps, p.scale);
+        break;
+    case 2:
+        quest_score<2><<<grid, kQuestWarps * 32, 0, st>>>(kv->seq_offsets_dev, qq, lo, hi, scores, p.Hq, p.Hkv, p.D,
+                                                         ps, p.scale);
+        break;
+    default:
+        quest_score<4><<<grid, kQuestWarps * 32, 0, st>>>(kv->seq_offsets_dev, qq, lo, hi, scores, p.Hq, p.Hkv, p.D,
+                                                         ps, p.scale);
+        break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quest_select(const Plan &p, const ts_kv_t *kv, const float *scores, int page_size, int k,
+                                int n_sink, int n_local, int32_t *ids, int32_t *count, cudaStream_t st)
+{
+    quest_select<<<p.B, kQuestSelThreads, 0, st>>>(scores, kv->seq_offsets_dev, log2_exact(page_size), k, n_sink,
+                                                   n_local, k + n_sink + n_local, ids, count);
+    return cudaGetLastError();
+}
+
+}  // namespace ts

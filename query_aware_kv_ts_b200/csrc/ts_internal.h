@@ -210,4 +210,14 @@ ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q,
 
 cudaError_t launch_selftest_wait(uint32_t *ctrl, uint32_t spin_limit, cudaStream_t st);
 
+// Page-level comparator (quest.cu): rows of the page metadata and scores,
+// page j of sequence b at row (seq_offsets[b] >> log2 P) + b + j.
+int64_t quest_rows(const Plan &p, int page_size);
+cudaError_t launch_quest_meta(const Plan &p, const ts_kv_t *kv, int page_size, void *kmin, void *kmax,
+                              cudaStream_t st);
+cudaError_t launch_quest_score(const Plan &p, const ts_kv_t *kv, const void *q, int page_size, const void *kmin,
+                               const void *kmax, float *scores, cudaStream_t st);
+cudaError_t launch_quest_select(const Plan &p, const ts_kv_t *kv, const float *scores, int page_size, int k,
+                                int n_sink, int n_local, int32_t *ids, int32_t *count, cudaStream_t st);
+
 }  // namespace ts
