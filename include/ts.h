@@ -361,8 +361,9 @@ TS_API ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t s
  */
 
 /* Rows of the page metadata and scores of this cache for page size P,
- * floor(n_total / P) + batch (n_total: the capacity of a growing cache), or
- * -1 with ts_last_error set when kv or P is invalid.  Host only. */
+ * floor(n_total / P) + batch rounded up to a multiple of 4 (n_total: the
+ * capacity of a growing cache), or -1 with ts_last_error set when kv or P
+ * is invalid.  Host only. */
 TS_API int64_t ts_quest_rows(const ts_kv_t *kv, int32_t page_size);
 
 /*
@@ -386,8 +387,8 @@ TS_API ts_status_t ts_quest_metadata(const ts_kv_t *kv, int32_t page_size, void 
  * head-summed positive and negative parts.
  *   q            device bf16 [batch][h_q][head_dim], contiguous, 16-byte aligned
  *   kmin, kmax   from ts_quest_metadata
- *   scores       device fp32 [ts_quest_rows] (caller-owned); only the rows of
- *                pages are written
+ *   scores       device fp32 [ts_quest_rows] (caller-owned), 16-byte aligned;
+ *                only the rows of pages are written
  */
 TS_API ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page_size, const void *kmin,
                                   const void *kmax, float *scores, void *stream);
@@ -400,9 +401,12 @@ TS_API ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page
  * ascending) [Quest, Abstract: only the Top-K critical pages are loaded];
  *   ids[b] = ascending [0, s') U (tokens of the chosen pages in [s', l0)) U [l0, n),
  * count[b] = their number (at most s' + k + (n - l0)); ids[b][count..) = -1.
- *   scores      from ts_quest_score
+ *   scores      from ts_quest_score (all ts_quest_rows entries readable)
  *   ids         device int32 [batch][k + n_sink + n_local]; count int32 [batch]
- * One CTA per sequence (a radix select over the pages' scores); no workspace.
+ * One CTA per sequence; no workspace.  The usual case (at most 2048 chosen
+ * pages, at most 2048 pages in the threshold's radix bucket) reads the
+ * scores three times; heavy ties or larger budgets take a general path that
+ * reads them five times.
  */
 TS_API ts_status_t ts_quest_select(const ts_kv_t *kv, const float *scores, int32_t page_size, int32_t k,
                                    int32_t n_sink, int32_t n_local, int32_t *ids, int32_t *count, void *stream);

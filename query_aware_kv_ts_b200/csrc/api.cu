@@ -950,9 +950,9 @@ ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page_size, 
     if (s != TS_OK)
         return s;
     if (q == nullptr || kmin == nullptr || kmax == nullptr || scores == nullptr ||
-        ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) &
-         15u)) {
-        set_error("q, kmin, kmax and scores are required; q, kmin and kmax 16-byte aligned");
+        ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax) |
+          reinterpret_cast<uintptr_t>(scores)) & 15u)) {
+        set_error("q, kmin, kmax and scores are required and 16-byte aligned");
         return TS_ERR_INVALID_ARG;
     }
     cudaError_t e = launch_quest_score(p, kv, q, page_size, kmin, kmax, scores, static_cast<cudaStream_t>(stream));
@@ -970,8 +970,8 @@ ts_status_t ts_quest_select(const ts_kv_t *kv, const float *scores, int32_t page
     ts_status_t s = quest_prologue(kv, page_size, k + n_sink + n_local, &p);
     if (s != TS_OK)
         return s;
-    if (scores == nullptr || ids == nullptr || count == nullptr) {
-        set_error("scores, ids and count are required");
+    if (scores == nullptr || ids == nullptr || count == nullptr || (reinterpret_cast<uintptr_t>(scores) & 15u)) {
+        set_error("scores, ids and count are required; scores 16-byte aligned");
         return TS_ERR_INVALID_ARG;
     }
     cudaError_t e = launch_quest_select(p, kv, scores, page_size, k, n_sink, n_local, ids, count,

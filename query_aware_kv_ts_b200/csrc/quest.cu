@@ -163,14 +163,15 @@ __global__ void __launch_bounds__(kQuestWarps * 32)
 quest_score(const int64_t *seq_off, const __nv_bfloat16 *q, const __nv_bfloat16 *kmin, const __nv_bfloat16 *kmax,
             float *scores, int Hq, int Hkv, int D, int P_shift, float scale)
 {
-    constexpr int U = 4 / CH > 0 ? 4 / CH : 1;
+    constexpr int U = 4 / CH > 0 ? 4 / CH : 1;   // pages per batch: 8 16-byte loads per lane
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t off0 = seq_off[b];
     const int64_t n = seq_off[b + 1] - off0;
     const int64_t pages = (n + (int64_t(1) << P_shift) - 1) >> P_shift;
-    const int64_t j0 = ((int64_t)blockIdx.x * kQuestWarps + warp) * U;
-    if (j0 >= pages)
+    const int64_t wid = (int64_t)blockIdx.x * kQuestWarps + warp;
+    const int64_t wstride = (int64_t)gridDim.x * kQuestWarps * U;
+    if (wid * U >= pages)
         return;
     const int E = Hkv * D, E8 = E >> 3, G = Hq / Hkv;
     float wA[CH][8], wB[CH][8];
@@ -201,38 +202,54 @@ quest_score(const int64_t *seq_off, const __nv_bfloat16 *q, const __nv_bfloat16 
     }
     const int64_t row0 = (off0 >> P_shift) + b;
     uint4 mn[U][CH], mx[U][CH];
+    auto load = [&](int64_t j0) {
 #pragma unroll
-    for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int x = 0; x < CH; ++x) {
-            const int qc = lane + 32 * x;
-            if (j0 + u < pages && qc < E8) {
-                const int64_t o = (row0 + j0 + u) * E + qc * 8;
-                mn[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmin + o));
-                mx[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmax + o));
+            for (int x = 0; x < CH; ++x) {
+                const int qc = lane + 32 * x;
+                if (j0 + u < pages && qc < E8) {
+                    const int64_t o = (row0 + j0 + u) * E + qc * 8;
+                    mn[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmin + o));
+                    mx[u][x] = __ldcs(reinterpret_cast<const uint4 *>(kmax + o));
+                }
             }
-        }
+    };
+    int64_t j0 = wid * U;
+    load(j0);
+    while (j0 < pages) {
+        // the batch's dot products, then the next batch's loads go out
+        // before the shuffle sums and the stores
+        float acc[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        float acc = 0.0f;
+        for (int u = 0; u < U; ++u) {
+            acc[u] = 0.0f;
 #pragma unroll
-        for (int x = 0; x < CH; ++x) {
-            const int qc = lane + 32 * x;
-            if (j0 + u < pages && qc < E8) {
-                const __nv_bfloat16 *lo = reinterpret_cast<const __nv_bfloat16 *>(&mn[u][x]);
-                const __nv_bfloat16 *hi = reinterpret_cast<const __nv_bfloat16 *>(&mx[u][x]);
+            for (int x = 0; x < CH; ++x) {
+                const int qc = lane + 32 * x;
+                if (j0 + u < pages && qc < E8) {
+                    const __nv_bfloat16 *lo = reinterpret_cast<const __nv_bfloat16 *>(&mn[u][x]);
+                    const __nv_bfloat16 *hi = reinterpret_cast<const __nv_bfloat16 *>(&mx[u][x]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    acc = fmaf(wA[x][e], __bfloat162float(hi[e]), acc);
-                    acc = fmaf(wB[x][e], __bfloat162float(lo[e]), acc);
+                    for (int e = 0; e < 8; ++e) {
+                        acc[u] = fmaf(wA[x][e], __bfloat162float(hi[e]), acc[u]);
+                        acc[u] = fmaf(wB[x][e], __bfloat162float(lo[e]), acc[u]);
+                    }
                 }
             }
         }
+        const int64_t jn = j0 + wstride;
+        if (jn < pages)
+            load(jn);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0 && j0 + u < pages)
-            scores[row0 + j0 + u] = acc;
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+            if (lane == 0 && j0 + u < pages)
+                scores[row0 + j0 + u] = acc[u];
+        }
+        j0 = jn;
     }
 }
 
@@ -272,11 +289,54 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t *war
     return before;
 }
 
-// Ascending unsigned key of a score: larger score, larger key.
+// Ascending unsigned key of a score: larger score, larger key; -0 and +0
+// are the same score (equal scores go to the lower page).
 __device__ __forceinline__ uint32_t score_key(float s)
 {
-    return (uint32_t)float_order_key(s) ^ 0x80000000u;
+    return (uint32_t)float_order_key(s == 0.0f ? 0.0f : s) ^ 0x80000000u;
 }
+
+// The page selection, one CTA of 1024 threads per sequence.  Candidate
+// pages [jlo, jlo + nc) are those holding a token of [s_end, l0); `take`
+// of them are chosen.
+//
+// Fast path (at most 2048 pages to choose, the usual case): the keys' min
+// and max span 2048 equal bins; one histogram over them finds the threshold
+// bin (equal bins in key space spread a concentrated score distribution
+// over many bins, so the histogram's shared atomics rarely collide); one
+// more pass puts the sure winners (a higher bin) and the threshold bin's
+// pages in shared memory, where the
+// rest is decided by counting ranks: the bucket's pages by (key desc, page
+// asc), the chosen pages by page for their token positions.  Three
+// coalesced passes over the scores.  When the threshold digit holds more
+// than 2048 pages (heavy ties), the general path takes over: a three-digit
+// radix select over all 32 key bits, then two passes in page order over a
+// contiguous range per thread (the ranks among pages tied at the threshold,
+// then the tokens).  Five passes; any number of candidates and ties.
+// Calls f(c, key) for this thread's candidates c = tid, tid + blockDim.x, ...
+// < nc, with kQSelBatch loads in flight.
+constexpr int kQSelBatch = 8;
+template <typename F>
+__device__ __forceinline__ void for_each_key(const float *sc, int64_t nc, F f)
+{
+    for (int64_t c0 = threadIdx.x; c0 < nc; c0 += (int64_t)kQSelBatch * blockDim.x) {
+        float v[kQSelBatch];
+#pragma unroll
+        for (int u = 0; u < kQSelBatch; ++u) {
+            const int64_t c = c0 + (int64_t)u * blockDim.x;
+            v[u] = c < nc ? __ldcg(sc + c) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kQSelBatch; ++u) {
+            const int64_t c = c0 + (int64_t)u * blockDim.x;
+            if (c < nc)
+                f(c, score_key(v[u]));
+        }
+    }
+}
+
+constexpr int kQSelList = 2048;     // chosen pages the fast path holds
+constexpr int kQSelBucket = 2048;   // pages of the threshold digit it holds
 
 __global__ void __launch_bounds__(kQuestSelThreads)
 quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, int n_sink, int n_local, int cap,
@@ -284,8 +344,13 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
 {
     __shared__ uint32_t hist[kQuestSelBins];
     __shared__ uint32_t warp_sums[32];
-    __shared__ uint32_t s_digit, s_above;
-    const int b = blockIdx.x, tid = threadIdx.x;
+    __shared__ uint32_t warp_lo[32], warp_hi[32];
+    __shared__ uint32_t s_kmin, s_kmax, s_digit, s_above, s_nlist, s_nbucket;
+    __shared__ int32_t list[kQSelList];
+    __shared__ uint32_t bkey[kQSelBucket];
+    __shared__ int32_t bidx[kQSelBucket];
+    __shared__ uint32_t spos[kQSelList];
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t off0 = seq_off[b];
     const int64_t n = seq_off[b + 1] - off0;
     const float *sc = scores + (off0 >> P_shift) + b;   // page j's score at sc[j]
@@ -293,102 +358,215 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
     const int64_t P = int64_t(1) << P_shift;
     const int64_t s_end = n_sink < n ? n_sink : n;
     const int64_t l0 = n - n_local > s_end ? n - n_local : s_end;
-    // candidate pages [jlo, jlo + nc): those with a token in [s_end, l0)
     const int64_t jlo = s_end >> P_shift;
     const int64_t nc = s_end < l0 ? ((l0 + P - 1) >> P_shift) - jlo : 0;
     const int64_t kp = (int64_t)k >> P_shift;
     const int64_t take = kp < nc ? kp : nc;
+    auto page_lo = [&](int64_t j) { return (j << P_shift) > s_end ? (j << P_shift) : s_end; };
+    auto page_hi = [&](int64_t j) { return ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0; };
 
-    // threshold key T and the count of pages above it: every page with a key
-    // above T is chosen, then the first `need` pages (in page order) with key T
-    uint32_t T = 0u, need = 0u;
-    bool all = take == nc;              // every candidate (or none: nc == 0)
-    if (!all && take > 0) {
-        uint32_t prefix = 0u, pmask = 0u, above = 0u;
-        const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
-        for (int pass = 0; pass < 3; ++pass) {
-            const int sh = shifts[pass], w = widths[pass];
-            const uint32_t dmask = (1u << w) - 1u;
+    uint32_t total_tok = 0u;
+    if (take == nc) {
+        // every candidate page (or none): every token of [s_end, l0)
+        total_tok = nc > 0 ? (uint32_t)(l0 - s_end) : 0u;
+        for (int64_t i = s_end + tid; i < s_end + total_tok; i += blockDim.x)
+            row[i] = (int32_t)i;
+    } else if (take > 0) {
+        bool fast = take <= kQSelList;
+        // digit of a key: its place among 2048 equal bins over [kmin, kmax]
+        // of the keys (a monotone map: a higher digit is a larger key)
+        uint32_t kbase = 0u;
+        float kscale = 0.0f;
+        auto digit_of = [&](uint32_t key) {
+            const uint32_t d = (uint32_t)((float)(key - kbase) * kscale);
+            return d < (uint32_t)(kQuestSelBins - 1) ? d : (uint32_t)(kQuestSelBins - 1);
+        };
+        if (fast) {
+            // pass 1: the smallest and largest key
+            uint32_t lo = 0xffffffffu, hi = 0u;
+            for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) {
+                lo = key < lo ? key : lo;
+                hi = key > hi ? key : hi;
+            });
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint32_t a2 = __shfl_xor_sync(0xffffffffu, lo, o), b2 = __shfl_xor_sync(0xffffffffu, hi, o);
+                lo = a2 < lo ? a2 : lo;
+                hi = b2 > hi ? b2 : hi;
+            }
+            if (lane == 0) {
+                warp_lo[warp] = lo;
+                warp_hi[warp] = hi;
+            }
             for (int i = tid; i < kQuestSelBins; i += blockDim.x)
                 hist[i] = 0u;
             __syncthreads();
-            for (int64_t c = tid; c < nc; c += blockDim.x) {
-                const uint32_t key = score_key(sc[jlo + c]);
-                if ((key & pmask) == prefix)
-                    atomicAdd(&hist[(key >> sh) & dmask], 1u);
+            if (warp == 0) {
+                lo = warp_lo[lane];
+                hi = warp_hi[lane];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const uint32_t a2 = __shfl_xor_sync(0xffffffffu, lo, o), b2 = __shfl_xor_sync(0xffffffffu, hi, o);
+                    lo = a2 < lo ? a2 : lo;
+                    hi = b2 > hi ? b2 : hi;
+                }
+                if (lane == 0) {
+                    s_kmin = lo;
+                    s_kmax = hi;
+                }
             }
             __syncthreads();
-            // digits in descending order, two per thread: thread t holds
-            // digits (top - 2t, top - 2t - 1) of the 2^w used bins
-            const int top = (int)dmask;
-            const int d1 = top - 2 * tid, d2 = d1 - 1;
-            const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
-            uint32_t tot;
-            const uint32_t before = above + cta_exclusive_scan(h1 + h2, warp_sums, &tot);
-            if (d1 >= 0 && before < (uint32_t)take && before + h1 >= (uint32_t)take) {
-                s_digit = (uint32_t)d1;
-                s_above = before;
-            } else if (d2 >= 0 && before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
-                s_digit = (uint32_t)d2;
-                s_above = before + h1;
+            kbase = s_kmin;
+            kscale = (float)kQuestSelBins / ((float)(s_kmax - s_kmin) + 1.0f);
+            // pass 2: the digit histogram
+            for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) { atomicAdd(&hist[digit_of(key)], 1u); });
+            __syncthreads();
+            // the threshold digit: digits in descending order, two per thread
+            {
+                const int d1 = kQuestSelBins - 1 - 2 * tid, d2 = d1 - 1;
+                const uint32_t h1 = hist[d1], h2 = hist[d2];
+                uint32_t tot;
+                const uint32_t before = cta_exclusive_scan(h1 + h2, warp_sums, &tot);
+                if (before < (uint32_t)take && before + h1 >= (uint32_t)take) {
+                    s_digit = (uint32_t)d1;
+                    s_above = before;
+                } else if (before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
+                    s_digit = (uint32_t)d2;
+                    s_above = before + h1;
+                }
+                if (tid == 0) {
+                    s_nlist = 0u;
+                    s_nbucket = 0u;
+                }
             }
             __syncthreads();
-            prefix |= s_digit << sh;
-            pmask |= dmask << sh;
-            above = s_above;
-            __syncthreads();
+            fast = hist[s_digit] <= (uint32_t)kQSelBucket;   // the same for every thread
+            __syncthreads();   // read by all before the general path rewrites hist
         }
-        T = prefix;
-        need = (uint32_t)take - above;
-    }
-
-    // ordered passes: thread t owns candidate pages [t*R, (t+1)*R)
-    const int64_t R = (nc + blockDim.x - 1) / blockDim.x;
-    const int64_t c0 = (int64_t)tid * R, c1 = c0 + R < nc ? c0 + R : nc;
-    uint32_t eq = 0u;
-    if (!all && take > 0)
-        for (int64_t c = c0; c < c1; ++c)
-            eq += score_key(sc[jlo + c]) == T ? 1u : 0u;
-    uint32_t unused;
-    uint32_t eq_rank = cta_exclusive_scan(eq, warp_sums, &unused);
-    // tokens of the chosen pages in this thread's range
-    auto chosen = [&](int64_t c, uint32_t &rank) -> bool {
-        if (all)
-            return true;
-        if (take == 0)
-            return false;
-        const uint32_t key = score_key(sc[jlo + c]);
-        if (key > T)
-            return true;
-        if (key == T)
-            return rank++ < need;
-        return false;
-    };
-    auto cand_tokens = [&](int64_t c) -> int64_t {
-        const int64_t j = jlo + c;
-        const int64_t lo = (j << P_shift) > s_end ? (j << P_shift) : s_end;
-        const int64_t hi = ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0;
-        return hi - lo;
-    };
-    uint32_t ntok = 0u;
-    {
-        uint32_t rank = eq_rank;
-        for (int64_t c = c0; c < c1; ++c)
-            if (chosen(c, rank))
-                ntok += (uint32_t)cand_tokens(c);
-    }
-    uint32_t total_tok;
-    uint32_t pos = (uint32_t)s_end + cta_exclusive_scan(ntok, warp_sums, &total_tok);
-    {
-        uint32_t rank = eq_rank;
-        for (int64_t c = c0; c < c1; ++c)
-            if (chosen(c, rank)) {
-                const int64_t j = jlo + c;
-                const int64_t lo = (j << P_shift) > s_end ? (j << P_shift) : s_end;
-                const int64_t hi = ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0;
-                for (int64_t i = lo; i < hi; ++i)
-                    row[pos++] = (int32_t)i;
+        if (fast) {
+            const uint32_t digit = s_digit, above = s_above;
+            // pass 3: the sure winners and the threshold digit's pages
+            for_each_key(sc + jlo, nc, [&](int64_t c, uint32_t key) {
+                const uint32_t d = digit_of(key);
+                if (d > digit) {
+                    list[atomicAdd(&s_nlist, 1u)] = (int32_t)c;
+                } else if (d == digit) {
+                    const uint32_t slot = atomicAdd(&s_nbucket, 1u);
+                    bkey[slot] = key;
+                    bidx[slot] = (int32_t)c;
+                }
+            });
+            __syncthreads();
+            // the bucket, ranked by (key desc, page asc): the first take - above join the list
+            const uint32_t nb = s_nbucket, need = (uint32_t)take - above;
+            for (uint32_t e = tid; e < nb; e += blockDim.x) {
+                const uint32_t ke = bkey[e];
+                const int32_t ie = bidx[e];
+                uint32_t rank = 0u;
+                for (uint32_t f = 0; f < nb; ++f)
+                    rank += (bkey[f] > ke || (bkey[f] == ke && bidx[f] < ie)) ? 1u : 0u;
+                if (rank < need)
+                    list[above + rank] = ie;
             }
+            __syncthreads();
+            // the chosen pages in page order: rank by counting, token counts by rank
+            const uint32_t nl = (uint32_t)take;
+            constexpr int kPer = kQSelList / kQuestSelThreads;
+            int32_t my_page[kPer];
+            uint32_t my_rank[kPer];
+#pragma unroll
+            for (int r = 0; r < kPer; ++r) {
+                const uint32_t e = tid + r * blockDim.x;
+                my_page[r] = -1;
+                my_rank[r] = 0u;
+                if (e < nl) {
+                    const int32_t pe = list[e];
+                    uint32_t rank = 0u;
+                    for (uint32_t f = 0; f < nl; ++f)
+                        rank += list[f] < pe ? 1u : 0u;
+                    my_page[r] = pe;
+                    my_rank[r] = rank;
+                    spos[rank] = (uint32_t)(page_hi(jlo + pe) - page_lo(jlo + pe));
+                }
+            }
+            __syncthreads();
+            // exclusive positions over the ranks, two entries per thread
+            const uint32_t a0 = 2 * tid < nl ? spos[2 * tid] : 0u;
+            const uint32_t a1 = 2 * tid + 1 < nl ? spos[2 * tid + 1] : 0u;
+            const uint32_t before = cta_exclusive_scan(a0 + a1, warp_sums, &total_tok);
+            if (2 * tid < nl)
+                spos[2 * tid] = before;
+            if (2 * tid + 1 < nl)
+                spos[2 * tid + 1] = before + a0;
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < kPer; ++r)
+                if (my_page[r] >= 0) {
+                    const int64_t j = jlo + my_page[r];
+                    uint32_t pos = (uint32_t)s_end + spos[my_rank[r]];
+                    for (int64_t i = page_lo(j); i < page_hi(j); ++i)
+                        row[pos++] = (int32_t)i;
+                }
+        } else {
+            // general path
+            uint32_t prefix = 0u, pmask = 0u, above = 0u;
+            for (int pass = 0; pass < 3; ++pass) {
+                const int psh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+                const uint32_t pdm = pass == 2 ? 1023u : 2047u;
+                for (int i = tid; i < kQuestSelBins; i += blockDim.x)
+                    hist[i] = 0u;
+                __syncthreads();
+                for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) {
+                    if ((key & pmask) == prefix)
+                        atomicAdd(&hist[(key >> psh) & pdm], 1u);
+                });
+                __syncthreads();
+                const int top = (int)pdm;
+                const int d1 = top - 2 * tid, d2 = d1 - 1;
+                const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
+                uint32_t tot;
+                const uint32_t before = above + cta_exclusive_scan(h1 + h2, warp_sums, &tot);
+                if (d1 >= 0 && before < (uint32_t)take && before + h1 >= (uint32_t)take) {
+                    s_digit = (uint32_t)d1;
+                    s_above = before;
+                } else if (d2 >= 0 && before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
+                    s_digit = (uint32_t)d2;
+                    s_above = before + h1;
+                }
+                __syncthreads();
+                prefix |= s_digit << psh;
+                pmask |= pdm << psh;
+                above = s_above;
+                __syncthreads();
+            }
+            const uint32_t T = prefix, need = (uint32_t)take - above;
+            const int64_t R = (nc + blockDim.x - 1) / blockDim.x;
+            const int64_t c0 = (int64_t)tid * R, c1 = c0 + R < nc ? c0 + R : nc;
+            uint32_t eq = 0u;
+            for (int64_t c = c0; c < c1; ++c)
+                eq += score_key(sc[jlo + c]) == T ? 1u : 0u;
+            uint32_t unused;
+            const uint32_t eq_rank = cta_exclusive_scan(eq, warp_sums, &unused);
+            uint32_t ntok = 0u;
+            {
+                uint32_t rank = eq_rank;
+                for (int64_t c = c0; c < c1; ++c) {
+                    const uint32_t key = score_key(sc[jlo + c]);
+                    if (key > T || (key == T && rank++ < need))
+                        ntok += (uint32_t)(page_hi(jlo + c) - page_lo(jlo + c));
+                }
+            }
+            uint32_t pos = (uint32_t)s_end + cta_exclusive_scan(ntok, warp_sums, &total_tok);
+            {
+                uint32_t rank = eq_rank;
+                for (int64_t c = c0; c < c1; ++c) {
+                    const uint32_t key = score_key(sc[jlo + c]);
+                    if (key > T || (key == T && rank++ < need))
+                        for (int64_t i = page_lo(jlo + c); i < page_hi(jlo + c); ++i)
+                            row[pos++] = (int32_t)i;
+                }
+            }
+        }
     }
     // the windows, the count and the padding
     const int64_t m = s_end + total_tok + (n - l0);
@@ -439,8 +617,9 @@ int chunks_per_lane(const Plan &p)
 int64_t quest_rows(const Plan &p, int page_size)
 {
     // sum over b of ceil(n_b / P) <= floor(n_total / P) + B (n_total: the
-    // capacity of a growing cache)
-    return p.n_total / page_size + p.B;
+    // capacity of a growing cache), rounded up to a multiple of 4 so that the
+    // selection may read the scores as aligned groups of four
+    return (p.n_total / page_size + p.B + 3) / 4 * 4;
 }
 
 cudaError_t launch_quest_meta(const Plan &p, const ts_kv_t *kv, int page_size, void *kmin, void *kmax,
@@ -474,8 +653,14 @@ cudaError_t launch_quest_score(const Plan &p, const ts_kv_t *kv, const void *q, 
     const int64_t max_pages = (p.n_max + page_size - 1) / page_size;
     if (max_pages == 0)
         return cudaSuccess;
+    // persistent warps: two resident CTAs per SM over the batch (about 110
+    // registers a thread), each warp walking its pages with a stride (its
+    // query weights built once)
     const int64_t per_cta = (int64_t)kQuestWarps * u;
-    const dim3 grid((unsigned)((max_pages + per_cta - 1) / per_cta), (unsigned)p.B);
+    int64_t gx = (max_pages + per_cta - 1) / per_cta;
+    const int64_t cap_x = (2 * (int64_t)p.sms + p.B - 1) / p.B;
+    gx = gx < cap_x ? gx : (cap_x > 0 ? cap_x : 1);
+    const dim3 grid((unsigned)gx, (unsigned)p.B);
     const __nv_bfloat16 *qq = static_cast<const __nv_bfloat16 *>(q);
     const __nv_bfloat16 *lo = static_cast<const __nv_bfloat16 *>(kmin), *hi = static_cast<const __nv_bfloat16 *>(kmax);
     const int ps = log2_exact(page_size);

@@ -114,6 +114,10 @@ CASES = {
     "integer_keys_many_ties": ([2000], 28, 4, 128, 200, 4, 64, 8, {"dist": "int"}),
     "padded_strides": ([3000], 28, 4, 128, 256, 4, 64, 16, {"strides": (4 * 128 * 2 + 64, 256)}),
     "sink_and_local_cut_pages": ([1003], 8, 2, 128, 64, 5, 21, 16, {}),
+    # the selection's general path: a threshold bucket of more than 2048
+    # tied pages, and more than 2048 pages to choose
+    "general_path_all_tied": ([5000], 4, 2, 64, 100, 4, 16, 1, {"dist": "const"}),
+    "general_path_large_budget": ([8000, 300], 4, 2, 64, 3000, 4, 64, 1, {}),
     "batch_40": ([int(x) for x in np.random.default_rng(40).integers(1, 700, 40)], 28, 4, 128, 64, 4, 32, 16, {}),
 }
 
