@@ -67,6 +67,9 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="run only the first N layers of the workload (a smaller case of the same kernels, "
                          "for profiler captures); the JSON line's config records it")
+    ap.add_argument("--comparator-page", type=int, default=16,
+                    help="page size of the page-level comparator (Quest's min/max page bounds) measured beside "
+                         "the token-level path (0: not measured)")
     ap.add_argument("--eager-steps", type=int, default=None,
                     help="profiler capture mode: after set-up, run this many decode steps of the workload as "
                          "plain (not graph-replayed) C-ABI calls, along the workload's query sequence, and exit "
@@ -414,6 +417,86 @@ def cpu_baseline_all_cores(wl, budget_s: float, threads=None):
 # arms
 # ---------------------------------------------------------------------------
 
+def selection_recall(ids: np.ndarray, count: int, want) -> float:
+    """Fraction of the token ids `want` that the selected row ids[:count] holds
+    (1.0 when `want` is empty)."""
+    want = set(int(x) for x in want)
+    if not want:
+        return 1.0
+    return len(want & set(ids[:count].tolist())) / len(want)
+
+
+def measure_comparator(wl, P: int, one, peak: float, peak_kind: str) -> dict:
+    """The page-level comparator (Quest's min/max page bounds, pages of P
+    tokens) on the same layers, queries and selection budget as the
+    token-level path: per-layer times of its kernels alone (the metadata pass,
+    which a serving loop runs once per page, apart), the score kernel's
+    bandwidth, and on layer 0 how many planted query-aligned keys each method
+    selects and how much of the token-level selection the page selection
+    covers."""
+    ts, cfg = wl.ts, wl.cfg
+    qb = [[ts.QuestBuffers(kv, P) for kv in copies] for copies in wl.kvs]
+    ids = [torch.full_like(b.ids, -1) for b in wl.bufs]
+    count = [torch.zeros_like(b.count) for b in wl.bufs]
+    out = [torch.zeros_like(b.out) for b in wl.bufs]
+
+    def kv_of(l, i):
+        return wl.kvs[l][i % wl.rotate], qb[l][i % wl.rotate]
+
+    for l in range(cfg.layers):
+        for r in range(wl.rotate):
+            ts.ts_quest_metadata(wl.kvs[l][r], P, qb[l][r].kmin, qb[l][r].kmax)
+
+    def score(l, i):
+        kv, b = kv_of(l, i)
+        ts.ts_quest_score(kv, wl.q[l][i % wl.T], P, b.kmin, b.kmax, b.scores)
+
+    def select(l, i):
+        kv, b = kv_of(l, i)
+        ts.ts_quest_select(kv, b.scores, P, cfg.k, cfg.n_sink, cfg.n_local, ids[l], count[l])
+
+    def attn(l, i):
+        ts.ts_sparse_attn(wl.kvs[l][i % wl.rotate], wl.q[l][i % wl.T], ids[l], count[l], out[l], wl.bufs[l].ws)
+
+    res = {"method": "page-level min/max key bounds (Quest), head-summed, top floor(k/P) pages + the windows",
+           "page_size": P}
+    res["metadata_us"] = 1e6 * one(lambda i: [ts.ts_quest_metadata(kv_of(l, i)[0], P, kv_of(l, i)[1].kmin,
+                                                                    kv_of(l, i)[1].kmax)
+                                              for l in range(cfg.layers)])
+    res["score_us"] = 1e6 * one(lambda i: [score(l, i) for l in range(cfg.layers)])
+    res["select_us"] = 1e6 * one(lambda i: [select(l, i) for l in range(cfg.layers)])
+    res["sparse_attn_us"] = 1e6 * one(lambda i: [attn(l, i) for l in range(cfg.layers)])
+    res["step_us"] = 1e6 * one(lambda i: [(score(l, i), select(l, i), attn(l, i)) for l in range(cfg.layers)])
+    pages = int(sum(-(-int(n) // P) for n in wl.lengths))
+    score_bytes = 2 * pages * cfg.h_kv * cfg.head_dim * 2
+    res["score_roofline"] = {"bound": "hbm", "alg_bytes_per_launch": score_bytes,
+                             "achieved": score_bytes / (res["score_us"] * 1e-6) / 1e9, "peak": peak,
+                             "peak_kind": peak_kind, "unit": "GB/s"}
+    res["score_roofline"]["frac"] = res["score_roofline"]["achieved"] / peak
+    # recall on layer 0, first query, every sequence: both methods select afresh
+    b0 = wl.bufs[0]
+    kv0, q0 = wl.kvs[0][0], wl.q[0][0]
+    ts.ts_score(kv0, q0, None, b0.votes, b0.ws)
+    ts.ts_select(kv0, b0.votes, cfg.k, cfg.n_sink, cfg.n_local, None, b0.ids, b0.count, b0.ws)
+    score(0, 0)
+    select(0, 0)
+    torch.cuda.synchronize()
+    t_ids, t_cnt = b0.ids.cpu().numpy(), b0.count.cpu().numpy()
+    p_ids, p_cnt = ids[0].cpu().numpy(), count[0].cpu().numpy()
+    planted = wl.layers[0].planted
+    rec_p, rec_t, cover = [], [], []
+    for bb in range(cfg.batch):
+        if planted is not None and len(planted[bb]):
+            rec_p.append(selection_recall(p_ids[bb], int(p_cnt[bb]), planted[bb]))
+            rec_t.append(selection_recall(t_ids[bb], int(t_cnt[bb]), planted[bb]))
+        cover.append(selection_recall(p_ids[bb], int(p_cnt[bb]), t_ids[bb][:int(t_cnt[bb])]))
+    res["planted_recall"] = float(np.mean(rec_p)) if rec_p else None
+    res["tokenselect_planted_recall"] = float(np.mean(rec_t)) if rec_t else None
+    res["covers_tokenselect_selection"] = float(np.mean(cover))
+    del qb
+    return res
+
+
 def run_ours(a, d: Dist):
     torch.cuda.set_device(d.local)
     dev = torch.device("cuda", d.local)
@@ -501,6 +584,10 @@ def run_ours(a, d: Dist):
                        for l in range(cfg.layers)])
     finally:
         del os.environ["TS_ATTN_CUDA_CORES"]
+
+    comparator = None
+    if a.comparator_page:
+        comparator = measure_comparator(wl, a.comparator_page, one, peak, peak_kind)
 
     # ---- end to end: pinned host query in, result out, every step ----
     q_host = [q.cpu().pin_memory() for q in wl.q]
@@ -601,6 +688,9 @@ def run_ours(a, d: Dist):
     }
     if reuse_rate is not None:
         result["reuse_rate"] = reuse_rate
+    if comparator is not None:
+        comparator["tokenselect_layer_step_us"] = ms_per_step * 1000.0 / cfg.layers
+        result["comparator"] = comparator
     if d.world == 1 and not a.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, 4.0)

@@ -150,3 +150,14 @@ def test_all_core_oracle_baseline_runs_threads_in_parallel():
     assert "2 threads" in two["sample"]
     if bench.usable_cores() >= 2:
         assert two["value"] > 1.3 * one["value"], (one, two)
+
+
+def test_selection_recall():
+    import numpy as np
+    row = np.array([0, 1, 5, 9, 12, -1, -1], np.int32)
+    assert bench.selection_recall(row, 5, [1, 9]) == 1.0
+    assert bench.selection_recall(row, 5, [1, 2, 9, 40]) == 0.5
+    assert bench.selection_recall(row, 3, [9]) == 0.0          # past the count
+    assert bench.selection_recall(row, 5, []) == 1.0
+    assert bench.parse_args([]).comparator_page == 16
+    assert bench.parse_args(["--comparator-page", "0"]).comparator_page == 0
