@@ -696,7 +696,7 @@ static ts_status_t decode_step_graph(const Plan &p, const CUtensorMap &kmap, con
     cudaError_t e = cudaGraphConditionalHandleCreate(&handle, graph, 1u, cudaGraphCondAssignDefault);
     if (e != cudaSuccess)
         return cuda_fail(e, "ts_decode_step: conditional handle");
-    SelcacheSkip skip;
+    SelcacheSkip skip = {};
     skip.handle = handle;
     skip.counters = reinterpret_cast<uint32_t *>(w + p.off_ctrl) + kCtrlSkipCounters;
     skip.enabled = 1;

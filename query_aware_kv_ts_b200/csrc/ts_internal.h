@@ -165,9 +165,9 @@ cudaError_t launch_append(int64_t *seq_offsets, void *k_cache, void *v_cache, co
 // counters: two words of the workspace control block (zero between steps).
 constexpr int kCtrlSkipCounters = 8;   // control-block words 8, 9
 struct SelcacheSkip {
-    cudaGraphConditionalHandle handle;
-    uint32_t *counters;
-    int enabled;
+    cudaGraphConditionalHandle handle = 0;
+    uint32_t *counters = nullptr;
+    int enabled = 0;
 };
 cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double *cos_out, int first_step,
                             int B, int len, double theta, cudaStream_t st, const SelcacheSkip *skip = nullptr);
