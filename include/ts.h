@@ -341,6 +341,83 @@ TS_API ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t s
 
 /*
  * ---------------------------------------------------------------------------
+ * Token-axis split of one sequence across ranks.  Each rank holds a
+ * contiguous shard [t, t + n_loc) of one sequence's tokens as a batch-1
+ * cache of its own (kv, without capacity) and runs the step's phases on it;
+ * three small exchanges, which the caller performs (e.g. NCCL all-gathers
+ * over NVLink), join them into exactly the single-sequence step:
+ *   1. ts_score_normalisers -> all-gather L -> ts_merge_normalisers ->
+ *      ts_score_vote_normalised: the votes of the shard's tokens under the
+ *      whole sequence's per-head softmax (TokenSelect README, "Key
+ *      Takeaways": the per-head softmax is over every cached token);
+ *   2. ts_select_candidates -> all-gather keys -> ts_select_merge: the whole
+ *      sequence's top-k (ties to the lower token id) with its sink and local
+ *      windows, as this shard's rows;
+ *   3. ts_sparse_attn_lse -> all-gather out and lse -> ts_merge_attention:
+ *      the attention over every selected token.
+ * Token ids in the shard's rows are shard-local (id + t is the sequence
+ * id); the keys carry sequence ids.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Score pass A and the normaliser merge on the shard (ts_score_logits), then
+ * L_out[b][h] = log sum_i exp(s[h][i]) over the shard's tokens (float64,
+ * device [batch][h_q]; -inf for an empty sequence). */
+TS_API ts_status_t ts_score_normalisers(const ts_kv_t *kv, const void *q, const int32_t *reuse, double *L_out,
+                                        void *ws, size_t ws_bytes, void *stream);
+
+/* Score pass B with given normalisers: votes[i] = sum_h exp(s[h][i] - L_in[b][h])
+ * for the logits of the last ts_score_normalisers / ts_score_logits call on
+ * this workspace (L_in: device float64 [batch][h_q]). */
+TS_API ts_status_t ts_score_vote_normalised(const ts_kv_t *kv, const int32_t *reuse, const double *L_in,
+                                            float *votes, void *ws, size_t ws_bytes, void *stream);
+
+/* L_out[i] = log sum_r exp(L_parts[r][i]) for i < count, r < parts (float64,
+ * device; -inf parts contribute nothing). */
+TS_API ts_status_t ts_merge_normalisers(const double *L_parts, int32_t parts, int64_t count, double *L_out,
+                                        void *stream);
+
+/*
+ * The shard's best min(k, its candidates) candidates of the sequence's top-k
+ * (candidates [s', l0) of the whole sequence as in ts_select, n_global its
+ * length, shard_offset = t) as keys: keys_out[j] = (vote bits << 32) |
+ * (2^32 - 1 - sequence id), ascending by id, 0 after them (device uint64
+ * [k]).  ids and count (device, k + n_sink + n_local entries) are scratch
+ * here: they hold the shard's own selection.  A larger key is a larger vote,
+ * or the lower id of two equal votes.
+ */
+TS_API ts_status_t ts_select_candidates(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink,
+                                        int32_t n_local, int64_t shard_offset, int64_t n_global, int32_t *ids,
+                                        int32_t *count, uint64_t *keys_out, void *ws, size_t ws_bytes,
+                                        void *stream);
+
+/*
+ * The sequence's selection, this shard's part: T = the k-th largest key of
+ * keys_all (device uint64 [parts][k], every shard's ts_select_candidates
+ * output, this one's at `rank`), or every key when there are at most k;
+ *   ids = [0, s_loc) U (this shard's keys >= T, as shard-local ids) U
+ *         [n_loc - l_loc, n_loc), ascending, -1 after count,
+ * s_loc and l_loc the shard's parts of the sequence's sink and local
+ * windows.  ids: device int32 [k + n_sink + n_local]; count: int32 [1].
+ */
+TS_API ts_status_t ts_select_merge(const ts_kv_t *kv, const uint64_t *keys_all, int32_t parts, int32_t rank,
+                                   int32_t k, int32_t n_sink, int32_t n_local, int64_t shard_offset,
+                                   int64_t n_global, int32_t *ids, int32_t *count, void *stream);
+
+/* ts_sparse_attn, also writing lse_out[b][h] = log sum_j exp(scale * q_h . K[ids[j]])
+ * over the selected tokens (device float32 [batch][h_q]; -inf when none). */
+TS_API ts_status_t ts_sparse_attn_lse(const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
+                                      int32_t ids_capacity, float *out, float *lse_out, void *ws,
+                                      size_t ws_bytes, void *stream);
+
+/* out[i][c] = sum_r w_r out_parts[r][i][c], w_r = exp(lse_parts[r][i] - LSE_i),
+ * LSE_i = log sum_r exp(lse_parts[r][i]) (rows i < rows, c < head_dim; 0
+ * where every part is -inf).  Device float32 throughout. */
+TS_API ts_status_t ts_merge_attention(const float *out_parts, const float *lse_parts, int32_t parts, int64_t rows,
+                                      int32_t head_dim, float *out, void *stream);
+
+/*
+ * ---------------------------------------------------------------------------
  * Page-level comparator after Quest (Bohrium page for "Quest: Query-Aware
  * Sparsity for Efficient Long-Context LLM Inference", arXiv 2406.10774:
  * Abstract; Method Overview, item 4).  Each page of P consecutive tokens of a

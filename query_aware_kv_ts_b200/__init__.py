@@ -76,6 +76,15 @@ _SIGS = {
     "ts_append_kv": (ctypes.c_int, [_KV, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "ts_get_device_status": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(_U32), _P]),
     "ts_selftest_expire_wait": (ctypes.c_int, [_P, _SZ, _U32, _P]),
+    "ts_score_normalisers": (ctypes.c_int, [_KV, _P, _P, _P, _P, _SZ, _P]),
+    "ts_score_vote_normalised": (ctypes.c_int, [_KV, _P, _P, _P, _P, _SZ, _P]),
+    "ts_merge_normalisers": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _P, _P]),
+    "ts_select_candidates": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64, _P, _P, _P,
+                                            _P, _SZ, _P]),
+    "ts_select_merge": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64, _P,
+                                       _P, _P]),
+    "ts_sparse_attn_lse": (ctypes.c_int, [_KV, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "ts_merge_attention": (ctypes.c_int, [_P, _P, _I32, ctypes.c_int64, _I32, _P, _P]),
     "ts_quest_rows": (ctypes.c_int64, [_KV, _I32]),
     "ts_quest_metadata": (ctypes.c_int, [_KV, _I32, _P, _P, _P]),
     "ts_quest_score": (ctypes.c_int, [_KV, _P, _I32, _P, _P, _P, _P]),
@@ -264,6 +273,46 @@ def ts_get_device_status(ws, stream=None):
 def ts_selftest_expire_wait(ws, spin_limit: int, stream=None):
     _check(_lib.ts_selftest_expire_wait(_ptr(ws), ws.numel() * ws.element_size(), spin_limit,
                                         _stream(stream)))
+
+
+# ---- token-axis split of one sequence (the joins; see split.py) ----
+
+def ts_score_normalisers(kv: KVCache, q, reuse, L_out, ws, stream=None):
+    _check(_lib.ts_score_normalisers(kv.ref(), _ptr(q), _ptr(reuse), _ptr(L_out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ts_score_vote_normalised(kv: KVCache, reuse, L_in, votes, ws, stream=None):
+    _check(_lib.ts_score_vote_normalised(kv.ref(), _ptr(reuse), _ptr(L_in), _ptr(votes), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ts_merge_normalisers(L_parts, parts: int, L_out, stream=None):
+    _check(_lib.ts_merge_normalisers(_ptr(L_parts), int(parts), L_out.numel(), _ptr(L_out), _stream(stream)))
+
+
+def ts_select_candidates(kv: KVCache, votes, k: int, n_sink: int, n_local: int, shard_offset: int, n_global: int,
+                         ids, count, keys_out, ws, stream=None):
+    _check(_lib.ts_select_candidates(kv.ref(), _ptr(votes), k, n_sink, n_local, int(shard_offset), int(n_global),
+                                     _ptr(ids), _ptr(count), _ptr(keys_out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ts_select_merge(kv: KVCache, keys_all, parts: int, rank: int, k: int, n_sink: int, n_local: int,
+                    shard_offset: int, n_global: int, ids, count, stream=None):
+    _check(_lib.ts_select_merge(kv.ref(), _ptr(keys_all), int(parts), int(rank), k, n_sink, n_local,
+                                int(shard_offset), int(n_global), _ptr(ids), _ptr(count), _stream(stream)))
+
+
+def ts_sparse_attn_lse(kv: KVCache, q, ids, count, out, lse_out, ws, stream=None):
+    _check(_lib.ts_sparse_attn_lse(kv.ref(), _ptr(q), _ptr(ids), _ptr(count), ids.shape[-1], _ptr(out),
+                                   _ptr(lse_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ts_merge_attention(out_parts, lse_parts, parts: int, out, stream=None):
+    rows, d = lse_parts.shape[-1], out.shape[-1]
+    _check(_lib.ts_merge_attention(_ptr(out_parts), _ptr(lse_parts), int(parts), rows, d, _ptr(out),
+                                   _stream(stream)))
 
 
 def ts_quest_rows(kv: KVCache, page_size: int) -> int:

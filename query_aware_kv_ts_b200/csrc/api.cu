@@ -907,6 +907,180 @@ ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t spin_lim
 }
 
 // ---------------------------------------------------------------------------
+// Token-axis split of one sequence across ranks
+// ---------------------------------------------------------------------------
+
+ts_status_t ts_score_normalisers(const ts_kv_t *kv, const void *q, const int32_t *reuse, double *L_out, void *ws,
+                                 size_t ws_bytes, void *stream)
+{
+    if (L_out == nullptr) {
+        set_error("L_out is required");
+        return TS_ERR_INVALID_ARG;
+    }
+    ts_status_t s = ts_score_logits(kv, q, reuse, ws, ws_bytes, stream);
+    if (s != TS_OK)
+        return s;
+    Plan p;
+    s = make_plan(kv, -1, &p);
+    if (s != TS_OK)
+        return s;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (p.n_total == 0)   // nothing scored: every L is -inf (a merge of no parts)
+        e = launch_merge_normalisers(nullptr, 0, (int64_t)p.B * p.Hq, L_out, st);
+    else
+        e = cudaMemcpyAsync(L_out, static_cast<uint8_t *>(ws) + p.off_L, sizeof(double) * p.B * p.Hq,
+                            cudaMemcpyDeviceToDevice, st);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "normalisers copy");
+}
+
+ts_status_t ts_score_vote_normalised(const ts_kv_t *kv, const int32_t *reuse, const double *L_in, float *votes,
+                                     void *ws, size_t ws_bytes, void *stream)
+{
+    Plan p;
+    ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
+    if (s != TS_OK)
+        return s;
+    if (votes == nullptr || L_in == nullptr) {
+        set_error("votes and L_in are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if (p.n_total == 0)
+        return TS_OK;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(static_cast<uint8_t *>(ws) + p.off_L, L_in, sizeof(double) * p.B * p.Hq,
+                                    cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+        e = launch_vote(p, kv->seq_offsets_dev, reuse, votes, static_cast<uint8_t *>(ws), st);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass B launch");
+}
+
+ts_status_t ts_merge_normalisers(const double *L_parts, int32_t parts, int64_t count, double *L_out, void *stream)
+{
+    if (L_parts == nullptr || L_out == nullptr || parts < 1 || count < 0) {
+        set_error("L_parts and L_out are required, parts >= 1, count >= 0");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_merge_normalisers(L_parts, parts, count, L_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "normaliser merge launch");
+}
+
+// The shard's share of the sequence's windows: sink [0, s') and local window
+// [l0, n) of the whole sequence, intersected with [t, t + n_loc), as counts
+// of the shard's first and last tokens.
+static ts_status_t shard_windows(const ts_kv_t *kv, int32_t n_sink, int32_t n_local, int64_t t, int64_t n_global,
+                                 int64_t *n_loc, int *s_loc, int *l_loc)
+{
+    if (kv == nullptr || kv->batch != 1 || kv->seq_offsets_host == nullptr || kv->capacity != 0) {
+        set_error("a shard is one sequence (batch 1, no capacity)");
+        return TS_ERR_INVALID_ARG;
+    }
+    *n_loc = kv->seq_offsets_host[1] - kv->seq_offsets_host[0];
+    if (t < 0 || *n_loc < 0 || t + *n_loc > n_global || n_global >= (int64_t(1) << 31)) {
+        set_error("shard [%lld, %lld) must lie in the sequence [0, %lld), below 2^31 tokens", (long long)t,
+                  (long long)(t + *n_loc), (long long)n_global);
+        return TS_ERR_INVALID_ARG;
+    }
+    const int64_t s = n_sink < n_global ? n_sink : n_global;
+    const int64_t l0 = n_global - n_local > s ? n_global - n_local : s;
+    int64_t a = (s < t + *n_loc ? s : t + *n_loc) - t;
+    int64_t c = t + *n_loc - (l0 > t ? l0 : t);
+    *s_loc = (int)(a < 0 ? 0 : a);
+    *l_loc = (int)(c < 0 ? 0 : c);
+    return TS_OK;
+}
+
+ts_status_t ts_select_candidates(const ts_kv_t *kv, const float *votes, int32_t k, int32_t n_sink, int32_t n_local,
+                                 int64_t shard_offset, int64_t n_global, int32_t *ids, int32_t *count,
+                                 uint64_t *keys_out, void *ws, size_t ws_bytes, void *stream)
+{
+    if (k < 1 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > kMaxCapacity) {
+        set_error("k >= 1, n_sink, n_local >= 0, k + n_sink + n_local <= %d", kMaxCapacity);
+        return TS_ERR_INVALID_ARG;
+    }
+    int64_t n_loc;
+    int s_loc, l_loc;
+    ts_status_t s = shard_windows(kv, n_sink, n_local, shard_offset, n_global, &n_loc, &s_loc, &l_loc);
+    if (s != TS_OK)
+        return s;
+    if (votes == nullptr || ids == nullptr || count == nullptr || keys_out == nullptr) {
+        set_error("votes, ids, count and keys_out are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    s = ts_select(kv, votes, k, s_loc, l_loc, nullptr, ids, count, ws, ws_bytes, stream);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_candidate_keys(votes, ids, count, s_loc, l_loc, shard_offset, k,
+                                          reinterpret_cast<unsigned long long *>(keys_out),
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "candidate keys launch");
+}
+
+ts_status_t ts_select_merge(const ts_kv_t *kv, const uint64_t *keys_all, int32_t parts, int32_t rank, int32_t k,
+                            int32_t n_sink, int32_t n_local, int64_t shard_offset, int64_t n_global, int32_t *ids,
+                            int32_t *count, void *stream)
+{
+    if (k < 1 || n_sink < 0 || n_local < 0 || (int64_t)k + n_sink + n_local > kMaxCapacity || parts < 1 ||
+        rank < 0 || rank >= parts || (int64_t)parts * k > (int64_t(1) << 30)) {
+        set_error("k >= 1, 0 <= rank < parts, k + n_sink + n_local <= %d", kMaxCapacity);
+        return TS_ERR_INVALID_ARG;
+    }
+    int64_t n_loc;
+    int s_loc, l_loc;
+    ts_status_t s = shard_windows(kv, n_sink, n_local, shard_offset, n_global, &n_loc, &s_loc, &l_loc);
+    if (s != TS_OK)
+        return s;
+    if (keys_all == nullptr || ids == nullptr || count == nullptr) {
+        set_error("keys_all, ids and count are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_select_merge(reinterpret_cast<const unsigned long long *>(keys_all), parts, k, k, rank,
+                                        s_loc, l_loc, n_loc, shard_offset, k + n_sink + n_local, ids, count,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "selection merge launch");
+}
+
+ts_status_t ts_sparse_attn_lse(const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
+                               int32_t ids_capacity, float *out, float *lse_out, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    if (ids_capacity < 1) {
+        set_error("ids_capacity must be >= 1");
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = make_plan(kv, ids_capacity, &p);
+    if (s != TS_OK)
+        return s;
+    if (q == nullptr || ids == nullptr || count == nullptr || out == nullptr || lse_out == nullptr) {
+        set_error("q, ids, count, out and lse_out are required");
+        return TS_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u) {
+        set_error("q and out must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    s = check_ws(p, ws, ws_bytes);
+    if (s != TS_OK)
+        return s;
+    cudaError_t e = launch_attn(p, kv, q, ids, count, out, static_cast<uint8_t *>(ws),
+                                static_cast<cudaStream_t>(stream), lse_out);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "sparse attention launch");
+}
+
+ts_status_t ts_merge_attention(const float *out_parts, const float *lse_parts, int32_t parts, int64_t rows,
+                               int32_t head_dim, float *out, void *stream)
+{
+    if (out_parts == nullptr || lse_parts == nullptr || out == nullptr || parts < 1 || rows < 0 || head_dim < 1) {
+        set_error("out_parts, lse_parts and out are required, parts >= 1, rows >= 0, head_dim >= 1");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e = launch_merge_attention(out_parts, lse_parts, parts, rows, head_dim, out,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "attention merge launch");
+}
+
+// ---------------------------------------------------------------------------
 // Page-level comparator
 // ---------------------------------------------------------------------------
 

@@ -31,6 +31,7 @@ namespace ts {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2f = 0.693147180559945309f;   // ln 2
 constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int R = kAttnRows;
 
@@ -46,6 +47,7 @@ struct AttnArgs {
     float *part;        // [B][Hkv][splits][G][D + 4]: D weighted-V sums, then (max, sum)
     int B, Hq, Hkv, G, splits;
     float scale_log2;   // scale * log2(e): logits in base-2 units
+    float *lse;         // or null: [B][Hq] natural log-sum-exp of each head's scaled logits
     // paged cache (page_table != null): token i of sequence b is pool row
     // page_table[b * pt_stride + (i >> page_shift)] << page_shift | (i & (page - 1))
     const int32_t *page_table;
@@ -460,6 +462,8 @@ attn_merge(const AttnArgs a)
     const float inv = Lt > 0.0f ? 1.0f / Lt : 0.0f;
     *reinterpret_cast<float4 *>(a.out + ((int64_t)b * a.Hq + h) * D + 4 * c) =
         make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    if (a.lse != nullptr && c == 0)   // (max and sum are the same in every channel quad)
+        a.lse[(int64_t)b * a.Hq + h] = Lt > 0.0f ? (Mt + log2f(Lt)) * kLn2f : -INFINITY;
 }
 
 template <int D, int NB, bool TC>
@@ -501,6 +505,7 @@ AttnArgs make_args(const Plan &p, const ts_kv_t *kv, const void *q, const int32_
                    float *out)
 {
     AttnArgs a;
+    a.lse = nullptr;
     a.k = static_cast<const __nv_bfloat16 *>(kv->k);
     a.v = static_cast<const __nv_bfloat16 *>(kv->v);
     a.st = kv->stride_tok;
@@ -601,10 +606,11 @@ ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q,
 }
 
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids, const int32_t *count,
-                        float *out, uint8_t *ws, cudaStream_t st)
+                        float *out, uint8_t *ws, cudaStream_t st, float *lse)
 {
     AttnArgs a = make_args(p, kv, q, ids, count, out);
     a.part = reinterpret_cast<float *>(ws + p.off_attn_part);
+    a.lse = lse;
     return launch_attn_any(p, a, st);
 }
 

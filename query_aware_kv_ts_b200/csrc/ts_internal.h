@@ -200,8 +200,10 @@ cudaError_t launch_select(const Plan &p, const int64_t *seq_off, const float *vo
                           int n_local, const int32_t *reuse, int32_t *ids, int32_t *count, uint8_t *ws,
                           cudaStream_t st, bool hist_ready = false);
 
+// lse (or null): [B][Hq] natural log-sum-exp of each head's scaled logits
+// over the selected tokens (-inf when none), for joining shards.
 cudaError_t launch_attn(const Plan &p, const ts_kv_t *kv, const void *q, const int32_t *ids,
-                        const int32_t *count, float *out, uint8_t *ws, cudaStream_t st);
+                        const int32_t *count, float *out, uint8_t *ws, cudaStream_t st, float *lse = nullptr);
 
 // Attention with its scratch in a fixed device array instead of a workspace
 // (sets the error message itself).
@@ -209,6 +211,17 @@ ts_status_t launch_attn_noalloc(const Plan &p, const ts_kv_t *kv, const void *q,
                                 const int32_t *count, float *out, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(uint32_t *ctrl, uint32_t spin_limit, cudaStream_t st);
+
+// Token-axis split of one sequence (split.cu): the joins' arithmetic.
+cudaError_t launch_merge_normalisers(const double *L_parts, int parts, int64_t count, double *L_out,
+                                     cudaStream_t st);
+cudaError_t launch_candidate_keys(const float *votes, const int32_t *ids, const int32_t *count, int s_loc, int l_loc,
+                                  int64_t shard_offset, int kcap, unsigned long long *keys, cudaStream_t st);
+cudaError_t launch_select_merge(const unsigned long long *keys, int parts, int kcap, int k, int rank, int s_loc,
+                                int l_loc, int64_t n_loc, int64_t shard_offset, int cap, int32_t *ids,
+                                int32_t *count, cudaStream_t st);
+cudaError_t launch_merge_attention(const float *o_parts, const float *lse_parts, int parts, int64_t rows, int d,
+                                   float *out, cudaStream_t st);
 
 // Page-level comparator (quest.cu): rows of the page metadata and scores,
 // page j of sequence b at row (seq_offsets[b] >> log2 P) + b + j.
