@@ -19,6 +19,7 @@
 // reads the metadata once and folds the sum over heads into one dot product
 // per page (below); the selection is one CTA per sequence doing a radix
 // select over the pages' order keys.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "score_common.cuh"
@@ -296,23 +297,6 @@ __device__ __forceinline__ uint32_t score_key(float s)
     return (uint32_t)float_order_key(s == 0.0f ? 0.0f : s) ^ 0x80000000u;
 }
 
-// The page selection, one CTA of 1024 threads per sequence.  Candidate
-// pages [jlo, jlo + nc) are those holding a token of [s_end, l0); `take`
-// of them are chosen.
-//
-// Fast path (at most 2048 pages to choose, the usual case): the keys' min
-// and max span 2048 equal bins; one histogram over them finds the threshold
-// bin (equal bins in key space spread a concentrated score distribution
-// over many bins, so the histogram's shared atomics rarely collide); one
-// more pass puts the sure winners (a higher bin) and the threshold bin's
-// pages in shared memory, where the
-// rest is decided by counting ranks: the bucket's pages by (key desc, page
-// asc), the chosen pages by page for their token positions.  Three
-// coalesced passes over the scores.  When the threshold digit holds more
-// than 2048 pages (heavy ties), the general path takes over: a three-digit
-// radix select over all 32 key bits, then two passes in page order over a
-// contiguous range per thread (the ranks among pages tied at the threshold,
-// then the tokens).  Five passes; any number of candidates and ties.
 // Calls f(c, key) for this thread's candidates c = tid, tid + blockDim.x, ...
 // < nc, with kQSelBatch loads in flight.
 constexpr int kQSelBatch = 8;
@@ -335,22 +319,49 @@ __device__ __forceinline__ void for_each_key(const float *sc, int64_t nc, F f)
     }
 }
 
+// The page selection, one cluster of kQSelCluster CTAs of 1024 threads per
+// sequence.  Candidate pages [jlo, jlo + nc) are those holding a token of
+// [s_end, l0); `take` of them are chosen.
+//
+// Fast path (at most 2048 pages to choose, the usual case): each CTA of the
+// cluster takes an equal slice of the candidates.  Their keys' min and max
+// (combined through distributed shared memory) span 2048 equal bins (equal
+// bins in key space spread a concentrated score distribution over many
+// bins, so the histograms' shared atomics rarely collide); the slices'
+// histograms are summed by rank 0, which finds the threshold bin; each CTA
+// then appends its sure winners (a higher bin) and its threshold-bin pages
+// to rank 0's shared memory, where rank 0 decides the rest by counting ranks:
+// the bucket's pages by (key desc, page asc), the chosen pages by page for
+// their token positions.  Three coalesced passes over the scores, spread
+// over the cluster's SMs (one SM's issue rate bounded a single-CTA version).
+// General path (more than 2048 pages to choose, or more than 2048 tied in
+// the threshold bin): rank 0 alone runs a three-digit radix select over all
+// 32 key bits and two passes in page order over a contiguous range per
+// thread.  Every cross-CTA access lies between cluster barriers, and no CTA
+// leaves while another may still read its shared memory.
+constexpr int kQSelCluster = 8;
 constexpr int kQSelList = 2048;     // chosen pages the fast path holds
-constexpr int kQSelBucket = 2048;   // pages of the threshold digit it holds
+constexpr int kQSelBucket = 2048;   // pages of the threshold bin it holds
 
 __global__ void __launch_bounds__(kQuestSelThreads)
 quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, int n_sink, int n_local, int cap,
              int32_t *ids, int32_t *count)
 {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
     __shared__ uint32_t hist[kQuestSelBins];
     __shared__ uint32_t warp_sums[32];
     __shared__ uint32_t warp_lo[32], warp_hi[32];
-    __shared__ uint32_t s_kmin, s_kmax, s_digit, s_above, s_nlist, s_nbucket;
+    __shared__ uint32_t s_kmin, s_kmax, s_gmin, s_gmax, s_digit, s_above, s_nlist, s_nbucket;
+    __shared__ uint32_t s_dec_digit, s_dec_above, s_dec_over;   // rank 0's decision, read by every rank
     __shared__ int32_t list[kQSelList];
     __shared__ uint32_t bkey[kQSelBucket];
     __shared__ int32_t bidx[kQSelBucket];
     __shared__ uint32_t spos[kQSelList];
-    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();   // the scores come from the previous kernel (launched with programmatic serialization)
+    pdl_launch_dependents();
+    const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t off0 = seq_off[b];
     const int64_t n = seq_off[b + 1] - off0;
     const float *sc = scores + (off0 >> P_shift) + b;   // page j's score at sc[j]
@@ -365,29 +376,108 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
     auto page_lo = [&](int64_t j) { return (j << P_shift) > s_end ? (j << P_shift) : s_end; };
     auto page_hi = [&](int64_t j) { return ((j + 1) << P_shift) < l0 ? ((j + 1) << P_shift) : l0; };
 
+    // general path: rank 0 alone (every decision that leads here is the same
+    // in every rank, and the other ranks have left or no longer touch rank
+    // 0's radix state)
+    auto general = [&]() -> uint32_t {
+        uint32_t prefix = 0u, pmask = 0u, above = 0u;
+        for (int pass = 0; pass < 3; ++pass) {
+            const int psh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+            const uint32_t pdm = pass == 2 ? 1023u : 2047u;
+            for (int i = tid; i < kQuestSelBins; i += blockDim.x)
+                hist[i] = 0u;
+            __syncthreads();
+            for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) {
+                if ((key & pmask) == prefix)
+                    atomicAdd(&hist[(key >> psh) & pdm], 1u);
+            });
+            __syncthreads();
+            const int top = (int)pdm;
+            const int d1 = top - 2 * tid, d2 = d1 - 1;
+            const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
+            uint32_t tot;
+            const uint32_t before = above + cta_exclusive_scan(h1 + h2, warp_sums, &tot);
+            if (d1 >= 0 && before < (uint32_t)take && before + h1 >= (uint32_t)take) {
+                s_digit = (uint32_t)d1;
+                s_above = before;
+            } else if (d2 >= 0 && before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
+                s_digit = (uint32_t)d2;
+                s_above = before + h1;
+            }
+            __syncthreads();
+            prefix |= s_digit << psh;
+            pmask |= pdm << psh;
+            above = s_above;
+            __syncthreads();
+        }
+        const uint32_t T = prefix, need = (uint32_t)take - above;
+        const int64_t R = (nc + blockDim.x - 1) / blockDim.x;
+        const int64_t c0 = (int64_t)tid * R, c1 = c0 + R < nc ? c0 + R : nc;
+        uint32_t eq = 0u;
+        for (int64_t c = c0; c < c1; ++c)
+            eq += score_key(sc[jlo + c]) == T ? 1u : 0u;
+        uint32_t unused;
+        const uint32_t eq_rank = cta_exclusive_scan(eq, warp_sums, &unused);
+        uint32_t ntok = 0u;
+        {
+            uint32_t rk = eq_rank;
+            for (int64_t c = c0; c < c1; ++c) {
+                const uint32_t key = score_key(sc[jlo + c]);
+                if (key > T || (key == T && rk++ < need))
+                    ntok += (uint32_t)(page_hi(jlo + c) - page_lo(jlo + c));
+            }
+        }
+        uint32_t tt;
+        uint32_t pos = (uint32_t)s_end + cta_exclusive_scan(ntok, warp_sums, &tt);
+        {
+            uint32_t rk = eq_rank;
+            for (int64_t c = c0; c < c1; ++c) {
+                const uint32_t key = score_key(sc[jlo + c]);
+                if (key > T || (key == T && rk++ < need))
+                    for (int64_t i = page_lo(jlo + c); i < page_hi(jlo + c); ++i)
+                        row[pos++] = (int32_t)i;
+            }
+        }
+        return tt;
+    };
+
     uint32_t total_tok = 0u;
     if (take == nc) {
+        if (rank != 0)
+            return;
         // every candidate page (or none): every token of [s_end, l0)
         total_tok = nc > 0 ? (uint32_t)(l0 - s_end) : 0u;
         for (int64_t i = s_end + tid; i < s_end + total_tok; i += blockDim.x)
             row[i] = (int32_t)i;
+    } else if (take > 0 && take > kQSelList) {
+        if (rank != 0)
+            return;
+        total_tok = general();
     } else if (take > 0) {
-        bool fast = take <= kQSelList;
-        // digit of a key: its place among 2048 equal bins over [kmin, kmax]
-        // of the keys (a monotone map: a higher digit is a larger key)
-        uint32_t kbase = 0u;
-        float kscale = 0.0f;
-        auto digit_of = [&](uint32_t key) {
-            const uint32_t d = (uint32_t)((float)(key - kbase) * kscale);
-            return d < (uint32_t)(kQuestSelBins - 1) ? d : (uint32_t)(kQuestSelBins - 1);
-        };
-        if (fast) {
-            // pass 1: the smallest and largest key
-            uint32_t lo = 0xffffffffu, hi = 0u;
-            for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) {
-                lo = key < lo ? key : lo;
-                hi = key > hi ? key : hi;
-            });
+        // this rank's slice of the candidates
+        const int64_t c_lo = nc * rank / C, c_hi = nc * (rank + 1) / C;
+        // pass 1: the slice's smallest and largest key
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for_each_key(sc + jlo + c_lo, c_hi - c_lo, [&](int64_t, uint32_t key) {
+            lo = key < lo ? key : lo;
+            hi = key > hi ? key : hi;
+        });
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t a2 = __shfl_xor_sync(0xffffffffu, lo, o), b2 = __shfl_xor_sync(0xffffffffu, hi, o);
+            lo = a2 < lo ? a2 : lo;
+            hi = b2 > hi ? b2 : hi;
+        }
+        if (lane == 0) {
+            warp_lo[warp] = lo;
+            warp_hi[warp] = hi;
+        }
+        for (int i = tid; i < kQuestSelBins; i += blockDim.x)
+            hist[i] = 0u;
+        __syncthreads();
+        if (warp == 0) {
+            lo = warp_lo[lane];
+            hi = warp_hi[lane];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const uint32_t a2 = __shfl_xor_sync(0xffffffffu, lo, o), b2 = __shfl_xor_sync(0xffffffffu, hi, o);
@@ -395,78 +485,97 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
                 hi = b2 > hi ? b2 : hi;
             }
             if (lane == 0) {
-                warp_lo[warp] = lo;
-                warp_hi[warp] = hi;
+                s_kmin = lo;
+                s_kmax = hi;
             }
-            for (int i = tid; i < kQuestSelBins; i += blockDim.x)
-                hist[i] = 0u;
-            __syncthreads();
-            if (warp == 0) {
-                lo = warp_lo[lane];
-                hi = warp_hi[lane];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const uint32_t a2 = __shfl_xor_sync(0xffffffffu, lo, o), b2 = __shfl_xor_sync(0xffffffffu, hi, o);
-                    lo = a2 < lo ? a2 : lo;
-                    hi = b2 > hi ? b2 : hi;
-                }
-                if (lane == 0) {
-                    s_kmin = lo;
-                    s_kmax = hi;
-                }
-            }
-            __syncthreads();
-            kbase = s_kmin;
-            kscale = (float)kQuestSelBins / ((float)(s_kmax - s_kmin) + 1.0f);
-            // pass 2: the digit histogram
-            for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) { atomicAdd(&hist[digit_of(key)], 1u); });
-            __syncthreads();
-            // the threshold digit: digits in descending order, two per thread
-            {
-                const int d1 = kQuestSelBins - 1 - 2 * tid, d2 = d1 - 1;
-                const uint32_t h1 = hist[d1], h2 = hist[d2];
-                uint32_t tot;
-                const uint32_t before = cta_exclusive_scan(h1 + h2, warp_sums, &tot);
-                if (before < (uint32_t)take && before + h1 >= (uint32_t)take) {
-                    s_digit = (uint32_t)d1;
-                    s_above = before;
-                } else if (before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
-                    s_digit = (uint32_t)d2;
-                    s_above = before + h1;
-                }
-                if (tid == 0) {
-                    s_nlist = 0u;
-                    s_nbucket = 0u;
-                }
-            }
-            __syncthreads();
-            fast = hist[s_digit] <= (uint32_t)kQSelBucket;   // the same for every thread
-            __syncthreads();   // read by all before the general path rewrites hist
         }
-        if (fast) {
-            const uint32_t digit = s_digit, above = s_above;
-            // pass 3: the sure winners and the threshold digit's pages
-            for_each_key(sc + jlo, nc, [&](int64_t c, uint32_t key) {
+        cl.sync();   // 1: every slice's min and max
+        if (tid == 0) {
+            uint32_t gl = 0xffffffffu, gh = 0u;
+            for (int r = 0; r < C; ++r) {
+                const uint32_t rl = *cl.map_shared_rank(&s_kmin, r), rh = *cl.map_shared_rank(&s_kmax, r);
+                gl = rl < gl ? rl : gl;
+                gh = rh > gh ? rh : gh;
+            }
+            s_gmin = gl;
+            s_gmax = gh;
+        }
+        __syncthreads();
+        // digit of a key: its place among 2048 equal bins over [kmin, kmax]
+        // of all the keys (a monotone map: a higher digit is a larger key)
+        const uint32_t kbase = s_gmin;
+        const float kscale = (float)kQuestSelBins / ((float)(s_gmax - s_gmin) + 1.0f);
+        auto digit_of = [&](uint32_t key) {
+            const uint32_t d = (uint32_t)((float)(key - kbase) * kscale);
+            return d < (uint32_t)(kQuestSelBins - 1) ? d : (uint32_t)(kQuestSelBins - 1);
+        };
+        // pass 2: the slice's histogram
+        for_each_key(sc + jlo + c_lo, c_hi - c_lo, [&](int64_t, uint32_t key) { atomicAdd(&hist[digit_of(key)], 1u); });
+        cl.sync();   // 2: every slice's histogram
+        if (rank == 0) {
+            // the threshold bin of the summed histograms (digits in descending
+            // order, two per thread; each thread sums and keeps its own two)
+            const int d1 = kQuestSelBins - 1 - 2 * tid, d2 = d1 - 1;
+            uint32_t h1 = 0u, h2 = 0u;
+            for (int r = 0; r < C; ++r) {
+                const uint32_t *rh = cl.map_shared_rank(hist, r);
+                h1 += rh[d1];
+                h2 += rh[d2];
+            }
+            uint32_t tot;
+            const uint32_t before = cta_exclusive_scan(h1 + h2, warp_sums, &tot);
+            if (before < (uint32_t)take && before + h1 >= (uint32_t)take) {
+                s_dec_digit = (uint32_t)d1;
+                s_dec_above = before;
+                s_dec_over = h1 > (uint32_t)kQSelBucket ? 1u : 0u;
+            } else if (before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
+                s_dec_digit = (uint32_t)d2;
+                s_dec_above = before + h1;
+                s_dec_over = h2 > (uint32_t)kQSelBucket ? 1u : 0u;
+            }
+            if (tid == 0) {
+                s_nlist = 0u;
+                s_nbucket = 0u;
+            }
+        }
+        cl.sync();   // 3: rank 0's decision; nobody reads another rank's histogram any more
+        const uint32_t digit = *cl.map_shared_rank(&s_dec_digit, 0);
+        const uint32_t above = *cl.map_shared_rank(&s_dec_above, 0);
+        const uint32_t over = *cl.map_shared_rank(&s_dec_over, 0);
+        if (over != 0u) {
+            if (rank != 0)
+                return;
+            total_tok = general();
+        } else {
+            // pass 3: the slice's sure winners and threshold-bin pages, into rank 0
+            uint32_t *r_nlist = cl.map_shared_rank(&s_nlist, 0);
+            uint32_t *r_nbucket = cl.map_shared_rank(&s_nbucket, 0);
+            int32_t *r_list = cl.map_shared_rank(list, 0);
+            uint32_t *r_bkey = cl.map_shared_rank(bkey, 0);
+            int32_t *r_bidx = cl.map_shared_rank(bidx, 0);
+            for_each_key(sc + jlo + c_lo, c_hi - c_lo, [&](int64_t c, uint32_t key) {
                 const uint32_t d = digit_of(key);
                 if (d > digit) {
-                    list[atomicAdd(&s_nlist, 1u)] = (int32_t)c;
+                    r_list[atomicAdd(r_nlist, 1u)] = (int32_t)(c_lo + c);
                 } else if (d == digit) {
-                    const uint32_t slot = atomicAdd(&s_nbucket, 1u);
-                    bkey[slot] = key;
-                    bidx[slot] = (int32_t)c;
+                    const uint32_t slot = atomicAdd(r_nbucket, 1u);
+                    r_bkey[slot] = key;
+                    r_bidx[slot] = (int32_t)(c_lo + c);
                 }
             });
-            __syncthreads();
+            cl.sync();   // 4: every slice's pages are in rank 0
+            if (rank != 0)
+                return;
             // the bucket, ranked by (key desc, page asc): the first take - above join the list
             const uint32_t nb = s_nbucket, need = (uint32_t)take - above;
             for (uint32_t e = tid; e < nb; e += blockDim.x) {
                 const uint32_t ke = bkey[e];
                 const int32_t ie = bidx[e];
-                uint32_t rank = 0u;
+                uint32_t rk = 0u;
                 for (uint32_t f = 0; f < nb; ++f)
-                    rank += (bkey[f] > ke || (bkey[f] == ke && bidx[f] < ie)) ? 1u : 0u;
-                if (rank < need)
-                    list[above + rank] = ie;
+                    rk += (bkey[f] > ke || (bkey[f] == ke && bidx[f] < ie)) ? 1u : 0u;
+                if (rk < need)
+                    list[above + rk] = ie;
             }
             __syncthreads();
             // the chosen pages in page order: rank by counting, token counts by rank
@@ -481,12 +590,12 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
                 my_rank[r] = 0u;
                 if (e < nl) {
                     const int32_t pe = list[e];
-                    uint32_t rank = 0u;
+                    uint32_t rk = 0u;
                     for (uint32_t f = 0; f < nl; ++f)
-                        rank += list[f] < pe ? 1u : 0u;
+                        rk += list[f] < pe ? 1u : 0u;
                     my_page[r] = pe;
-                    my_rank[r] = rank;
-                    spos[rank] = (uint32_t)(page_hi(jlo + pe) - page_lo(jlo + pe));
+                    my_rank[r] = rk;
+                    spos[rk] = (uint32_t)(page_hi(jlo + pe) - page_lo(jlo + pe));
                 }
             }
             __syncthreads();
@@ -507,68 +616,11 @@ quest_select(const float *scores, const int64_t *seq_off, int P_shift, int k, in
                     for (int64_t i = page_lo(j); i < page_hi(j); ++i)
                         row[pos++] = (int32_t)i;
                 }
-        } else {
-            // general path
-            uint32_t prefix = 0u, pmask = 0u, above = 0u;
-            for (int pass = 0; pass < 3; ++pass) {
-                const int psh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-                const uint32_t pdm = pass == 2 ? 1023u : 2047u;
-                for (int i = tid; i < kQuestSelBins; i += blockDim.x)
-                    hist[i] = 0u;
-                __syncthreads();
-                for_each_key(sc + jlo, nc, [&](int64_t, uint32_t key) {
-                    if ((key & pmask) == prefix)
-                        atomicAdd(&hist[(key >> psh) & pdm], 1u);
-                });
-                __syncthreads();
-                const int top = (int)pdm;
-                const int d1 = top - 2 * tid, d2 = d1 - 1;
-                const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
-                uint32_t tot;
-                const uint32_t before = above + cta_exclusive_scan(h1 + h2, warp_sums, &tot);
-                if (d1 >= 0 && before < (uint32_t)take && before + h1 >= (uint32_t)take) {
-                    s_digit = (uint32_t)d1;
-                    s_above = before;
-                } else if (d2 >= 0 && before + h1 < (uint32_t)take && before + h1 + h2 >= (uint32_t)take) {
-                    s_digit = (uint32_t)d2;
-                    s_above = before + h1;
-                }
-                __syncthreads();
-                prefix |= s_digit << psh;
-                pmask |= pdm << psh;
-                above = s_above;
-                __syncthreads();
-            }
-            const uint32_t T = prefix, need = (uint32_t)take - above;
-            const int64_t R = (nc + blockDim.x - 1) / blockDim.x;
-            const int64_t c0 = (int64_t)tid * R, c1 = c0 + R < nc ? c0 + R : nc;
-            uint32_t eq = 0u;
-            for (int64_t c = c0; c < c1; ++c)
-                eq += score_key(sc[jlo + c]) == T ? 1u : 0u;
-            uint32_t unused;
-            const uint32_t eq_rank = cta_exclusive_scan(eq, warp_sums, &unused);
-            uint32_t ntok = 0u;
-            {
-                uint32_t rank = eq_rank;
-                for (int64_t c = c0; c < c1; ++c) {
-                    const uint32_t key = score_key(sc[jlo + c]);
-                    if (key > T || (key == T && rank++ < need))
-                        ntok += (uint32_t)(page_hi(jlo + c) - page_lo(jlo + c));
-                }
-            }
-            uint32_t pos = (uint32_t)s_end + cta_exclusive_scan(ntok, warp_sums, &total_tok);
-            {
-                uint32_t rank = eq_rank;
-                for (int64_t c = c0; c < c1; ++c) {
-                    const uint32_t key = score_key(sc[jlo + c]);
-                    if (key > T || (key == T && rank++ < need))
-                        for (int64_t i = page_lo(jlo + c); i < page_hi(jlo + c); ++i)
-                            row[pos++] = (int32_t)i;
-                }
-            }
         }
+    } else if (rank != 0) {
+        return;   // nothing to choose: rank 0 writes the windows
     }
-    // the windows, the count and the padding
+    // (rank 0) the windows, the count and the padding
     const int64_t m = s_end + total_tok + (n - l0);
     for (int64_t i = tid; i < s_end; i += blockDim.x)
         row[i] = (int32_t)i;
@@ -684,9 +736,10 @@ cudaError_t launch_quest_score(const Plan &p, const ts_kv_t *kv, const void *q, 
 cudaError_t launch_quest_select(const Plan &p, const ts_kv_t *kv, const float *scores, int page_size, int k,
                                 int n_sink, int n_local, int32_t *ids, int32_t *count, cudaStream_t st)
 {
-    quest_select<<<p.B, kQuestSelThreads, 0, st>>>(scores, kv->seq_offsets_dev, log2_exact(page_size), k, n_sink,
-                                                   n_local, k + n_sink + n_local, ids, count);
-    return cudaGetLastError();
+    // one cluster of kQSelCluster CTAs per sequence
+    return launch_ex(quest_select, dim3(kQSelCluster, (unsigned)p.B), dim3(kQuestSelThreads), 0, st, kQSelCluster,
+                     scores, kv->seq_offsets_dev, log2_exact(page_size), k, n_sink, n_local, k + n_sink + n_local, ids,
+                     count);
 }
 
 }  // namespace ts
