@@ -480,10 +480,10 @@ TS_API ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page
  * count[b] = their number (at most s' + k + (n - l0)); ids[b][count..) = -1.
  *   scores      from ts_quest_score (all ts_quest_rows entries readable)
  *   ids         device int32 [batch][k + n_sink + n_local]; count int32 [batch]
- * One CTA per sequence; no workspace.  The usual case (at most 2048 chosen
- * pages, at most 2048 pages in the threshold's radix bucket) reads the
- * scores three times; heavy ties or larger budgets take a general path that
- * reads them five times.
+ * One cluster of 8 CTAs per sequence (the pages split among them); no
+ * workspace.  The usual case (at most 2048 chosen pages, at most 2048 pages
+ * tied in the threshold's bin) reads the scores three times; heavy ties or
+ * larger budgets take a general path on one CTA that reads them five times.
  */
 TS_API ts_status_t ts_quest_select(const ts_kv_t *kv, const float *scores, int32_t page_size, int32_t k,
                                    int32_t n_sink, int32_t n_local, int32_t *ids, int32_t *count, void *stream);
