@@ -181,3 +181,39 @@ def test_paged_cache_arguments_are_checked_on_the_host(lib):
     assert b"page_table_stride" in lib.ts_last_error()
     assert lib.ts_decode_step_kernels(ctypes.byref(kv(4096, 1, 1 << 19)), 16, 4, 8) == -1
     assert b"2^31" in lib.ts_last_error()
+
+
+def test_split_and_comparator_arguments_are_checked_on_the_host(lib):
+    """The page-level comparator's and the token split's entry points reject
+    bad arguments on the host, before any device query or launch."""
+    lib.ts_last_error.restype = ctypes.c_char_p
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    off1 = (ctypes.c_int64 * 2)(0, 500)
+    off2 = (ctypes.c_int64 * 3)(0, 500, 900)
+    one = _KV(1, 8, 4, 64, ctypes.addressof(off1), ctypes.addressof(off1), 16, 16, 256, 64, 0.0, 0)
+    two = _KV(2, 8, 4, 64, ctypes.addressof(off2), ctypes.addressof(off2), 16, 16, 256, 64, 0.0, 0)
+    lib.ts_quest_rows.restype = I64
+    lib.ts_quest_rows.argtypes = [ctypes.POINTER(_KV), I32]
+    for page in (0, 3, 8192):
+        assert lib.ts_quest_rows(ctypes.byref(one), page) == -1 and b"page_size" in lib.ts_last_error()
+    assert lib.ts_quest_rows(None, 16) == -1
+    lib.ts_merge_normalisers.argtypes = [P, I32, I64, P, P]
+    assert lib.ts_merge_normalisers(None, 2, 8, None, None) == 1
+    lib.ts_merge_attention.argtypes = [P, P, I32, I64, I32, P, P]
+    assert lib.ts_merge_attention(None, None, 2, 8, 64, None, None) == 1
+    lib.ts_score_normalisers.argtypes = [ctypes.POINTER(_KV), P, P, P, P, SZ, P]
+    assert lib.ts_score_normalisers(ctypes.byref(one), None, None, None, None, 0, None) == 1
+    assert b"L_out" in lib.ts_last_error()
+    lib.ts_select_candidates.argtypes = [ctypes.POINTER(_KV), P, I32, I32, I32, I64, I64, P, P, P, P, SZ, P]
+    # k < 1; a batch of two sequences; a shard reaching past the sequence
+    assert lib.ts_select_candidates(ctypes.byref(one), None, 0, 4, 8, 0, 500, None, None, None, None, 0, None) == 1
+    assert lib.ts_select_candidates(ctypes.byref(two), None, 16, 4, 8, 0, 900, None, None, None, None, 0, None) == 1
+    assert b"batch 1" in lib.ts_last_error()
+    assert lib.ts_select_candidates(ctypes.byref(one), None, 16, 4, 8, 600, 1000, None, None, None, None, 0,
+                                    None) == 1
+    assert b"must lie in the sequence" in lib.ts_last_error()
+    lib.ts_select_merge.argtypes = [ctypes.POINTER(_KV), P, I32, I32, I32, I32, I32, I64, I64, P, P, P]
+    # rank outside [0, parts)
+    assert lib.ts_select_merge(ctypes.byref(one), None, 2, 2, 16, 4, 8, 0, 1000, None, None, None) == 1
+    lib.ts_sparse_attn_lse.argtypes = [ctypes.POINTER(_KV), P, P, P, I32, P, P, P, SZ, P]
+    assert lib.ts_sparse_attn_lse(ctypes.byref(one), None, None, None, 0, None, None, None, 0, None) == 1
