@@ -70,6 +70,9 @@ def parse_args(argv=None):
     ap.add_argument("--comparator-page", type=int, default=16,
                     help="page size of the page-level comparator (Quest's min/max page bounds) measured beside "
                          "the token-level path (0: not measured)")
+    ap.add_argument("--paged-page", type=int, default=16,
+                    help="page size of the paged-cache measurement: the same layers read through a block table "
+                         "of scattered pages, timed beside the packed cache (0: not measured)")
     ap.add_argument("--eager-steps", type=int, default=None,
                     help="profiler capture mode: after set-up, run this many decode steps of the workload as "
                          "plain (not graph-replayed) C-ABI calls, along the workload's query sequence, and exit "
@@ -497,6 +500,72 @@ def measure_comparator(wl, P: int, one, peak: float, peak_kind: str) -> dict:
     return res
 
 
+def scattered_page_table(lengths, P: int, rng):
+    """Block table of a pool that holds exactly the sequences' pages of P
+    tokens, each sequence's pages at distinct pool pages drawn as one random
+    permutation of the pool: int32 [B, max pages], unused entries 0.  None
+    when a length is not a multiple of P (the pool is then not the packed
+    cache)."""
+    lengths = np.asarray(lengths, np.int64)
+    if P <= 0 or np.any(lengths % P):
+        return None
+    pages = lengths // P
+    perm = rng.permutation(int(pages.sum())).astype(np.int32)
+    table = np.zeros((lengths.size, max(1, int(pages.max()))), np.int32)
+    o = 0
+    for b, c in enumerate(pages):
+        table[b, :c] = perm[o:o + c]
+        o += c
+    return table
+
+
+def measure_paged(wl, P: int, one) -> dict:
+    """The same layers as a paged cache (pages of P tokens): the packed K and
+    V tensors serve as the pool and each layer's block table scatters every
+    sequence's pages over it at random, as in a serving pool, so no copy is
+    made (the paged sequence is the packed one with its pages permuted, the
+    same amount of work).  Timed beside the packed cache, every layer-step
+    scored afresh (the selection cache off) on both: the scoring scan alone,
+    the whole one-call step, and the attention gather alone."""
+    ts, cfg = wl.ts, wl.cfg
+    res = {"page_size": P, "table": "one random permutation of the pool's pages per layer (seeded)"}
+    rng = np.random.default_rng(20240)
+    pkvs = []
+    for l in range(cfg.layers):
+        table = scattered_page_table(wl.lengths, P, rng)
+        if table is None:
+            res["skipped"] = "a sequence length is not a multiple of the page size"
+            return res
+        t = torch.from_numpy(table).to(wl.device)
+        pkvs.append([ts.KVCache(c.k, c.v, wl.layers[l].seq_offsets, cfg.h_q, page_table=t, page_size=P)
+                     for c in wl.kvs[l]])
+    kvs = {"packed": wl.kvs, "paged": pkvs}
+    bufs = {"packed": wl.bufs, "paged": [ts.StepBuffers(c[0], cfg.k, cfg.n_sink, cfg.n_local) for c in pkvs]}
+
+    def fresh_step(name, l, i):
+        b = bufs[name][l]
+        ts.ts_decode_step(kvs[name][l][i % wl.rotate], wl.q[l][i % wl.T], b.q_prev, b.reuse, True, 2.0, b.k,
+                          b.n_sink, b.n_local, b.votes, b.ids, b.count, b.out, b.ws, b.cos)
+
+    for name in kvs:                 # eager first calls (kernel attributes, tensor maps) before any capture
+        for l in range(cfg.layers):
+            fresh_step(name, l, 0)
+    torch.cuda.synchronize()
+    for key in ("score_pass_a_us", "step_us", "sparse_attn_us"):
+        res[key] = {}
+    for name in kvs:
+        kv_, bf = kvs[name], bufs[name]
+        res["score_pass_a_us"][name] = 1e6 * one(
+            lambda i: [ts.ts_score_logits(kv_[l][i % wl.rotate], wl.q[l][i % wl.T], None, bf[l].ws)
+                       for l in range(cfg.layers)])
+        res["step_us"][name] = 1e6 * one(lambda i: [fresh_step(name, l, i) for l in range(cfg.layers)])
+        res["sparse_attn_us"][name] = 1e6 * one(
+            lambda i: [ts.ts_sparse_attn(kv_[l][i % wl.rotate], wl.q[l][i % wl.T], bf[l].ids, bf[l].count,
+                                         bf[l].out, bf[l].ws) for l in range(cfg.layers)])
+    del bufs["paged"]
+    return res
+
+
 def run_ours(a, d: Dist):
     torch.cuda.set_device(d.local)
     dev = torch.device("cuda", d.local)
@@ -588,6 +657,8 @@ def run_ours(a, d: Dist):
     comparator = None
     if a.comparator_page:
         comparator = measure_comparator(wl, a.comparator_page, one, peak, peak_kind)
+
+    paged = measure_paged(wl, a.paged_page, one) if a.paged_page else None
 
     # ---- end to end: pinned host query in, result out, every step ----
     q_host = [q.cpu().pin_memory() for q in wl.q]
@@ -691,6 +762,8 @@ def run_ours(a, d: Dist):
     if comparator is not None:
         comparator["tokenselect_layer_step_us"] = ms_per_step * 1000.0 / cfg.layers
         result["comparator"] = comparator
+    if paged is not None:
+        result["paged"] = paged
     if d.world == 1 and not a.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, 4.0)

@@ -9,6 +9,7 @@ import sys
 import time
 import types
 
+import numpy as np
 import pytest
 
 import bench
@@ -161,3 +162,20 @@ def test_selection_recall():
     assert bench.selection_recall(row, 5, []) == 1.0
     assert bench.parse_args([]).comparator_page == 16
     assert bench.parse_args(["--comparator-page", "0"]).comparator_page == 0
+
+
+def test_scattered_page_table():
+    """The paged measurement's block table: every pool page used exactly once,
+    each sequence's own pages in its row, unused entries 0; lengths that are
+    not multiples of the page size give no table."""
+    rng = np.random.default_rng(3)
+    lengths = np.array([64, 16, 0, 48])
+    t = bench.scattered_page_table(lengths, 16, rng)
+    assert t.dtype == np.int32 and t.shape == (4, 4)
+    used = np.concatenate([t[b, :n // 16] for b, n in enumerate(lengths)])
+    assert sorted(used.tolist()) == list(range(8))
+    assert not t[1, 1:].any() and not t[2].any() and not t[3, 3:].any()
+    assert bench.scattered_page_table(np.array([64, 20]), 16, rng) is None
+    assert bench.scattered_page_table(lengths, 0, rng) is None
+    big = bench.scattered_page_table(np.array([1 << 20]), 16, np.random.default_rng(1))
+    assert big.shape == (1, 65536) and np.array_equal(np.sort(big[0]), np.arange(65536))
