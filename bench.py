@@ -73,6 +73,9 @@ def parse_args(argv=None):
     ap.add_argument("--paged-page", type=int, default=16,
                     help="page size of the paged-cache measurement: the same layers read through a block table "
                          "of scattered pages, timed beside the packed cache (0: not measured)")
+    ap.add_argument("--split-parts", default="2,4,8",
+                    help="shard counts of the token-axis split of one sequence timed on this GPU (rank 0's "
+                         "phases; batch-1 workloads whose shards exceed L2; empty: not measured)")
     ap.add_argument("--eager-steps", type=int, default=None,
                     help="profiler capture mode: after set-up, run this many decode steps of the workload as "
                          "plain (not graph-replayed) C-ABI calls, along the workload's query sequence, and exit "
@@ -85,6 +88,12 @@ def parse_args(argv=None):
         a.warmup = 3 if a.impl == "reference" else (10 if big else 50)
     if a.warmup < 3:
         raise SystemExit("at least 3 warm-up steps are required")
+    try:
+        parts = [int(x) for x in a.split_parts.split(",") if x.strip()]
+    except ValueError:
+        raise SystemExit("--split-parts must be a comma-separated list of shard counts")
+    if any(not 1 <= r <= 64 for r in parts):
+        raise SystemExit("--split-parts: shard counts must be in [1, 64]")
     if a.layers is not None and not 1 <= a.layers <= W.CONFIGS[a.workload].layers:
         raise SystemExit("--layers must be in [1, %d] for %s" % (W.CONFIGS[a.workload].layers, a.workload))
     return a
@@ -566,6 +575,72 @@ def measure_paged(wl, P: int, one) -> dict:
     return res
 
 
+def shard_bounds(n: int, parts: int):
+    """Equal contiguous shards of n tokens over `parts` ranks: [t_r, t_{r+1})."""
+    return [n * r // parts for r in range(parts + 1)]
+
+
+def measure_split(wl, parts_list, one) -> dict:
+    """The token-axis split of one sequence (query_aware_kv_ts_b200.split) on
+    this GPU: every layer's sequence cut into R equal shards (views of the
+    packed cache), one emulated step run to fill every shard's gathered
+    buffers (all shards' phases, the all-gathers as copies), then rank 0's
+    phases alone timed over the layers, in total and phase by phase: one
+    rank's compute per layer-step, the three all-gathers not included."""
+    from query_aware_kv_ts_b200 import split
+    ts, cfg = wl.ts, wl.cfg
+    res = {"what": "rank 0's phases per layer-step, exchanges excluded; equal shards; each phase alone and "
+                   "all five in order",
+           "phases": ["normalisers (pass A + merge)", "votes (normaliser join + pass B)",
+                      "candidates (shard selection + keys)", "select_and_attend (key merge + attention with lse)",
+                      "join (attention merge)"]}
+    if cfg.batch != 1:
+        res["skipped"] = "the split shards one sequence (batch 1)"
+        return res
+    if wl.k_bytes * cfg.layers // max(parts_list) < 4 * L2_BYTES:
+        res["skipped"] = "one rank's shards of all layers fit in L2 at the largest shard count"
+        return res
+    n = int(wl.lengths[0])
+    res["per_parts"] = {}
+    for R in parts_list:
+        bounds = shard_bounds(n, R)
+        shards = []
+        for l in range(cfg.layers):
+            kv = wl.kvs[l][0]
+            row = []
+            for r in range(R):
+                t0, t1 = bounds[r], bounds[r + 1]
+                skv = ts.KVCache(kv.k[t0:t1], kv.v[t0:t1], np.array([0, t1 - t0]), cfg.h_q)
+                row.append((skv, split.ShardBuffers(skv, cfg.k, cfg.n_sink, cfg.n_local, R), t0))
+            shards.append(row)
+        for l in range(cfg.layers):
+            split.emulate_split_decode_step(shards[l], wl.q[l][0], n)
+        torch.cuda.synchronize()
+
+        def phase(name, l):
+            kv, b, t = shards[l][0]
+            q = wl.q[l][0]
+            if name == "normalisers":
+                split.phase_normalisers(kv, q, b)
+            elif name == "votes":
+                split.phase_votes(kv, b)
+            elif name == "candidates":
+                split.phase_candidates(kv, b, t, n)
+            elif name == "select_and_attend":
+                split.phase_select_and_attend(kv, q, b, 0, t, n)
+            else:
+                split.phase_join_attention(b)
+
+        names = ["normalisers", "votes", "candidates", "select_and_attend", "join"]
+        per = {"shard_tokens": bounds[1] - bounds[0], "phases_us": {}}
+        for name in names:
+            per["phases_us"][name] = 1e6 * one(lambda i: [phase(name, l) for l in range(cfg.layers)])
+        per["rank_compute_us"] = 1e6 * one(lambda i: [phase(nm, l) for l in range(cfg.layers) for nm in names])
+        res["per_parts"][str(R)] = per
+        del shards
+    return res
+
+
 def run_ours(a, d: Dist):
     torch.cuda.set_device(d.local)
     dev = torch.device("cuda", d.local)
@@ -659,6 +734,10 @@ def run_ours(a, d: Dist):
         comparator = measure_comparator(wl, a.comparator_page, one, peak, peak_kind)
 
     paged = measure_paged(wl, a.paged_page, one) if a.paged_page else None
+    split_parts = [int(x) for x in a.split_parts.split(",") if x.strip()]
+    split_res = measure_split(wl, split_parts, one) if split_parts else None
+    if split_res is not None and paged is not None and "step_us" in paged:
+        split_res["one_gpu_fresh_step_us"] = paged["step_us"]["packed"]
 
     # ---- end to end: pinned host query in, result out, every step ----
     q_host = [q.cpu().pin_memory() for q in wl.q]
@@ -764,6 +843,8 @@ def run_ours(a, d: Dist):
         result["comparator"] = comparator
     if paged is not None:
         result["paged"] = paged
+    if split_res is not None:
+        result["split"] = split_res
     if d.world == 1 and not a.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, 4.0)

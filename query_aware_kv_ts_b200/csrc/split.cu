@@ -26,6 +26,7 @@ namespace {
 constexpr int kJoinThreads = 256;
 constexpr int kSelMergeThreads = 1024;
 constexpr int kSelMergeBins = 2048;   // 11-bit digits of the 64-bit keys
+constexpr int kSelMergeBatch = 8;     // keys a thread loads per round trip
 
 // L = log(sum_r exp(L_r)) per entry, in float64 (an entry of -inf is a shard
 // with no tokens).
@@ -100,8 +101,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
 
 // The sequence's threshold and this rank's row.  keys: [parts][kcap] (every
 // rank's list, this rank's at `rank`, ascending by id); k: the sequence's
-// budget.  T = the k-th largest key of all (a six-digit radix select over the
-// 64-bit keys), or the smallest nonzero key when there are at most k.  The
+// budget.  T: a key such that exactly k keys are >= T (a radix select over
+// the 64-bit keys, six digits at most), or 1 when there are at most k nonzero
+// keys (every one is chosen).  The
 // row: the shard's sink part [0, s_loc), its own keys >= T (as shard-local
 // ids, ascending), its local-window part [n_loc - l_loc, n_loc); -1 after.
 __global__ void __launch_bounds__(kSelMergeThreads)
@@ -110,35 +112,71 @@ select_merge(const unsigned long long *keys, int parts, int kcap, int k, int ran
 {
     __shared__ uint32_t hist[kSelMergeBins];
     __shared__ uint32_t warp_sums[32];
-    __shared__ uint32_t s_digit, s_above, s_nonzero;
+    __shared__ uint32_t s_digit, s_above, s_bin, s_nonzero;
     const int tid = threadIdx.x;
     const int64_t total = (int64_t)parts * kcap;
+    for (int i = tid; i < kSelMergeBins; i += blockDim.x)
+        hist[i] = 0u;
     if (tid == 0)
         s_nonzero = 0u;
     __syncthreads();
+    unsigned long long prefix = 0ull, pmask = 0ull;
     uint32_t nz = 0u;
-    for (int64_t i = tid; i < total; i += blockDim.x)
-        nz += __ldcg(keys + i) != 0ull ? 1u : 0u;
-    atomicAdd(&s_nonzero, nz);
+    // Histogram of the digit (key >> sh) & dmask of the nonzero keys under the
+    // current prefix, counting the nonzero keys too when asked.  The keys are
+    // read in trips of kSelMergeBatch independent loads per thread (one memory
+    // round trip per trip, not per key), with the same loop bounds for the
+    // whole block (the warp-wide match needs every lane); a warp adds each
+    // distinct digit once with its multiplicity: the high digits of the top
+    // candidates' votes fall into a few bins, on which one shared atomic per
+    // lane would serialise.
+    auto histogram = [&](int sh, uint32_t dmask, bool count_nonzero) {
+        const int64_t per_trip = (int64_t)blockDim.x * kSelMergeBatch;
+        for (int64_t base = 0; base < total; base += per_trip) {
+            unsigned long long kk[kSelMergeBatch];
+#pragma unroll
+            for (int u = 0; u < kSelMergeBatch; ++u) {
+                const int64_t i = base + (int64_t)u * blockDim.x + tid;
+                kk[u] = i < total ? __ldcg(keys + i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kSelMergeBatch; ++u) {
+                if (count_nonzero)
+                    nz += kk[u] != 0ull ? 1u : 0u;
+                const bool take = kk[u] != 0ull && (kk[u] & pmask) == prefix;
+                const uint32_t bin = take ? (uint32_t)(kk[u] >> sh) & dmask : 0xffffffffu;
+                const unsigned grp = __match_any_sync(0xffffffffu, bin);
+                if (take && __ffs(grp) - 1 == (int)(tid & 31))
+                    atomicAdd(&hist[bin], (uint32_t)__popc(grp));
+            }
+        }
+    };
+    // the first digit's histogram in the same trips as the count
+    histogram(53, 0x7ffu, true);
+    nz = __reduce_add_sync(0xffffffffu, nz);
+    if ((tid & 31) == 0)
+        atomicAdd(&s_nonzero, nz);
     __syncthreads();
     const uint32_t real = s_nonzero;
     unsigned long long T = 1ull;   // at most k keys: every nonzero key
     if (real > (uint32_t)k && k > 0) {
-        unsigned long long prefix = 0ull, pmask = 0ull;
+        // the k-th largest key lies among the nonzero ones: digits from the
+        // top, until the chosen digit's bin holds exactly the keys still
+        // needed (then every key under the prefix is chosen and the prefix
+        // with its lower bits 0 is the threshold), at the latest at the last
+        // digit (keys are distinct: its bin holds the k-th key alone)
         uint32_t above = 0u;
         for (int pass = 0; pass < 6; ++pass) {
             const int sh = pass < 5 ? 53 - 11 * pass : 0;
             const int width = pass < 5 ? 11 : 9;
             const uint32_t dmask = (1u << width) - 1u;
-            for (int i = tid; i < kSelMergeBins; i += blockDim.x)
-                hist[i] = 0u;
-            __syncthreads();
-            for (int64_t i = tid; i < total; i += blockDim.x) {
-                const unsigned long long key = __ldcg(keys + i);
-                if ((key & pmask) == prefix)
-                    atomicAdd(&hist[(uint32_t)(key >> sh) & dmask], 1u);
+            if (pass > 0) {
+                for (int i = tid; i < kSelMergeBins; i += blockDim.x)
+                    hist[i] = 0u;
+                __syncthreads();
+                histogram(sh, dmask, false);
+                __syncthreads();
             }
-            __syncthreads();
             const int top = (int)dmask;
             const int d1 = top - 2 * tid, d2 = d1 - 1;
             const uint32_t h1 = d1 >= 0 ? hist[d1] : 0u, h2 = d2 >= 0 ? hist[d2] : 0u;
@@ -147,17 +185,22 @@ select_merge(const unsigned long long *keys, int parts, int kcap, int k, int ran
             if (d1 >= 0 && before < (uint32_t)k && before + h1 >= (uint32_t)k) {
                 s_digit = (uint32_t)d1;
                 s_above = before;
+                s_bin = h1;
             } else if (d2 >= 0 && before + h1 < (uint32_t)k && before + h1 + h2 >= (uint32_t)k) {
                 s_digit = (uint32_t)d2;
                 s_above = before + h1;
+                s_bin = h2;
             }
             __syncthreads();
             prefix |= (unsigned long long)s_digit << sh;
             pmask |= (unsigned long long)dmask << sh;
             above = s_above;
+            const bool whole_bin = s_above + s_bin == (uint32_t)k;
             __syncthreads();
+            if (whole_bin)
+                break;
         }
-        T = prefix;   // keys are distinct: exactly k are >= T
+        T = prefix;   // exactly k keys are >= T
     } else if (k == 0) {
         T = ~0ull;    // nothing chosen (no key reaches it: the id field is never all ones)
     }

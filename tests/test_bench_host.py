@@ -179,3 +179,16 @@ def test_scattered_page_table():
     assert bench.scattered_page_table(lengths, 0, rng) is None
     big = bench.scattered_page_table(np.array([1 << 20]), 16, np.random.default_rng(1))
     assert big.shape == (1, 65536) and np.array_equal(np.sort(big[0]), np.arange(65536))
+
+
+def test_split_shards_and_arguments():
+    """Equal contiguous shards cover the sequence exactly; bad shard counts
+    are refused."""
+    for n, r in [(1 << 20, 8), (10, 3), (5, 5), (7, 1)]:
+        b = bench.shard_bounds(n, r)
+        assert b[0] == 0 and b[-1] == n and len(b) == r + 1
+        assert all(0 <= y - x <= -(-n // r) for x, y in zip(b, b[1:]))
+    assert bench.parse_args(["--split-parts", ""]).split_parts == ""
+    for bad in ("0", "2,x", "65"):
+        with pytest.raises(SystemExit):
+            bench.parse_args(["--split-parts", bad])
