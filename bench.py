@@ -441,8 +441,9 @@ def selection_recall(ids: np.ndarray, count: int, want) -> float:
 def measure_comparator(wl, P: int, one, peak: float, peak_kind: str) -> dict:
     """The page-level comparator (Quest's min/max page bounds, pages of P
     tokens) on the same layers, queries and selection budget as the
-    token-level path: per-layer times of its kernels alone (the metadata pass,
-    which a serving loop runs once per page, apart), the score kernel's
+    token-level path: per-layer times of its kernels alone (the full metadata
+    pass, and the update of the newest token's page that a decode loop runs
+    per token, apart), the score kernel's
     bandwidth, and on layer 0 how many planted query-aligned keys each method
     selects and how much of the token-level selection the page selection
     covers."""
@@ -475,6 +476,10 @@ def measure_comparator(wl, P: int, one, peak: float, peak_kind: str) -> dict:
     res["metadata_us"] = 1e6 * one(lambda i: [ts.ts_quest_metadata(kv_of(l, i)[0], P, kv_of(l, i)[1].kmin,
                                                                     kv_of(l, i)[1].kmax)
                                               for l in range(cfg.layers)])
+    # a decode loop's per-token cost: the page that took the newest token
+    res["metadata_update_us"] = 1e6 * one(
+        lambda i: [ts.ts_quest_metadata_update(kv_of(l, i)[0], P, 1, kv_of(l, i)[1].kmin, kv_of(l, i)[1].kmax)
+                   for l in range(cfg.layers)])
     res["score_us"] = 1e6 * one(lambda i: [score(l, i) for l in range(cfg.layers)])
     res["select_us"] = 1e6 * one(lambda i: [select(l, i) for l in range(cfg.layers)])
     res["sparse_attn_us"] = 1e6 * one(lambda i: [attn(l, i) for l in range(cfg.layers)])

@@ -449,9 +449,23 @@ TS_API int64_t ts_quest_rows(const ts_kv_t *kv, int32_t page_size);
  * the page's tokens of K[token][g][c].
  *   kmin, kmax   device bf16 [ts_quest_rows][h_kv][head_dim] each, 16-byte
  *                aligned (caller-owned); only the rows of pages are written
- * Reads K once; a growing cache's metadata is recomputed by calling again.
+ * Reads K once.
  */
 TS_API ts_status_t ts_quest_metadata(const ts_kv_t *kv, int32_t page_size, void *kmin, void *kmax, void *stream);
+
+/*
+ * Page metadata of the newest tokens only: the rows of every page that holds
+ * one of a sequence's last last_tokens tokens are recomputed from all the
+ * page's tokens, as ts_quest_metadata computes them; every other row is left
+ * as it is.  The current lengths are read from seq_offsets_dev on the
+ * device, so after ts_append_kv (one token: last_tokens = 1) the call
+ * updates the page that took the token, also inside a captured graph.
+ *   last_tokens  >= 1 (a value above a sequence's length covers all of it)
+ *   kmin, kmax   as for ts_quest_metadata, holding the other pages' rows
+ * Reads at most (floor(last_tokens / P) + 2) * P tokens of K per sequence.
+ */
+TS_API ts_status_t ts_quest_metadata_update(const ts_kv_t *kv, int32_t page_size, int64_t last_tokens, void *kmin,
+                                            void *kmax, void *stream);
 
 /*
  * Page scores [Quest, Method Overview (4)]: with scale as in ts_score and

@@ -87,6 +87,7 @@ _SIGS = {
     "ts_merge_attention": (ctypes.c_int, [_P, _P, _I32, ctypes.c_int64, _I32, _P, _P]),
     "ts_quest_rows": (ctypes.c_int64, [_KV, _I32]),
     "ts_quest_metadata": (ctypes.c_int, [_KV, _I32, _P, _P, _P]),
+    "ts_quest_metadata_update": (ctypes.c_int, [_KV, _I32, ctypes.c_int64, _P, _P, _P]),
     "ts_quest_score": (ctypes.c_int, [_KV, _P, _I32, _P, _P, _P, _P]),
     "ts_quest_select": (ctypes.c_int, [_KV, _P, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "ts_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -325,6 +326,11 @@ def ts_quest_rows(kv: KVCache, page_size: int) -> int:
 
 def ts_quest_metadata(kv: KVCache, page_size: int, kmin, kmax, stream=None):
     _check(_lib.ts_quest_metadata(kv.ref(), int(page_size), _ptr(kmin), _ptr(kmax), _stream(stream)))
+
+
+def ts_quest_metadata_update(kv: KVCache, page_size: int, last_tokens: int, kmin, kmax, stream=None):
+    _check(_lib.ts_quest_metadata_update(kv.ref(), int(page_size), int(last_tokens), _ptr(kmin), _ptr(kmax),
+                                         _stream(stream)))
 
 
 def ts_quest_score(kv: KVCache, q, page_size: int, kmin, kmax, scores, stream=None):

@@ -1116,6 +1116,27 @@ ts_status_t ts_quest_metadata(const ts_kv_t *kv, int32_t page_size, void *kmin, 
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "quest metadata launch");
 }
 
+ts_status_t ts_quest_metadata_update(const ts_kv_t *kv, int32_t page_size, int64_t last_tokens, void *kmin,
+                                     void *kmax, void *stream)
+{
+    if (last_tokens < 1) {
+        set_error("last_tokens %lld must be at least 1", (long long)last_tokens);
+        return TS_ERR_INVALID_ARG;
+    }
+    Plan p;
+    ts_status_t s = quest_prologue(kv, page_size, 1, &p);
+    if (s != TS_OK)
+        return s;
+    if (kmin == nullptr || kmax == nullptr ||
+        ((reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) & 15u)) {
+        set_error("kmin and kmax are required and must be 16-byte aligned");
+        return TS_ERR_INVALID_ARG;
+    }
+    cudaError_t e =
+        launch_quest_meta(p, kv, page_size, kmin, kmax, static_cast<cudaStream_t>(stream), last_tokens);
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "quest metadata update launch");
+}
+
 ts_status_t ts_quest_score(const ts_kv_t *kv, const void *q, int32_t page_size, const void *kmin, const void *kmax,
                            float *scores, void *stream)
 {

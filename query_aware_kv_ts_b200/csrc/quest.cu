@@ -85,18 +85,22 @@ __device__ __forceinline__ uint4 bf16x8_max(uint4 x, uint4 y)
 // Page metadata: one warp per page.  Lane l owns the 16-byte chunks l,
 // l + 32, ... (CH of them) of the h_kv * d channels of a token row; the
 // warp's lanes look up the rows of 32 tokens at a time and walk them, U
-// tokens' loads in flight.
+// tokens' loads in flight.  last_tokens > 0: only the pages holding one of
+// the sequence's last last_tokens tokens (its current length read here, so
+// that the update follows appends made on the device), each recomputed
+// from all its tokens.
 // ---------------------------------------------------------------------------
 template <int CH>
 __global__ void __launch_bounds__(kQuestWarps * 32)
-quest_meta(const QuestKV a, __nv_bfloat16 *kmin, __nv_bfloat16 *kmax)
+quest_meta(const QuestKV a, __nv_bfloat16 *kmin, __nv_bfloat16 *kmax, int64_t last_tokens)
 {
     constexpr int U = 8 / CH;
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t off0 = a.seq_off[b];
     const int64_t n = a.seq_off[b + 1] - off0;
-    const int64_t j = (int64_t)blockIdx.x * kQuestWarps + warp;   // page of the sequence
+    const int64_t j_first = last_tokens > 0 ? max((int64_t)0, n - last_tokens) >> a.P_shift : 0;
+    const int64_t j = j_first + (int64_t)blockIdx.x * kQuestWarps + warp;   // page of the sequence
     const int64_t t0 = j << a.P_shift;
     if (t0 >= n)
         return;
@@ -675,23 +679,25 @@ int64_t quest_rows(const Plan &p, int page_size)
 }
 
 cudaError_t launch_quest_meta(const Plan &p, const ts_kv_t *kv, int page_size, void *kmin, void *kmax,
-                              cudaStream_t st)
+                              cudaStream_t st, int64_t last_tokens)
 {
     const QuestKV a = make_quest_kv(p, kv, page_size);
-    const int64_t max_pages = (p.n_max + page_size - 1) / page_size;
+    int64_t max_pages = (p.n_max + page_size - 1) / page_size;
+    if (last_tokens > 0)   // the last t tokens span at most floor(t / P) + 2 pages
+        max_pages = min(max_pages, last_tokens / page_size + 2);
     const dim3 grid((unsigned)((max_pages + kQuestWarps - 1) / kQuestWarps), (unsigned)p.B);
     if (max_pages == 0)
         return cudaSuccess;
     __nv_bfloat16 *lo = static_cast<__nv_bfloat16 *>(kmin), *hi = static_cast<__nv_bfloat16 *>(kmax);
     switch (chunks_per_lane(p)) {
     case 1:
-        quest_meta<1><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        quest_meta<1><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi, last_tokens);
         break;
     case 2:
-        quest_meta<2><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        quest_meta<2><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi, last_tokens);
         break;
     default:
-        quest_meta<4><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi);
+        quest_meta<4><<<grid, kQuestWarps * 32, 0, st>>>(a, lo, hi, last_tokens);
         break;
     }
     return cudaGetLastError();

@@ -226,8 +226,9 @@ cudaError_t launch_merge_attention(const float *o_parts, const float *lse_parts,
 // Page-level comparator (quest.cu): rows of the page metadata and scores,
 // page j of sequence b at row (seq_offsets[b] >> log2 P) + b + j.
 int64_t quest_rows(const Plan &p, int page_size);
+// last_tokens > 0: only the pages holding the sequences' last last_tokens tokens
 cudaError_t launch_quest_meta(const Plan &p, const ts_kv_t *kv, int page_size, void *kmin, void *kmax,
-                              cudaStream_t st);
+                              cudaStream_t st, int64_t last_tokens = 0);
 cudaError_t launch_quest_score(const Plan &p, const ts_kv_t *kv, const void *q, int page_size, const void *kmin,
                                const void *kmax, float *scores, cudaStream_t st);
 cudaError_t launch_quest_select(const Plan &p, const ts_kv_t *kv, const float *scores, int page_size, int k,

@@ -197,6 +197,12 @@ def test_split_and_comparator_arguments_are_checked_on_the_host(lib):
     for page in (0, 3, 8192):
         assert lib.ts_quest_rows(ctypes.byref(one), page) == -1 and b"page_size" in lib.ts_last_error()
     assert lib.ts_quest_rows(None, 16) == -1
+    lib.ts_quest_metadata_update.argtypes = [ctypes.POINTER(_KV), I32, I64, P, P, P]
+    for last in (0, -5):
+        assert lib.ts_quest_metadata_update(ctypes.byref(one), 16, last, None, None, None) == 1
+        assert b"last_tokens" in lib.ts_last_error()
+    assert lib.ts_quest_metadata_update(ctypes.byref(one), 3, 1, None, None, None) == 1
+    assert b"page_size" in lib.ts_last_error()
     lib.ts_merge_normalisers.argtypes = [P, I32, I64, P, P]
     assert lib.ts_merge_normalisers(None, 2, 8, None, None) == 1
     lib.ts_merge_attention.argtypes = [P, P, I32, I64, I32, P, P]

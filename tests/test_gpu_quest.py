@@ -226,3 +226,57 @@ def test_quest_rejects_bad_page_sizes():
     for P in (0, 3, 8192):
         with pytest.raises(m.TsError, match="page_size"):
             m.ts_quest_rows(kv, P)
+
+
+@pytest.mark.parametrize("P", [1, 16, 64])
+def test_metadata_update_follows_appends(P):
+    """ts_quest_metadata_update on a growing cache (one sequence, capacity
+    mode): after every appended token (last_tokens = 1), after a run of
+    appended tokens updated at once (last_tokens = the run's length), and in
+    a replayed graph of [append, update], every page row of the current
+    length equals the oracle's metadata of the tokens so far, exactly."""
+    m = H.ts()
+    n0, T, h_kv, d, h_q = 1000, 70, 4, 128, 28
+    k, v = W.random_kv(n0 + T, h_kv, d, 99 + P, device="cuda")
+    kbuf, vbuf = torch.zeros_like(k), torch.zeros_like(v)
+    kbuf[:n0], vbuf[:n0] = k[:n0], v[:n0]
+    kv = m.KVCache(kbuf, vbuf, np.array([0, n0]), h_q, capacity=n0 + T)
+    buf = m.StepBuffers(kv, 64, 4, 16)          # the append's workspace
+    qbuf = m.QuestBuffers(kv, P)
+    m.ts_quest_metadata(kv, P, qbuf.kmin, qbuf.kmax)
+    kb = W.bf16_bits(k)
+
+    def check(n):
+        torch.cuda.synchronize()
+        assert int(kv.seq_offsets_dev[1].item()) == n
+        pages = oracle.quest_pages(n, P)
+        want_lo, want_hi = oracle.quest_meta(kb[:n], P)
+        assert np.array_equal(_f(W.bf16_bits(qbuf.kmin)[:pages]), _f(want_lo)), n
+        assert np.array_equal(_f(W.bf16_bits(qbuf.kmax)[:pages]), _f(want_hi)), n
+
+    check(n0)
+    n = n0
+    for t in range(20):                          # one token at a time
+        m.ts_append_kv(kv, k[n], v[n], buf.ws)
+        m.ts_quest_metadata_update(kv, P, 1, qbuf.kmin, qbuf.kmax)
+        n += 1
+        if t % 5 == 4:
+            check(n)
+    for _ in range(17):                          # a run, updated at once
+        m.ts_append_kv(kv, k[n], v[n], buf.ws)
+        n += 1
+    m.ts_quest_metadata_update(kv, P, 17, qbuf.kmin, qbuf.kmax)
+    check(n)
+    k_new, v_new = torch.empty_like(k[0]), torch.empty_like(v[0])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.ts_append_kv(kv, k_new, v_new, buf.ws)
+        m.ts_quest_metadata_update(kv, P, 1, qbuf.kmin, qbuf.kmax)
+    torch.cuda.synchronize()
+    while n < n0 + T:                            # the graph, replayed
+        k_new.copy_(k[n])
+        v_new.copy_(v[n])
+        g.replay()
+        n += 1
+    check(n)
+    del g
