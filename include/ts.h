@@ -360,15 +360,19 @@ TS_API ts_status_t ts_selftest_expire_wait(void *ws, size_t ws_bytes, uint32_t s
  * ---------------------------------------------------------------------------
  */
 
-/* Score pass A and the normaliser merge on the shard (ts_score_logits), then
- * L_out[b][h] = log sum_i exp(s[h][i]) over the shard's tokens (float64,
- * device [batch][h_q]; -inf for an empty sequence). */
+/* Score pass A and the normaliser merge on the shard (ts_score_logits), the
+ * merge writing L_out[b][h] = log sum_i exp(s[h][i]) over the shard's tokens
+ * (float64, device [batch][h_q]): every entry -inf when the shard holds no
+ * token; in a batch of several sequences, the rows of a sequence that
+ * reuses (reuse[b] != 0) or is empty are left as they were.  The
+ * workspace's own normalisers are not written. */
 TS_API ts_status_t ts_score_normalisers(const ts_kv_t *kv, const void *q, const int32_t *reuse, double *L_out,
                                         void *ws, size_t ws_bytes, void *stream);
 
 /* Score pass B with given normalisers: votes[i] = sum_h exp(s[h][i] - L_in[b][h])
  * for the logits of the last ts_score_normalisers / ts_score_logits call on
- * this workspace (L_in: device float64 [batch][h_q]). */
+ * this workspace (L_in: device float64 [batch][h_q], read in place by the
+ * kernel). */
 TS_API ts_status_t ts_score_vote_normalised(const ts_kv_t *kv, const int32_t *reuse, const double *L_in,
                                             float *votes, void *ws, size_t ws_bytes, void *stream);
 

@@ -527,8 +527,10 @@ static ts_status_t score_prologue(const ts_kv_t *kv, void *ws, size_t ws_bytes, 
     return TS_OK;
 }
 
-ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reuse, void *ws, size_t ws_bytes,
-                            void *stream)
+// Pass A and the normaliser merge, the merge writing L to L_out (null: the
+// workspace, where pass B reads it).
+static ts_status_t score_logits_to(const ts_kv_t *kv, const void *q, const int32_t *reuse, void *ws,
+                                   size_t ws_bytes, void *stream, double *L_out)
 {
     Plan p;
     ts_status_t s = score_prologue(kv, ws, ws_bytes, &p);
@@ -545,8 +547,14 @@ ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reu
     if (s != TS_OK)
         return s;
     cudaError_t e = launch_score(p, kmap, q, kv->seq_offsets_dev, kv->seq_offsets_host, reuse, static_cast<uint8_t *>(ws),
-                                 static_cast<cudaStream_t>(stream), kv->page_table_dev, kv->page_table_stride);
+                                 static_cast<cudaStream_t>(stream), kv->page_table_dev, kv->page_table_stride, L_out);
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass A launch");
+}
+
+ts_status_t ts_score_logits(const ts_kv_t *kv, const void *q, const int32_t *reuse, void *ws, size_t ws_bytes,
+                            void *stream)
+{
+    return score_logits_to(kv, q, reuse, ws, ws_bytes, stream, nullptr);
 }
 
 ts_status_t ts_score_vote(const ts_kv_t *kv, const int32_t *reuse, float *votes, void *ws, size_t ws_bytes,
@@ -917,21 +925,20 @@ ts_status_t ts_score_normalisers(const ts_kv_t *kv, const void *q, const int32_t
         set_error("L_out is required");
         return TS_ERR_INVALID_ARG;
     }
-    ts_status_t s = ts_score_logits(kv, q, reuse, ws, ws_bytes, stream);
+    // the merge writes L_out itself (no copy between kernels: the chain keeps
+    // its programmatic launches)
+    ts_status_t s = score_logits_to(kv, q, reuse, ws, ws_bytes, stream, L_out);
     if (s != TS_OK)
         return s;
     Plan p;
     s = make_plan(kv, -1, &p);
     if (s != TS_OK)
         return s;
-    const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (p.n_total == 0)   // nothing scored: every L is -inf (a merge of no parts)
-        e = launch_merge_normalisers(nullptr, 0, (int64_t)p.B * p.Hq, L_out, st);
-    else
-        e = cudaMemcpyAsync(L_out, static_cast<uint8_t *>(ws) + p.off_L, sizeof(double) * p.B * p.Hq,
-                            cudaMemcpyDeviceToDevice, st);
-    return e == cudaSuccess ? TS_OK : cuda_fail(e, "normalisers copy");
+    if (p.n_total != 0)
+        return TS_OK;
+    // nothing scored: every L is -inf (a merge of no parts)
+    cudaError_t e = launch_merge_normalisers(nullptr, 0, (int64_t)p.B * p.Hq, L_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : cuda_fail(e, "normalisers launch");
 }
 
 ts_status_t ts_score_vote_normalised(const ts_kv_t *kv, const int32_t *reuse, const double *L_in, float *votes,
@@ -947,11 +954,8 @@ ts_status_t ts_score_vote_normalised(const ts_kv_t *kv, const int32_t *reuse, co
     }
     if (p.n_total == 0)
         return TS_OK;
-    const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(static_cast<uint8_t *>(ws) + p.off_L, L_in, sizeof(double) * p.B * p.Hq,
-                                    cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess)
-        e = launch_vote(p, kv->seq_offsets_dev, reuse, votes, static_cast<uint8_t *>(ws), st);
+    cudaError_t e = launch_vote(p, kv->seq_offsets_dev, reuse, votes, static_cast<uint8_t *>(ws),
+                                static_cast<cudaStream_t>(stream), nullptr, L_in);
     return e == cudaSuccess ? TS_OK : cuda_fail(e, "score pass B launch");
 }
 

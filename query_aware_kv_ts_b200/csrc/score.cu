@@ -744,7 +744,7 @@ cudaError_t launch_score_t(const Plan &p, const CUtensorMap &kmap, ScoreArgs arg
 
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
                          const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st,
-                         const int32_t *page_table, int page_table_stride)
+                         const int32_t *page_table, int page_table_stride, double *L_out)
 {
     ScoreArgs a;
     for (int b = 0; b <= 32; ++b)
@@ -786,7 +786,7 @@ cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, 
         return e;
     const float2 *parts = reinterpret_cast<const float2 *>(ws + p.off_partials);
     const int32_t *table = reinterpret_cast<const int32_t *>(ws + p.off_chunk_table);
-    double *Lp = reinterpret_cast<double *>(ws + p.off_L);
+    double *Lp = L_out != nullptr ? L_out : reinterpret_cast<double *>(ws + p.off_L);
     const dim3 mgrid((unsigned)p.Hq, (unsigned)p.B);
     const int S = p.score_grid + p.B;
     switch (p.score_partials_per_slot) {

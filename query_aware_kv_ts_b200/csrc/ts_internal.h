@@ -175,9 +175,10 @@ cudaError_t launch_selcache(const void *q, void *q_prev, int32_t *reuse, double 
 // seq_off_host: the host copy of the offsets (prefetch hints before the
 // dependency wait; the device copy decides the work).
 // page_table, page_table_stride: the block table of a paged cache (p.paged).
+// L_out: where the normaliser merge writes L (null: the workspace).
 cudaError_t launch_score(const Plan &p, const CUtensorMap &kmap, const void *q, const int64_t *seq_off,
                          const int64_t *seq_off_host, const int32_t *reuse, uint8_t *ws, cudaStream_t st,
-                         const int32_t *page_table = nullptr, int page_table_stride = 0);
+                         const int32_t *page_table = nullptr, int page_table_stride = 0, double *L_out = nullptr);
 
 // Selection parameters, for the vote pass that also builds the selection's
 // level-1 histogram.
@@ -185,8 +186,9 @@ struct SelectWindow {
     int k, n_sink, n_local;
 };
 
+// L_in: the normalisers to use instead of the workspace's (null: the workspace's)
 cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
-                        cudaStream_t st, const SelectWindow *hist_window = nullptr);
+                        cudaStream_t st, const SelectWindow *hist_window = nullptr, const double *L_in = nullptr);
 
 // Logits, normalisers and votes in one cooperative kernel, one kv-head group
 // at a time (kmap_head: boxes of {64 channels, 128 tokens, 1 head}); with a

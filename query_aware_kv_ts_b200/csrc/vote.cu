@@ -276,14 +276,14 @@ vote_pass_b(const VoteArgs a)
 }  // namespace
 
 cudaError_t launch_vote(const Plan &p, const int64_t *seq_off, const int32_t *reuse, float *votes, uint8_t *ws,
-                        cudaStream_t st, const SelectWindow *hist_window)
+                        cudaStream_t st, const SelectWindow *hist_window, const double *L_in)
 {
     if (p.n_max <= 0)
         return cudaSuccess;
     VoteArgs a;
     a.logits = reinterpret_cast<const float *>(ws + p.off_logits);
     a.ld = p.ld_logits;
-    a.L = reinterpret_cast<const double *>(ws + p.off_L);
+    a.L = L_in != nullptr ? L_in : reinterpret_cast<const double *>(ws + p.off_L);
     a.seq_off = seq_off;
     a.reuse = reuse;
     a.votes = votes;
