@@ -21,6 +21,14 @@ afresh, plus the gathered K and V rows of every layer-step) over the timed
 region's duration; which layer-steps reused their selection is read back from
 a replay of exactly the timed sequence of steps.
 
+Beside the main line, each measured after the timed region: `kernels` (each
+kernel alone), `comparator` (the page-level comparator after Quest on the
+same layers: its kernels, the per-token metadata update, recall),
+`paged` (the same layers read through a scattered block table of 16-token
+pages, beside the packed cache), `split` (the token-axis split of one
+sequence: one rank's phases at R = 2, 4, 8, exchanges excluded) and `e2e`
+(every step's queries in and outputs out through pinned host memory).
+
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 (the path has no cross-sequence exchange); the timed region is bracketed by
 barriers and the elapsed time is the max over ranks.
