@@ -280,3 +280,44 @@ def test_metadata_update_follows_appends(P):
         n += 1
     check(n)
     del g
+
+
+@pytest.mark.parametrize("P", [8, 16, 64])
+def test_metadata_update_on_a_paged_batch(P):
+    """ts_quest_metadata_update on a paged KV cache of several ragged
+    sequences (one of them empty, one shorter than a page): after the rows of
+    every page are overwritten with junk, an update over each sequence's
+    last 2P tokens rewrites exactly the pages those tokens lie in, bit for
+    bit as the full metadata pass computes them, and leaves every other row
+    as it was."""
+    from test_gpu_paged import _paged
+    lengths, h_q, h_kv, d = [3000, 77, 0, 5, 4100], 28, 4, 128
+    off = W.seq_offsets(lengths)
+    kk, vv = W.random_kv(int(off[-1]), h_kv, d, 11, device="cuda")
+    kp, vp, table = _paged(kk, vv, off, 16, seed=12)
+    m = H.ts()
+    kv = m.KVCache(kp, vp, off, h_q, page_table=table, page_size=16)
+    full = m.QuestBuffers(kv, P)
+    m.ts_quest_metadata(kv, P, full.kmin, full.kmax)
+    upd = m.QuestBuffers(kv, P)
+    upd.kmin.fill_(7.0)
+    upd.kmax.fill_(-7.0)
+    m.ts_quest_metadata_update(kv, P, 2 * P, upd.kmin, upd.kmax)
+    torch.cuda.synchronize()
+    want_lo, want_hi = full.kmin.cpu().view(torch.int16), full.kmax.cpu().view(torch.int16)
+    got_lo, got_hi = upd.kmin.cpu().view(torch.int16), upd.kmax.cpu().view(torch.int16)
+    junk_lo = torch.full(got_lo[0].shape, 7.0, dtype=torch.bfloat16).view(torch.int16)
+    junk_hi = torch.full(got_hi[0].shape, -7.0, dtype=torch.bfloat16).view(torch.int16)
+    updated = set()
+    for b, n in enumerate(lengths):
+        if n == 0:
+            continue
+        r0 = int(off[b]) // P + b
+        first, last = max(0, n - 2 * P) // P, (n - 1) // P
+        for j in range(first, last + 1):
+            updated.add(r0 + j)
+            assert torch.equal(got_lo[r0 + j], want_lo[r0 + j]) and torch.equal(got_hi[r0 + j], want_hi[r0 + j]), \
+                (b, j)
+    for r in range(upd.rows):
+        if r not in updated:
+            assert torch.equal(got_lo[r], junk_lo) and torch.equal(got_hi[r], junk_hi), r
