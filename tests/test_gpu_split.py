@@ -97,3 +97,30 @@ def test_split_equals_one_gpu_step():
         assert all(abs(v1[i] - thr) <= 1e-6 * thr for i in diff), diff
     assert np.allclose(votes, buf.votes.cpu().numpy()[:n], rtol=1e-5, atol=1e-30)
     assert float((out - buf.out).abs().max()) <= H.OUT_ATOL
+
+
+def test_normalisers_of_a_batch_with_reuse_and_an_empty_sequence():
+    """ts_score_normalisers on a batch of several sequences: the merge writes
+    every fresh, nonempty sequence's per-head log-normalisers straight into
+    L_out (against the oracle's, 1e-4 absolute: a vote's relative error is
+    about the normaliser's absolute one), and leaves the rows of the
+    sequence that reuses and of the empty one as they were."""
+    lengths, h_q, h_kv, d = [2000, 0, 1500, 700], 28, 4, 128
+    off = W.seq_offsets(lengths)
+    kk, vv = W.random_kv(int(off[-1]), h_kv, d, 21, device="cuda")
+    q = torch.randn((len(lengths), h_q, d), generator=torch.Generator().manual_seed(22)).to(torch.bfloat16).cuda()
+    m = H.ts()
+    kv = m.KVCache(kk, vv, off, h_q)
+    buf = m.StepBuffers(kv, 64, 4, 16)
+    reuse = torch.tensor([0, 0, 1, 0], dtype=torch.int32, device="cuda")
+    L_out = torch.full((len(lengths) * h_q,), 123.0, dtype=torch.float64, device="cuda")
+    m.ts_score_normalisers(kv, q, reuse, L_out, buf.ws)
+    torch.cuda.synchronize()
+    got = L_out.cpu().numpy().reshape(len(lengths), h_q)
+    kb, qb = W.bf16_bits(kk), W.bf16_bits(q)
+    for b, n in enumerate(lengths):
+        if n == 0 or b == 2:
+            assert np.all(got[b] == 123.0), b
+            continue
+        _, L_ref = oracle.votes(kb[int(off[b]):int(off[b + 1])], qb[b])
+        assert np.abs(got[b] - L_ref).max() <= 1e-4, (b, np.abs(got[b] - L_ref).max())
