@@ -124,3 +124,34 @@ def test_normalisers_of_a_batch_with_reuse_and_an_empty_sequence():
             continue
         _, L_ref = oracle.votes(kb[int(off[b]):int(off[b + 1])], qb[b])
         assert np.abs(got[b] - L_ref).max() <= 1e-4, (b, np.abs(got[b] - L_ref).max())
+
+
+def test_split_rank_with_nothing_selected():
+    """A middle shard whose keys are all zero (logits 0, below the other
+    shards' top votes), outside the sink and local windows: its rank selects
+    no token at all (count 0, log-sum-exp -inf), and the join leaves it out;
+    the joined selection and output still follow the oracle."""
+    n, h_q, h_kv, d, k, s, l = 3000, 8, 2, 128, 16, 4, 16
+    lens = [1000, 1000, 1000]
+    kk, vv = W.random_kv(n, h_kv, d, 31, device="cuda")
+    kk[1000:2000] = 0
+    q = torch.randn((1, h_q, d), generator=torch.Generator().manual_seed(32)).to(torch.bfloat16).cuda()
+    m = H.ts()
+    from query_aware_kv_ts_b200 import split
+    shards, t = [], 0
+    for ln in lens:
+        kv = m.KVCache(kk[t:t + ln], vv[t:t + ln], np.array([0, ln]), h_q)
+        shards.append((kv, split.ShardBuffers(kv, k, s, l, len(lens)), t))
+        t += ln
+    out = split.emulate_split_decode_step(shards, q, n)
+    torch.cuda.synchronize()
+    assert int(shards[1][1].step.count.cpu()[0]) == 0
+    assert torch.isinf(shards[1][1].lse).all() and (shards[1][1].lse < 0).all()
+    kb, vb, qb = W.bf16_bits(kk), W.bf16_bits(vv), W.bf16_bits(q)[0]
+    votes = np.concatenate([b.step.votes.cpu().numpy()[:kv.n_total] for kv, b, _ in shards])
+    union = np.array(sorted(int(x) + t for kv, b, t in shards
+                            for x in b.step.ids.cpu().numpy()[0][:int(b.step.count.cpu()[0])]), np.int32)
+    want, m_ = oracle.select(votes.astype(np.float64), k, s, l)
+    assert union.size == m_ and np.array_equal(union, want[:m_])
+    o_ref = oracle.sparse_attn(kb, vb, qb, union, union.size)
+    assert float(np.abs(out.cpu().numpy()[0] - o_ref).max()) <= H.OUT_ATOL
