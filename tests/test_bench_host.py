@@ -192,3 +192,21 @@ def test_split_shards_and_arguments():
     for bad in ("0", "2,x", "65"):
         with pytest.raises(SystemExit):
             bench.parse_args(["--split-parts", bad])
+
+
+def test_paged_and_split_measurements_skip_where_they_do_not_apply():
+    """The paged measurement needs every length to be a multiple of the page
+    size (the packed cache is then the pool); the split one shards a single
+    sequence and needs its shards to exceed L2.  Both say why they skip,
+    before touching a device."""
+    cfg = types.SimpleNamespace(layers=2, batch=2, h_q=8, k=16, n_sink=4, n_local=8)
+    wl = types.SimpleNamespace(ts=None, cfg=cfg, lengths=np.array([100, 37]), k_bytes=1 << 20, layers=[None] * 2,
+                               kvs=[[None], [None]])
+    r = bench.measure_paged(wl, 16, one=None)
+    assert r["page_size"] == 16 and "multiple of the page size" in r["skipped"]
+    r = bench.measure_split(wl, [2, 4, 8], one=None)
+    assert "one sequence" in r["skipped"] and "per_parts" not in r
+    wl.cfg = types.SimpleNamespace(**{**vars(cfg), "batch": 1})
+    wl.lengths = np.array([4096])
+    r = bench.measure_split(wl, [2, 4, 8], one=None)
+    assert "fit in L2" in r["skipped"]
